@@ -1,0 +1,290 @@
+"""fp64 CPU oracle for the sparse-attention hot path.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this package.  The CUDA library
+(``sparse_attention_07_b200``) never imports, links or calls it, and the two
+share no code: the only module both read is ``workloads`` (seeded inputs, no
+arithmetic of the method).
+
+The heavy loops live in ``sa_oracle.c`` (plain C, double precision, built by
+``build()`` below with gcc + OpenMP over independent queries).  This file
+converts inputs to float64 (bf16, fp8 e4m3 and fp32 values are all exact in
+fp64; the conversion is torch's CPU cast), looks up pages, and holds the small
+numpy helpers the pins use.  Each function cites the passage it follows:
+
+  [Notes]  "Sparse Attention 数学学习笔记" (echobase-5bl.pages.dev, 2026.09.14)
+  [MLA-S]  "MLA 与稀疏注意力：少存一点，还是少看一点？" (tianyi-zhang-02.github.io)
+  [Ch11]   "第 11 章 稀疏注意力" (book.shippingwang.com)
+  [LLMRes] "LLM注意力优化：稀疏注意力" (wln20.github.io)
+
+Parity status: every function here is pinned by a test in
+``tests/test_oracle_pins.py``; none is "parity unpinned", except the block
+selection of near-tied blocks, which fp64 and fp32 may order differently (the
+GPU tests accept a differing block only when its score is within the stated
+tolerance of the boundary score).
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import subprocess
+from typing import Optional, Sequence
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "sa_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "libsa_oracle.so")
+_lib = None
+
+PAGE = 64
+
+
+def build(force: bool = False) -> str:
+    """Compile sa_oracle.c into libsa_oracle.so (gcc -O2 -fopenmp)."""
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11",
+                               "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        P = ctypes.c_void_p
+        I = ctypes.c_int
+        I64 = ctypes.c_int64
+        D = ctypes.c_double
+        lib.sa_oracle_index_scores.argtypes = [I, I, I, P, P, P, P, P, P, I64]
+        lib.sa_oracle_topk.argtypes = [I, P, I64, P, I, P]
+        lib.sa_oracle_sparse_mla.argtypes = [I, I, I, I, P, P, P, P, P, I, D, P, P]
+        lib.sa_oracle_block_mean_pool.argtypes = [I, I, I, P, P]
+        lib.sa_oracle_block_sparse.argtypes = [I, I, I, I, I, I, D, P, P, P, P, P, P]
+        lib.sa_oracle_threads.restype = I
+        _lib = lib
+    return _lib
+
+
+def threads() -> int:
+    """Host threads the C oracle runs on (OpenMP)."""
+    return int(_load().sa_oracle_threads())
+
+
+def _f64(a) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _i64(a) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(a, dtype=np.int64))
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+# --------------------------------------------------------------------------
+# C-backed definitions
+
+def index_scores(q, w, keys, key0, n_vis, out_ld: Optional[int] = None) -> np.ndarray:
+    """Lightning-indexer scores, [Notes] §9 (I_{t,s}) / [MLA-S] DSA section.
+
+    q [rows,H_I,d_I], w [rows,H_I], keys [n_keys,d_I] (each sequence in logical
+    order), key0[r] = index in ``keys`` of the row's position 0, n_vis[r] =
+    visible positions.  Returns [rows, out_ld] float64; entries s >= n_vis[r]
+    are NaN.
+    """
+    q, w, keys = _f64(q), _f64(w), _f64(keys)
+    key0, n_vis = _i64(key0), _i64(n_vis)
+    rows, H_I, d_I = q.shape
+    out_ld = int(out_ld if out_ld is not None else (n_vis.max() if rows else 0))
+    out = np.full((rows, max(out_ld, 1)), np.nan)
+    _load().sa_oracle_index_scores(rows, H_I, d_I, _ptr(q), _ptr(w), _ptr(keys), _ptr(key0),
+                                   _ptr(n_vis), _ptr(out), out.shape[1])
+    return out[:, :out_ld]
+
+
+def topk(scores, n_valid, k: int) -> np.ndarray:
+    """Exact Top-K, [Notes] §9 and [MLA-S] ``selected_positions`` order.
+
+    Keeps the min(k, n) positions with the largest score, equal scores going to
+    the lower position; returns them ascending, padded with -1 to k.
+    """
+    s = _f64(scores)
+    if s.ndim == 1:
+        s = s[None]
+    n_valid = _i64(np.broadcast_to(np.asarray(n_valid), (s.shape[0],)))
+    out = np.empty((s.shape[0], k), dtype=np.int32)
+    _load().sa_oracle_topk(s.shape[0], _ptr(s), s.shape[1], _ptr(n_valid), k, _ptr(out))
+    return out
+
+
+def sparse_mla(q_lat, q_rope, c, kr, sel, scale: float):
+    """Sparse MLA latent attention, [MLA-S] full-score section + [Notes] §2/§8.
+
+    q_lat [rows,H,d_c] (absorbed), q_rope [rows,H,d_R], c [n,d_c], kr [n,d_R],
+    sel [rows,k] row of c/kr per selected slot (-1 = empty).  Returns
+    (out [rows,H,d_c] = sum_j a_j c_j, lse [rows,H] natural log).
+    """
+    q_lat, q_rope, c, kr = _f64(q_lat), _f64(q_rope), _f64(c), _f64(kr)
+    sel = _i64(sel)
+    rows, H, d_c = q_lat.shape
+    d_R = q_rope.shape[2]
+    k = sel.shape[1]
+    out = np.zeros((rows, H, d_c))
+    lse = np.zeros((rows, H))
+    _load().sa_oracle_sparse_mla(rows, H, d_c, d_R, _ptr(q_lat), _ptr(q_rope), _ptr(c), _ptr(kr),
+                                 _ptr(sel), k, float(scale), _ptr(out), _ptr(lse))
+    return out, lse
+
+
+def block_mean_pool(K, block: int) -> np.ndarray:
+    """Mean of each complete block of keys, [Ch11] §12.6 (k_blocks.mean)."""
+    K = _f64(K)
+    L, D = K.shape
+    out = np.zeros((L // block, D))
+    _load().sa_oracle_block_mean_pool(L, D, block, _ptr(K), _ptr(out))
+    return out
+
+
+def block_sparse(q, K, V, block: int, top_blocks: int, sink_blocks: int, window: int, scale: float):
+    """Block-sparse decode for one (sequence, head), [Ch11] §12.5-12.6 + [LLMRes] MoBA.
+
+    Returns (out [D], chosen blocks [top_blocks] ascending -1 padded,
+    block scores [L//block]).
+    """
+    q, K, V = _f64(q), _f64(K), _f64(V)
+    L, D = K.shape
+    out = np.zeros(D)
+    sel = np.empty(top_blocks, dtype=np.int32)
+    bs = np.zeros(max(L // block, 1))
+    _load().sa_oracle_block_sparse(L, D, block, top_blocks, sink_blocks, window, float(scale),
+                                   _ptr(q), _ptr(K), _ptr(V), _ptr(out), _ptr(sel), _ptr(bs))
+    return out, sel, bs[: L // block]
+
+
+# --------------------------------------------------------------------------
+# numpy helpers used by the pins
+
+def dense_attention(q, K, V, scale: float):
+    """[Notes] §1: o = sum_j softmax_j(q.k_j * scale) v_j over all positions."""
+    q, K, V = _f64(q), _f64(K), _f64(V)
+    s = K @ q * scale
+    a = np.exp(s - s.max())
+    a /= a.sum()
+    return a @ V, a
+
+
+def masked_attention(scores, values, visible):
+    """[Notes] §3: softmax(S + M) with M = 0 on the visible set, -inf elsewhere;
+    the mask enters before the softmax ([MLA-S] masked_scalar_attention)."""
+    s = _f64(scores)
+    vis = np.asarray(visible, dtype=bool)
+    if s.shape != vis.shape or not vis.any():
+        raise ValueError("expected equal lengths and at least one visible position")
+    m = np.where(vis, 0.0, -np.inf)
+    z = s + m
+    a = np.exp(z - z[vis].max())
+    a /= a.sum()
+    return float(a @ _f64(values))
+
+
+def absorb(U_K, q):
+    """[MLA-S] absorbed query: q^T U_K c = (U_K^T q)^T c."""
+    return _f64(U_K).T @ _f64(q)
+
+
+def dense_mass(alpha_dense, selected) -> float:
+    """[Notes] §6: Z_i = sum_{j in S_i} alpha_ij."""
+    a = _f64(alpha_dense)
+    return float(a[np.asarray(selected, dtype=np.int64)].sum())
+
+
+def error_bound(v_max: float, Z: float) -> float:
+    """[Notes] §6: ||o^dense - o^sparse|| <= 2 V_max (1 - Z_i)."""
+    return 2.0 * v_max * (1.0 - Z)
+
+
+# --------------------------------------------------------------------------
+# Whole-step reference on workload tensors (any device; values copied to host)
+
+def _host64(t):
+    import torch
+    return t.detach().to("cpu").to(torch.float64).numpy()
+
+
+def pool_rows(page_table, pages_per_seq: int, seq: int, positions) -> np.ndarray:
+    """Row of the page pool holding each logical position of ``seq``."""
+    pos = _i64(positions)
+    page = pos // PAGE
+    if page_table is None:
+        phys = seq * pages_per_seq + page
+    else:
+        phys = np.asarray(page_table)[seq, page].astype(np.int64)
+    return phys * PAGE + pos % PAGE
+
+
+def dsa_step(inp: dict, rows: Sequence[int], with_scores: bool = True) -> dict:
+    """Indexer -> Top-K -> sparse MLA for the chosen query rows of a workload.
+
+    ``inp`` is a dict made by ``workloads.dsa_inputs``.  Returns, per chosen
+    row (in the order given): ``scores`` [n_rows, L_max] (NaN past the visible
+    length), ``idx`` [n_rows, k] int32 and ``out`` [n_rows,H,d_c], ``lse``
+    [n_rows,H] float64.
+    """
+    import torch
+    cfg = inp["cfg"]
+    rows = [int(r) for r in rows]
+    table = None if inp["page_table"] is None else inp["page_table"].cpu().numpy()
+    pps = cfg.pages_per_seq
+    n_vis_all = inp["n_visible"].cpu().numpy().astype(np.int64)
+    sor = inp["seq_of_row"]
+    sor = np.arange(cfg.rows) if sor is None else sor.cpu().numpy().astype(np.int64)
+    seqs = sorted({int(sor[r]) for r in rows})
+    key_blocks, key0_of_seq, off = [], {}, 0
+    for s in seqs:
+        n = int(max(n_vis_all[r] for r in rows if sor[r] == s))
+        pr = torch.from_numpy(pool_rows(table, pps, s, np.arange(n)))
+        key_blocks.append(_host64(inp["k_idx_cache"][pr.to(inp["k_idx_cache"].device)]))
+        key0_of_seq[s] = off
+        off += n
+    keys = np.concatenate(key_blocks, axis=0) if key_blocks else np.zeros((0, cfg.d_I))
+    ridx = torch.tensor(rows, dtype=torch.long, device=inp["q_idx"].device)
+    q = _host64(inp["q_idx"][ridx])
+    w = _host64(inp["w"][ridx])
+    n_vis = np.array([n_vis_all[r] for r in rows], dtype=np.int64)
+    key0 = np.array([key0_of_seq[int(sor[r])] for r in rows], dtype=np.int64)
+    scores = index_scores(q, w, keys, key0, n_vis, out_ld=cfg.L_max)
+    idx = topk(np.nan_to_num(scores, nan=-np.inf), n_vis, cfg.topk)
+    # gather the selected latent rows of every chosen query row
+    sel = np.full(idx.shape, -1, dtype=np.int64)
+    flat = []
+    for i, r in enumerate(rows):
+        valid = idx[i] >= 0
+        pr = pool_rows(table, pps, int(sor[r]), idx[i][valid])
+        sel[i, valid] = np.arange(len(flat), len(flat) + len(pr))
+        flat.extend(pr.tolist())
+    fr = torch.tensor(flat, dtype=torch.long, device=inp["c_cache"].device)
+    c = _host64(inp["c_cache"][fr]) if flat else np.zeros((0, cfg.d_c))
+    kr = _host64(inp["kr_cache"][fr]) if flat else np.zeros((0, cfg.d_R))
+    out, lse = sparse_mla(_host64(inp["q_lat"][ridx]), _host64(inp["q_rope"][ridx]), c, kr, sel, cfg.scale)
+    res = dict(idx=idx, out=out, lse=lse, n_visible=n_vis)
+    if with_scores:
+        res["scores"] = scores
+    return res
+
+
+def block_step(inp: dict, pairs: Sequence[tuple]) -> dict:
+    """Block-sparse decode for chosen (sequence, head) pairs of a block workload."""
+    cfg = inp["cfg"]
+    outs, sels, scores = [], [], []
+    for b, h in pairs:
+        q = _host64(inp["q"][b, h])
+        K = _host64(inp["K"][b, :, h])
+        V = _host64(inp["V"][b, :, h])
+        o, s, bs = block_sparse(q, K, V, cfg.block, cfg.top_blocks, cfg.sink_blocks, cfg.window, cfg.scale)
+        outs.append(o); sels.append(s); scores.append(bs)
+    return dict(out=np.stack(outs), sel=np.stack(sels), block_scores=np.stack(scores))

@@ -1,0 +1,354 @@
+"""Pins for the fp64 oracle: the pages' worked examples, closed forms,
+invariants and library routines.  None of these compares the oracle with
+itself; each is chosen so that a dropped term, a wrong sign or index, or a
+transposed operand in the oracle fails at least one of them.
+
+CPU only.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+
+
+def _golden(golden_dir, name):
+    with open(os.path.join(golden_dir, name)) as f:
+        return json.load(f)
+
+
+# ---------------------------------------------------------------- MLA scores
+
+def test_absorbed_query_example(golden_dir):
+    """MLA-S "先看一条压缩后的表示": score -3 computed directly and via U_K^T q."""
+    g = _golden(golden_dir, "absorbed_score.json")
+    c, U, q = np.array(g["latent_c"]), np.array(g["U_K"]), np.array(g["query_q"])
+    assert (U @ c).tolist() == g["key_k"]
+    assert float(q @ (U @ c)) == g["score"]
+    qa = oracle.absorb(U, q)
+    assert qa.tolist() == g["absorbed_query"]
+    # the oracle's score path consumes the absorbed query; with one selected
+    # row and scale 1 its log-sum-exp is exactly that row's score
+    out, lse = oracle.sparse_mla(qa[None, None], np.zeros((1, 1, 1)), c[None], np.zeros((1, 1)),
+                                 np.array([[0]]), 1.0)
+    assert lse[0, 0] == g["score"]
+    assert out[0, 0].tolist() == c.tolist()      # one row: weight 1, output = that latent
+
+
+def test_absorbed_identity_random():
+    """q^T U_K c_j = (U_K^T q)^T c_j for every row: the oracle on the absorbed
+    query equals dense attention on the expanded keys k_j = U_K c_j (values c_j)."""
+    rng = np.random.default_rng(7)
+    d_k, d_c, n = 24, 16, 9
+    U = rng.standard_normal((d_k, d_c))
+    q = rng.standard_normal(d_k)
+    C = rng.standard_normal((n, d_c))
+    keys = C @ U.T
+    scale = 0.3
+    ref, _ = oracle.dense_attention(q, keys, C, scale)
+    out, _ = oracle.sparse_mla(oracle.absorb(U, q)[None, None], np.zeros((1, 1, 1)), C,
+                               np.zeros((n, 1)), np.arange(n)[None], scale)
+    np.testing.assert_allclose(out[0, 0], ref, rtol=0, atol=1e-12)
+
+
+def test_content_plus_position_example(golden_dir):
+    """MLA-S "分开以后": content 1,1 + RoPE 0,2, /sqrt(4) -> 0.5,1.5 -> 0.269,0.731."""
+    g = _golden(golden_dir, "content_position.json")
+    # latent rows are unit vectors, so the output is the weight vector itself
+    c = np.eye(2)
+    q_lat = np.array([[[1.0, 1.0]]])                 # content scores 1 and 1
+    q_rope = np.array([[[1.0]]])
+    kr = np.array([[0.0], [2.0]])                    # RoPE scores 0 and 2
+    out, lse = oracle.sparse_mla(q_lat, q_rope, c, kr, np.array([[0, 1]]), 1.0 / math.sqrt(g["total_dim"]))
+    w = out[0, 0]
+    assert np.round(w, g["printed_decimals"]).tolist() == g["weights_printed"]
+    # closed form: softmax of (0.5, 1.5) is (1/(1+e), e/(1+e))
+    np.testing.assert_allclose(w, [1 / (1 + math.e), math.e / (1 + math.e)], rtol=0, atol=1e-15)
+    np.testing.assert_allclose(lse[0, 0], math.log(math.exp(0.5) + math.exp(1.5)), atol=1e-15)
+
+
+def test_missed_position_example(golden_dir):
+    """MLA-S "稀疏注意力": 8 zero scores, value 8 at one position: dense 1, sparse 0."""
+    g = _golden(golden_dir, "missed_position.json")
+    n = g["n_positions"]
+    c = np.zeros((n, 1)); c[g["evidence_position"], 0] = g["evidence_value"]
+    q_lat = np.zeros((1, 1, 1)); q_rope = np.zeros((1, 1, 1)); kr = np.zeros((n, 1))
+    dense, _ = oracle.sparse_mla(q_lat, q_rope, c, kr, np.arange(n)[None], 1.0)
+    others = [j for j in range(n) if j != g["evidence_position"]]
+    sparse, _ = oracle.sparse_mla(q_lat, q_rope, c, kr, np.array([others]), 1.0)
+    assert dense[0, 0, 0] == pytest.approx(g["dense_output"], abs=1e-15)
+    assert sparse[0, 0, 0] == g["sparse_output_without_it"]
+
+
+def test_selected_positions_example(golden_dir):
+    """MLA-S "一次错选会丢掉什么？": Top-2 of [3,2,1,0] is [0,1]; the dense output
+    10e^4/(e^4+3) > 9 while the selection's output is 0."""
+    g = _golden(golden_dir, "selected_positions.json")
+    chosen = oracle.topk(np.array(g["index_scores"]), len(g["index_scores"]), g["count"])[0]
+    assert chosen.tolist() == g["chosen"]
+    n = len(g["values"])
+    c = np.array(g["values"])[:, None]               # value = latent row
+    kr = np.array(g["attention_scores"])[:, None]    # score carried by the RoPE branch
+    q_lat = np.zeros((1, 1, 1)); q_rope = np.ones((1, 1, 1))
+    dense, _ = oracle.sparse_mla(q_lat, q_rope, c, kr, np.arange(n)[None], 1.0)
+    sparse, _ = oracle.sparse_mla(q_lat, q_rope, c, kr, chosen[None].astype(np.int64), 1.0)
+    e4 = math.exp(4.0)
+    assert dense[0, 0, 0] == pytest.approx(10 * e4 / (e4 + 3), abs=1e-12)
+    assert dense[0, 0, 0] > g["dense_output_greater_than"]
+    assert sparse[0, 0, 0] == g["sparse_output"]
+
+
+def test_causal_mask_example(golden_dir):
+    """MLA-S causal check: masking before the softmax gives 3 for any future
+    score; the plausible mistake (masking after the softmax) gives 2 and then
+    below 0.001, so this pin tells the two apart."""
+    g = _golden(golden_dir, "causal_mask.json")
+    vals, vis = np.array(g["values"]), np.array(g["visible"])
+
+    def mask_after(scores):            # the mistake the page warns about, written here on purpose
+        a = np.exp(np.array(scores) - max(scores))
+        return float((a * vals * vis).sum() / a.sum())
+
+    for case in g["cases"]:
+        assert oracle.masked_attention(case["scores"], vals, vis) == case["mask_before"]
+        # the sparse-MLA oracle over the visible set S = {0, 1} agrees
+        c = vals[:2, None]; kr = np.array(case["scores"])[:2, None]
+        out, _ = oracle.sparse_mla(np.zeros((1, 1, 1)), np.ones((1, 1, 1)), c, kr, np.array([[0, 1]]), 1.0)
+        assert out[0, 0, 0] == case["mask_before"]
+        if "mask_after" in case:
+            assert mask_after(case["scores"]) == case["mask_after"]
+        else:
+            assert mask_after(case["scores"]) < case["mask_after_below"]
+
+
+def test_mask_form_equals_renormalisation():
+    """Notes §3 vs §2/§6: softmax(S + M) over all positions equals the dense
+    weights renormalised by Z on the chosen set, and the sparse-MLA oracle."""
+    rng = np.random.default_rng(11)
+    n, d = 40, 12
+    C = rng.standard_normal((n, d))
+    qc = rng.standard_normal(d)
+    scale = 0.37
+    S = np.sort(rng.choice(n, size=13, replace=False))
+    _, alpha = oracle.dense_attention(qc, C, C, scale)
+    Z = oracle.dense_mass(alpha, S)
+    renorm = (alpha[S, None] / Z * C[S]).sum(0)
+    vis = np.zeros(n, dtype=bool); vis[S] = True
+    mask_form = np.array([oracle.masked_attention(C @ qc * scale, C[:, j], vis) for j in range(d)])
+    out, _ = oracle.sparse_mla(qc[None, None], np.zeros((1, 1, 1)), C, np.zeros((n, 1)), S[None], scale)
+    np.testing.assert_allclose(mask_form, renorm, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(out[0, 0], renorm, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2, 3])
+def test_topk_error_bound(seed):
+    """Notes §6: ||o_dense - o_sparse|| <= 2 V_max (1 - Z) with V_max bounding every value."""
+    rng = np.random.default_rng(seed)
+    n, d = 64, 8
+    C = rng.standard_normal((n, d)) * rng.uniform(0.5, 3.0)
+    qc = rng.standard_normal(d)
+    S = np.sort(rng.choice(n, size=rng.integers(1, n), replace=False))
+    dense, alpha = oracle.dense_attention(qc, C, C, 1.0)
+    out, _ = oracle.sparse_mla(qc[None, None], np.zeros((1, 1, 1)), C, np.zeros((n, 1)), S[None], 1.0)
+    vmax = np.linalg.norm(C, axis=1).max()
+    Z = oracle.dense_mass(alpha, S)
+    assert np.linalg.norm(dense - out[0, 0]) <= oracle.error_bound(vmax, Z) + 1e-12
+
+
+def test_k_equals_L_is_dense_attention():
+    """Notes §1: selecting every position gives dense attention (torch softmax, fp64)."""
+    rng = np.random.default_rng(5)
+    n, H, d_c, d_R = 50, 3, 16, 4
+    q_lat, q_rope = rng.standard_normal((1, H, d_c)), rng.standard_normal((1, H, d_R))
+    C, KR = rng.standard_normal((n, d_c)), rng.standard_normal((n, d_R))
+    scale = 1 / math.sqrt(20)
+    out, lse = oracle.sparse_mla(q_lat, q_rope, C, KR, np.arange(n)[None], scale)
+    t = lambda a: torch.from_numpy(a)
+    s = (t(q_lat[0]) @ t(C).T + t(q_rope[0]) @ t(KR).T) * scale
+    ref = torch.softmax(s, dim=-1) @ t(C)
+    np.testing.assert_allclose(out[0], ref.numpy(), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse[0], torch.logsumexp(s, -1).numpy(), rtol=0, atol=1e-12)
+
+
+def test_sparse_mla_heads_independent_and_empty_slots():
+    """MLA-S: heads share the rows but not the distribution; -1 slots are skipped."""
+    rng = np.random.default_rng(9)
+    n, H, d_c, d_R = 20, 4, 8, 2
+    q_lat, q_rope = rng.standard_normal((1, H, d_c)), rng.standard_normal((1, H, d_R))
+    C, KR = rng.standard_normal((n, d_c)), rng.standard_normal((n, d_R))
+    sel = np.array([[3, 7, -1, 11, -1]])
+    out, lse = oracle.sparse_mla(q_lat, q_rope, C, KR, sel, 0.5)
+    for h in range(H):
+        ref, _ = oracle.dense_attention(np.concatenate([q_lat[0, h], q_rope[0, h]]),
+                                        np.concatenate([C, KR], 1)[[3, 7, 11]], C[[3, 7, 11]], 0.5)
+        np.testing.assert_allclose(out[0, h], ref, atol=1e-12)
+    empty_out, empty_lse = oracle.sparse_mla(q_lat, q_rope, C, KR, np.full((1, 3), -1), 0.5)
+    assert (empty_out == 0).all() and np.isneginf(empty_lse).all()
+
+
+# ------------------------------------------------------------------ indexer
+
+def test_index_score_hand_example():
+    """Notes §9 by hand: heads (1,2) and (-1,1), weights 0.5 and 2, key (3,-1):
+    dots 1 and -4, ReLU 1 and 0, score 0.5.  Key (-1,2): dots 3 and 3 -> 1.5 + 6."""
+    q = np.array([[[1.0, 2.0], [-1.0, 1.0]]])
+    w = np.array([[0.5, 2.0]])
+    keys = np.array([[3.0, -1.0], [-1.0, 2.0]])
+    s = oracle.index_scores(q, w, keys, [0], [2])
+    assert s[0].tolist() == [0.5, 7.5]
+
+
+def test_index_scores_vs_einsum_and_causal_bound():
+    """Random integer inputs against numpy einsum + maximum (a library routine);
+    positions past the visible length are not scored."""
+    rng = np.random.default_rng(3)
+    rows, H_I, d_I, n = 5, 6, 16, 300
+    q = rng.integers(-8, 9, size=(rows, H_I, d_I)).astype(float)
+    w = 2.0 ** rng.integers(-4, 2, size=(rows, H_I))
+    keys = rng.integers(-8, 9, size=(2 * n, d_I)).astype(float)
+    key0 = np.array([0, n, 0, n, n])
+    n_vis = np.array([n, n - 7, 1, 0, 123])
+    s = oracle.index_scores(q, w, keys, key0, n_vis, out_ld=n)
+    for r in range(rows):
+        K = keys[key0[r]: key0[r] + n_vis[r]]
+        ref = (np.maximum(np.einsum("hd,sd->sh", q[r], K), 0) * w[r]).sum(1)
+        assert np.array_equal(s[r, :n_vis[r]], ref)        # integers x 2^-4: exact
+        assert np.isnan(s[r, n_vis[r]:]).all()
+
+
+# --------------------------------------------------------------------- top-k
+
+def test_topk_selected_positions_example(golden_dir):
+    g = _golden(golden_dir, "selected_positions.json")
+    assert oracle.topk(g["index_scores"], 4, 2)[0].tolist() == g["chosen"]
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_topk_bruteforce_with_ties(seed):
+    """Brute force via numpy lexsort on (-score, position), ascending output."""
+    rng = np.random.default_rng(seed)
+    rows, n, k = 7, 97, 13
+    scores = rng.integers(-3, 4, size=(rows, n)).astype(float)       # many ties
+    n_valid = rng.integers(0, n + 1, size=rows)
+    got = oracle.topk(scores, n_valid, k)
+    for r in range(rows):
+        m = n_valid[r]
+        order = np.lexsort((np.arange(m), -scores[r, :m]))
+        want = np.sort(order[: min(k, m)])
+        assert got[r, : len(want)].tolist() == want.tolist()
+        assert (got[r, len(want):] == -1).all()
+
+
+def test_topk_degenerate_cases():
+    eq = oracle.topk(np.zeros((1, 50)), 50, 8)[0]
+    assert eq.tolist() == list(range(8))                 # all equal: lowest positions
+    few = oracle.topk(np.arange(5.0)[None], 5, 8)[0]
+    assert few.tolist() == [0, 1, 2, 3, 4, -1, -1, -1]   # k > n: all, then -1
+    none = oracle.topk(np.zeros((1, 4)), 0, 3)[0]
+    assert none.tolist() == [-1, -1, -1]
+    neg = oracle.topk(np.array([[-1.0, -0.0, 0.0, -5.0]]), 4, 2)[0]
+    assert neg.tolist() == [1, 2]                        # -0 == +0: tie to lower
+
+
+# -------------------------------------------------------------- block-sparse
+
+def test_block_toy_example(golden_dir):
+    """Ch11 §12.5: n=16, B=4; choosing blocks {0 (sink), 1} reads tokens 0-7.
+    The oracle is steered so block 1 is the top-1 block; with one sink block
+    and no window its output is dense attention over tokens 0-7."""
+    g = _golden(golden_dir, "block_toy.json")
+    rng = np.random.default_rng(1)
+    n, B, d = g["n"], g["B"], 8
+    K = rng.standard_normal((n, d)) * 0.1
+    V = rng.standard_normal((n, d))
+    q = np.ones(d)
+    K[4:8] += 1.0                                        # block 1 has the largest mean key
+    out, sel, bs = oracle.block_sparse(q, K, V, B, 1, 1, 0, d ** -0.5)
+    assert sel.tolist() == [1]
+    toks = [t for b in g["selected_blocks"] for t in range(g["block_tokens"][b][0], g["block_tokens"][b][1] + 1)]
+    assert toks == g["tokens_read"]
+    ref, _ = oracle.dense_attention(q, K[toks], V[toks], d ** -0.5)
+    np.testing.assert_allclose(out, ref, atol=1e-12)
+
+
+def test_block_scores_mean_pool_vs_numpy():
+    """Ch11 §12.6: block score = (q . mean(K_block)) * d^-1/2; numpy mean/argsort."""
+    rng = np.random.default_rng(2)
+    L, D, B = 1000, 16, 64                               # 15 complete blocks + a 40-token tail
+    K, V, q = rng.standard_normal((L, D)), rng.standard_normal((L, D)), rng.standard_normal(D)
+    pooled = oracle.block_mean_pool(K, B)
+    np.testing.assert_allclose(pooled, K[: (L // B) * B].reshape(L // B, B, D).mean(1), atol=1e-14)
+    out, sel, bs = oracle.block_sparse(q, K, V, B, 4, 1, 100, D ** -0.5)
+    np.testing.assert_allclose(bs, pooled @ q * D ** -0.5, atol=1e-13)
+    assert len(bs) == L // B                             # the partial tail block is no candidate
+    want = np.sort(np.lexsort((np.arange(len(bs)), -bs))[:4])
+    assert sel.tolist() == want.tolist()
+    toks = sorted(set(t for b in want for t in range(b * B, b * B + B)) | set(range(B)) | set(range(L - 100, L)))
+    ref, _ = oracle.dense_attention(q, K[toks], V[toks], D ** -0.5)
+    np.testing.assert_allclose(out, ref, atol=1e-12)
+
+
+def test_block_window_only_is_sliding_window():
+    """Notes §4: S = {j : i - w < j <= i}; no blocks, no sink -> last w tokens."""
+    rng = np.random.default_rng(4)
+    L, D, w = 300, 8, 37
+    K, V, q = rng.standard_normal((L, D)), rng.standard_normal((L, D)), rng.standard_normal(D)
+    out, sel, _ = oracle.block_sparse(q, K, V, 64, 0, 0, w, 0.25)
+    ref, _ = oracle.dense_attention(q, K[L - w:], V[L - w:], 0.25)
+    np.testing.assert_allclose(out, ref, atol=1e-12)
+
+
+def test_block_all_blocks_is_dense():
+    rng = np.random.default_rng(6)
+    L, D = 256, 8
+    K, V, q = rng.standard_normal((L, D)), rng.standard_normal((L, D)), rng.standard_normal(D)
+    out, sel, _ = oracle.block_sparse(q, K, V, 64, 8, 1, 16, 0.3)
+    assert sel.tolist() == [0, 1, 2, 3, -1, -1, -1, -1]
+    ref, _ = oracle.dense_attention(q, K, V, 0.3)
+    np.testing.assert_allclose(out, ref, atol=1e-12)
+
+
+def test_block_sink_tokens_always_in():
+    """Ch11 §12.4 / LLMRes MoBA: the sink block is read even when it scores lowest."""
+    rng = np.random.default_rng(8)
+    L, D, B = 512, 8, 64
+    K, V = rng.standard_normal((L, D)) * 0.01, rng.standard_normal((L, D))
+    q = np.ones(D)
+    K[:B] -= 5.0                                         # block 0 scores lowest
+    out, sel, _ = oracle.block_sparse(q, K, V, B, 1, 1, 0, 1.0)
+    assert 0 not in sel.tolist()
+    toks = list(range(B)) + list(range(sel[0] * B, sel[0] * B + B))
+    ref, _ = oracle.dense_attention(q, K[toks], V[toks], 1.0)
+    np.testing.assert_allclose(out, ref, atol=1e-12)
+
+
+# ------------------------------------------------------------ whole step
+
+def test_dsa_step_placement_invariance():
+    """Notes §11: moving KV between storage places (here: a different page
+    permutation) leaves the whole step's output unchanged."""
+    import workloads
+    cfg = workloads.small_dsa(workloads.RAGGED, n_seqs=3, rows=3, lens=(200, 64, 130), H_I=4, d_I=16,
+                              topk=40, H=4, d_c=16, d_R=4)
+    a = workloads.dsa_inputs(cfg, seed=5)
+    b = dict(a)
+    table, _ = workloads.page_layout(cfg, 99)
+    # move every page's rows to its new place in all three caches
+    old = a["page_table"].numpy()
+    perm_rows = np.zeros(a["c_cache"].shape[0], dtype=np.int64)
+    for s in range(cfg.n_seqs):
+        for p in range(cfg.pages_per_seq):
+            if old[s, p] >= 0:
+                perm_rows[table[s, p] * 64: table[s, p] * 64 + 64] = np.arange(old[s, p] * 64, old[s, p] * 64 + 64)
+    idx = torch.from_numpy(perm_rows)
+    for key in ("k_idx_cache", "c_cache", "kr_cache"):
+        b[key] = a[key][idx]
+    b["page_table"] = torch.from_numpy(table)
+    ra, rb = oracle.dsa_step(a, range(3)), oracle.dsa_step(b, range(3))
+    assert np.array_equal(ra["idx"], rb["idx"])
+    np.testing.assert_array_equal(ra["out"], rb["out"])
+    np.testing.assert_array_equal(np.nan_to_num(ra["scores"]), np.nan_to_num(rb["scores"]))
