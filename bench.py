@@ -1,0 +1,481 @@
+#!/usr/bin/env python
+"""Benchmark of the sparse-attention hot path on B200.
+
+One step = the whole decode path over one batch: lightning indexer ->
+exact Top-K -> sparse MLA, i.e. one query per sequence of the workload.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config long|ragged|tiny|prefill|block]
+                    [--impl native|reference]
+
+Default workload: long decode, 32 sequences x 32768 tokens, H^I=64 fp8
+indexer, top-2048, 128-head sparse MLA (latent 512 + RoPE 64, bf16).  With N
+GPUs (torchrun, one process per GPU) every rank runs its own batch of the
+same shape (weak scaling, no data-path collective); the step time is the max
+over ranks.  Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+DECODE_METRIC = "sparse-MLA decode queries/s (indexer+topk+attn) at L=32K/128K; % HBM roofline"
+L2_FLUSH_BYTES = 256 << 20  # > 126 MB L2
+
+# dram__bytes_read.sum + dram__bytes_write.sum of the indexer kernel, per launch,
+# from one ncu capture of the long-decode workload, with the sha256 of the
+# kernel source it was taken on (the figure is reported only while they match).
+TRAFFIC = {
+    "long": {"bytes_per_launch": None, "src_sha": None},
+}
+
+
+def src_sha(rel: str) -> str:
+    with open(os.path.join(ROOT, rel), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+# ---------------------------------------------------------------- work model
+def decode_bytes(cfg: W.DSAConfig):
+    """Algorithmic bytes of one decode step: every visible indexer key once plus
+    every selected latent row (512 bf16 + 64 bf16 RoPE key) once."""
+    esize = 1 if cfg.idx_dtype == "e4m3" else 4
+    nv = cfg.n_visible()
+    keys = int(nv.sum()) * cfg.d_I * esize
+    rows = int(np.minimum(nv, cfg.topk).sum()) * (cfg.d_c + cfg.d_R) * 2
+    return keys, rows
+
+
+def prefill_flops(cfg: W.DSAConfig):
+    nv = cfg.n_visible().astype(np.float64)
+    idx = float((nv * 2 * cfg.H_I * cfg.d_I).sum())
+    mla = float((np.minimum(nv, cfg.topk) * cfg.H * 2 * (cfg.d_c + cfg.d_R + cfg.d_c)).sum())
+    return idx, mla
+
+
+def block_bytes(cfg: W.BlockConfig):
+    """Pooled-key scan plus the union's K and V rows, for every (sequence, head)."""
+    pooled = cfg.B * cfg.H * cfg.n_blocks * cfg.D * 4
+    # the union holds at most top*block + sink*block + window tokens
+    u_max = min(cfg.L, cfg.top_blocks * cfg.block + cfg.sink_blocks * cfg.block + cfg.window)
+    return pooled, u_max
+
+
+# ---------------------------------------------------------------- ranks
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def reduce_max(values, world_size: int, device):
+    """Element-wise max over ranks (identity for one rank)."""
+    if world_size == 1:
+        return list(values)
+    import torch.distributed as dist
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def rank_seed(base: int, rank: int) -> int:
+    return base + 7919 * rank
+
+
+# ---------------------------------------------------------------- clocks
+REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+           0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+           0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+
+class ClockSampler:
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.samples, self.reasons = [], 0
+        self.period = period_s
+        self._stop = threading.Event()
+        self.max_mhz = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nv = None
+
+    def _sample(self):
+        try:
+            self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+            self.reasons |= int(self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h))
+        except Exception:
+            pass
+
+    def _run(self):
+        while not self._stop.is_set():
+            self._sample()
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nv:
+            self._sample()
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.nv:
+            self._stop.set()
+            self.t.join()
+            self._sample()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        names = [n for bit, n in REASONS.items() if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz, "reasons": names,
+                "samples": len(self.samples)}
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), float(p.get("bf16_tflops_sustained", p["bf16_tflops"])), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# ---------------------------------------------------------------- native arm
+class DecodeStep:
+    """Buffers and launches of one indexer -> Top-K -> sparse-MLA step."""
+
+    def __init__(self, inp, sa):
+        self.sa, self.inp, self.cfg = sa, inp, inp["cfg"]
+        cfg, dev = self.cfg, inp["q_idx"].device
+        self.scores = torch.empty(cfg.rows, cfg.L_max, dtype=torch.float32, device=dev)
+        self.idx = torch.empty(cfg.rows, cfg.topk, dtype=torch.int32, device=dev)
+        self.out = torch.empty(cfg.rows, cfg.H, cfg.d_c, dtype=torch.float32, device=dev)
+        self.lse = torch.empty(cfg.rows, cfg.H, dtype=torch.float32, device=dev)
+        self.prefill = cfg.prefill_start >= 0
+        ws = 0 if self.prefill else sa.sparse_mla_workspace_size(cfg.rows, cfg.H, cfg.topk, cfg.d_c)
+        self.ws = torch.empty(max(ws, 256), dtype=torch.uint8, device=dev) if ws else None
+        self.launches_per_step = 3 + (1 if ws else 0)
+
+    def indexer(self):
+        i, c = self.inp, self.cfg
+        self.sa.index_scores(i["q_idx"], i["w"], i["k_idx_cache"], i["n_visible"], c.pages_per_seq,
+                             page_table=i["page_table"], seq_of_row=i["seq_of_row"], scores=self.scores)
+
+    def rest(self):
+        i, c = self.inp, self.cfg
+        self.sa.topk_select(self.scores, i["n_visible"], c.topk, idx_out=self.idx)
+        if self.prefill:
+            self.sa.sparse_mla_prefill(i["q_lat"], i["q_rope"], i["c_cache"], i["kr_cache"], self.idx, c.scale,
+                                       c.pages_per_seq, page_table=i["page_table"], seq_of_row=i["seq_of_row"],
+                                       out=self.out, lse=self.lse)
+        else:
+            self.sa.sparse_mla_decode(i["q_lat"], i["q_rope"], i["c_cache"], i["kr_cache"], self.idx, c.scale,
+                                      c.pages_per_seq, page_table=i["page_table"], seq_of_row=i["seq_of_row"],
+                                      out=self.out, lse=self.lse, workspace=self.ws)
+
+
+class BlockStep:
+    def __init__(self, inp, sa):
+        self.sa, self.inp, self.cfg = sa, inp, inp["cfg"]
+        c = self.cfg
+        self.pooled = sa.block_mean_pool(inp["K"], c.block)  # once, when the blocks completed
+        self.out = torch.empty(c.B, c.H, c.D, dtype=torch.float32, device=inp["q"].device)
+        self.launches_per_step = 1
+
+    def indexer(self):
+        i, c = self.inp, self.cfg
+        self.sa.block_sparse_attn(i["q"], self.pooled, i["K"], i["V"], c.block, c.top_blocks, c.sink_blocks,
+                                  c.window, c.scale, out=self.out)
+
+    def rest(self):
+        pass
+
+
+def time_steps(step, K: int, flush):
+    """K steps, each bracketed by CUDA events on the launching stream; the L2
+    flush runs between steps outside the events.  Returns per-step and
+    first-kernel times (ms)."""
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    for e0, e1, e2 in ev:
+        flush.zero_()
+        e0.record()
+        step.indexer()
+        e1.record()
+        step.rest()
+        e2.record()
+    torch.cuda.synchronize()
+    return [e0.elapsed_time(e2) for e0, e1, e2 in ev], [e0.elapsed_time(e1) for e0, e1, e2 in ev]
+
+
+def e2e_steps(step, K: int, flush):
+    """Same step through the public API with the step's query inputs copied in
+    from pinned host memory and the output read back, inside the events."""
+    inp = step.inp
+    if isinstance(step, DecodeStep):
+        names = ["q_idx", "w", "q_lat", "q_rope"]
+        result = step.out
+    else:
+        names = ["q"]
+        result = step.out
+    host_in = {n: inp[n].cpu().pin_memory() for n in names}
+    host_out = torch.empty(result.shape, dtype=result.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    d2h = host_out.numel() * host_out.element_size()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    for e0, e1 in ev:
+        flush.zero_()
+        e0.record()
+        for n, t in host_in.items():
+            inp[n].copy_(t, non_blocking=True)
+        step.indexer()
+        step.rest()
+        host_out.copy_(result, non_blocking=True)
+        e1.record()
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in ev], h2d, d2h
+
+
+def cpu_baseline(inp, cfg, budget_s: float = 12.0):
+    """The fp64 oracle as it stands, on a bounded sample of the workload's query rows."""
+    import oracle
+    threads = oracle.threads()
+    if isinstance(cfg, W.DSAConfig):
+        rows_all = list(range(cfg.rows))
+        t0 = time.perf_counter()
+        oracle.dsa_step(inp, rows_all[:1], with_scores=False)
+        one = time.perf_counter() - t0
+        n = int(max(1, min(len(rows_all), threads * max(1, budget_s // max(one * 1.0, 1e-3) // 1))))
+        n = max(1, min(n, len(rows_all), threads * 4))
+        rows = rows_all[:n]
+        t0 = time.perf_counter()
+        oracle.dsa_step(inp, rows, with_scores=False)
+        dt = time.perf_counter() - t0
+        unit_n = n
+        what = "query rows" if cfg.prefill_start < 0 else "query tokens"
+        sample = f"{n} of {cfg.rows} {what} of the workload (indexer over every visible key, top-{cfg.topk}, sparse MLA)"
+    else:
+        pairs = [(b, h) for b in range(cfg.B) for h in range(cfg.H)]
+        t0 = time.perf_counter()
+        oracle.block_step(inp, pairs[:1])
+        one = time.perf_counter() - t0
+        n = int(max(1, min(len(pairs), budget_s // max(one, 1e-3))))
+        t0 = time.perf_counter()
+        oracle.block_step(inp, pairs[:n])
+        dt = time.perf_counter() - t0
+        unit_n = n / cfg.H  # queries = sequences; one query spans H heads
+        sample = f"{n} of {cfg.B * cfg.H} (sequence, head) pairs"
+    return {"value": unit_n / dt, "cores": threads, "kind": "oracle", "sample": sample, "seconds": round(dt, 3)}
+
+
+def workload(name: str):
+    if name in W.DSA_CONFIGS:
+        return W.DSA_CONFIGS[name]
+    return W.BLOCK_CONFIGS[name]
+
+
+def describe(cfg, flush_note):
+    if isinstance(cfg, W.DSAConfig):
+        kind = "prefill chunk" if cfg.prefill_start >= 0 else "decode"
+        lens = (f"L={cfg.lens[0]}" if len(set(cfg.lens)) == 1 else
+                f"L_b in [{min(cfg.lens)},{max(cfg.lens)}] (sum {sum(cfg.lens)}), 64-token pages, shuffled page table")
+        return {"workload": f"{cfg.name} {kind}: {cfg.rows} queries, {lens}, indexer H^I={cfg.H_I} d^I={cfg.d_I} "
+                            f"{cfg.idx_dtype}, top-{cfg.topk}, sparse MLA {cfg.H} heads d_c={cfg.d_c} d_R={cfg.d_R} bf16",
+                "batch": cfg.rows, "seq_len": max(cfg.lens), "topk": cfg.topk, "heads": cfg.H, "l2": flush_note}
+    return {"workload": f"block-sparse decode: B={cfg.B}, L={cfg.L}, {cfg.H} MHA heads, head_dim {cfg.D} bf16, "
+                        f"block {cfg.block}, top-{cfg.top_blocks} + {cfg.sink_blocks} sink block + {cfg.window}-token window",
+            "batch": cfg.B, "seq_len": cfg.L, "heads": cfg.H, "l2": flush_note}
+
+
+def run_native(args):
+    ws, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    import sparse_attention_07_b200 as sa
+    sa.lib()
+    cfg = workload(args.config)
+    if isinstance(cfg, W.DSAConfig):
+        inp = W.dsa_inputs(cfg, dev, seed=rank_seed(cfg.seed, rank))
+        step = DecodeStep(inp, sa)
+    else:
+        inp = W.block_inputs(cfg, dev, seed=rank_seed(cfg.seed, rank))
+        step = BlockStep(inp, sa)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    for _ in range(args.warmup):
+        flush.zero_()
+        step.indexer()
+        step.rest()
+    torch.cuda.synchronize()
+    if sa.check_device_error() != 0:
+        raise RuntimeError("device error word set during warm-up")
+
+    if ws > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        step_ms, first_ms = time_steps(step, args.steps, flush)
+    if ws > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    e2e_ms, h2d, d2h = e2e_steps(step, args.steps, flush)
+    err = sa.check_device_error()
+    if err != 0:
+        raise RuntimeError(f"device error word 0x{err:x}")
+
+    ms = statistics.mean(step_ms)
+    first = statistics.mean(first_ms)
+    e2e = statistics.mean(e2e_ms)
+    ms, first, e2e = reduce_max([ms, first, e2e], ws, dev)
+
+    hbm, bf16_burst, bf16_sus, peak_src = peaks()
+    res = {"impl": "native"}
+    if isinstance(cfg, W.DSAConfig):
+        prefill = cfg.prefill_start >= 0
+        units = cfg.rows * ws
+        unit = "tokens/s" if prefill else "queries/s"
+        metric = "sparse-MLA prefill tokens/s (indexer+topk+attn)" if prefill else DECODE_METRIC
+        keys_b, rows_b = decode_bytes(cfg)
+        if prefill:
+            fi, fm = prefill_flops(cfg)
+            fp8_peak = bf16_burst * 2.0  # fp8 dense rate = 2x bf16 (nominal ratio)
+            ach = fi / (first * 1e-3) / 1e12
+            roof = {"bound": "tensor", "achieved": round(ach, 1), "peak": fp8_peak, "unit": "TFLOP/s",
+                    "frac": round(ach / fp8_peak, 4), "traffic": None,
+                    "kernel": "idx_tc_kernel (fp8 kind::f8f6f4)",
+                    "peak_source": f"{peak_src} bf16 burst x 2 (nominal fp8/bf16 ratio)"}
+        else:
+            ach = keys_b / (first * 1e-3) / 1e9
+            tr = TRAFFIC.get(args.config, {})
+            traffic = tr.get("bytes_per_launch") if tr.get("src_sha") == src_sha(
+                "sparse_attention_07_b200/csrc/index_scores.cu") else None
+            roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": hbm, "unit": "GB/s",
+                    "frac": round(ach / hbm, 4), "traffic": traffic,
+                    "kernel": "idx_tc_kernel" if cfg.idx_dtype == "e4m3" else "idx_cc_kernel",
+                    "peak_source": f"{peak_src} hbm_gbs"}
+        step_gbs = (keys_b + rows_b) / (ms * 1e-3) / 1e9
+        res["step_roofline"] = {"bytes_per_step": keys_b + rows_b, "indexer_key_bytes": keys_b,
+                                "gathered_row_bytes": rows_b, "achieved": round(step_gbs, 1), "peak": hbm,
+                                "unit": "GB/s", "frac": round(step_gbs / hbm, 4)}
+    else:
+        units = cfg.B * ws
+        unit = "queries/s"
+        metric = "block-sparse decode queries/s (pooled-block scan+top-k+block attention)"
+        pooled_b, u_max = block_bytes(cfg)
+        ach = pooled_b / (first * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": hbm, "unit": "GB/s", "frac": round(ach / hbm, 4),
+                "traffic": None, "kernel": "block_sparse_kernel (pooled-key bytes only)",
+                "peak_source": f"{peak_src} hbm_gbs"}
+    value = units / (ms * 1e-3)
+    res.update({
+        "metric": metric, "value": round(value, 1), "unit": unit, "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "e4m3 indexer / bf16 MLA, fp32 accumulate" if isinstance(cfg, W.DSAConfig)
+        else "bf16, fp32 accumulate",
+        "data": "synthetic (seeded, shapes and value distributions of the workload)",
+        "config": describe(cfg, f"flushed between steps ({L2_FLUSH_BYTES >> 20} MiB write, outside the events)"),
+        "roofline": roof,
+        "e2e": {"value": round(units / (e2e * 1e-3), 1), "unit": unit, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": step.launches_per_step * args.steps,
+        "clocks": clk.summary(),
+    })
+    if ws == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline(inp, cfg)
+        res["cpu_baseline"]["unit"] = unit
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    if ws > 1:
+        torch.distributed.destroy_process_group()
+
+
+def run_reference(args):
+    """The oracle as the reference arm, timed on the host cores."""
+    ws, rank, local = dist_env()
+    if rank != 0:
+        return
+    import oracle
+    cfg = workload(args.config)
+    dev = torch.device("cuda", local) if torch.cuda.is_available() else torch.device("cpu")
+    if isinstance(cfg, W.DSAConfig):
+        inp = W.dsa_inputs(cfg, dev, seed=cfg.seed)
+        prefill = cfg.prefill_start >= 0
+        unit = "tokens/s" if prefill else "queries/s"
+        metric = "sparse-MLA prefill tokens/s (indexer+topk+attn)" if prefill else DECODE_METRIC
+        t0 = time.perf_counter()
+        oracle.dsa_step(inp, [0], with_scores=False)
+        one = time.perf_counter() - t0
+        per_step = max(1, min(cfg.rows, oracle.threads(), int(150.0 / max(1, args.steps + args.warmup) / max(one, 1e-3))))
+        rows = list(range(per_step))
+        run = lambda: oracle.dsa_step(inp, rows, with_scores=False)  # noqa: E731
+        units_per_step = per_step
+        sample = f"{per_step} query rows of the workload per step"
+    else:
+        inp = W.block_inputs(cfg, dev, seed=cfg.seed)
+        unit, metric = "queries/s", "block-sparse decode queries/s (pooled-block scan+top-k+block attention)"
+        pairs = [(0, h) for h in range(cfg.H)]
+        run = lambda: oracle.block_step(inp, pairs)  # noqa: E731
+        units_per_step = 1
+        sample = f"one sequence ({cfg.H} heads) per step"
+    for _ in range(args.warmup):
+        run()
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        run()
+        times.append(time.perf_counter() - t0)
+    ms = statistics.mean(times) * 1e3
+    value = units_per_step / (ms * 1e-3)
+    print(json.dumps({
+        "impl": "reference", "metric": metric, "value": round(value, 3), "unit": unit, "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
+        "config": describe(cfg, "n/a (host)"),
+        "cpu_baseline": {"value": round(value, 3), "unit": unit, "cores": oracle.threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 3), "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main(argv=None):
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--warmup", type=int, default=10)
+    p.add_argument("--impl", choices=["native", "reference"], default="native")
+    p.add_argument("--config", default="long", choices=sorted(list(W.DSA_CONFIGS) + list(W.BLOCK_CONFIGS)))
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    args = p.parse_args(argv)
+    if args.warmup < 3 and args.impl == "native":
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_native(args)
+
+
+if __name__ == "__main__":
+    main()

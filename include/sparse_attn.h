@@ -1,0 +1,202 @@
+/*
+ * sparse_attn.h — C ABI of the B200 (sm_100a) sparse-attention library
+ * (libsparse_attn.so).
+ *
+ * The library computes DeepSeek-Sparse-Attention-style decode and prefill in
+ * three stream-ordered calls, plus a block-sparse (MoBA/NSA-style) decode:
+ *
+ *   sa_index_scores      lightning indexer  I_{t,s} = sum_j w_{t,j} ReLU(q^I_{t,j} . k^I_s)
+ *   sa_topk_select       exact Top-K of I_{t,:} (ties to the lower position)
+ *   sa_sparse_mla_decode / sa_sparse_mla_prefill
+ *                        softmax over the selected set of the absorbed content score
+ *                        plus the RoPE score, scaled; output sum_j a_j c_j in latent space
+ *   sa_block_mean_pool   mean-pooled block keys (run when blocks complete)
+ *   sa_block_sparse_attn top blocks by q . mean(K_block), plus sink and window; softmax
+ *                        over the union of their tokens
+ *
+ * Sources, cited by page title and section:
+ *   [Notes]  "Sparse Attention 数学学习笔记" (echobase-5bl.pages.dev, 2026.09.14)
+ *   [MLA-S]  "MLA 与稀疏注意力：少存一点，还是少看一点？" (tianyi-zhang-02.github.io)
+ *   [Ch11]   "第 11 章 稀疏注意力" (book.shippingwang.com)
+ *   [LLMRes] "LLM注意力优化：稀疏注意力" (wln20.github.io)
+ *
+ * Conventions shared by every call:
+ *  - Every pointer is device memory owned by the caller unless stated.  The
+ *    library allocates nothing and keeps no state between calls other than
+ *    one device error word per GPU (see sa_check_device_error) and a cache of
+ *    driver entry points.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *    default stream) and never synchronise the host.
+ *  - Arguments are checked on the host before anything is launched: a bad
+ *    count, a null required pointer, or a pointer that breaks the alignment a
+ *    call states returns SA_EINVAL; shapes the kernels do not handle return
+ *    SA_EUNSUPPORTED.  In both cases nothing is launched.  A failed launch
+ *    returns SA_ECUDA.
+ *  - Contents the caller promises (finite scores, page ids inside the pool,
+ *    positions below the sequence length) are preconditions: they are not
+ *    checked on the device, except where a call says so.
+ *  - Paging: a cache is a pool of 64-token pages, row = page * 64 + (pos % 64).
+ *    `page_table` [n_seqs][pages_per_seq] int32 gives the physical page of each
+ *    (sequence, pos / 64); NULL means contiguous: page = seq * pages_per_seq +
+ *    pos / 64.  Placement never changes a result ([Notes] §11).
+ *  - `seq_of_row` [rows] int32 maps a query row to its sequence; NULL means
+ *    row r is sequence r (decode: one query per sequence).
+ */
+#ifndef SPARSE_ATTN_H
+#define SPARSE_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* sa_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+    SA_OK = 0,
+    SA_EINVAL = 1,        /* bad argument; nothing launched */
+    SA_EUNSUPPORTED = 2,  /* valid for the method, not handled by the kernels; nothing launched */
+    SA_ECUDA = 3,         /* a CUDA runtime call or launch failed */
+    SA_ETIMEOUT = 4       /* reported by sa_check_device_error: a kernel's bounded wait ran out */
+} sa_status;
+
+typedef enum {
+    SA_F32 = 0,   /* IEEE binary32 */
+    SA_E4M3 = 1,  /* fp8 e4m3 (OCP "e4m3fn", no infinities) */
+    SA_BF16 = 2   /* bfloat16 */
+} sa_dtype;
+
+/* Short name of a status code (static string). */
+const char* sa_status_string(sa_status s);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int sa_version(void);
+
+/*
+ * Waits for `stream`, then reads and clears this GPU's device error word.
+ * Kernels that wait on barriers give every wait a time limit; when one runs
+ * out the kernel records a nonzero site code here, abandons its work
+ * (outputs of that launch are then undefined) and returns.  *code_out gets
+ * the code (0 = none).  Returns SA_ETIMEOUT if a code was set, SA_ECUDA if
+ * the stream reported an error, else SA_OK.  This is the only call that
+ * synchronises.
+ */
+sa_status sa_check_device_error(int* code_out, sa_stream_t stream);
+
+/*
+ * Lightning indexer ([Notes] §9, index score I_{t,s}; [MLA-S] "DSA：先用便宜的
+ * indexer 选位置"):
+ *     scores[r][s] = sum_{j<H_I} w[r][j] * max(0, sum_{d<d_I} q[r][j][d] * k(seq(r), s)[d])
+ * for 0 <= s < n_visible[r].  No scale, no softmax.  Entries s >= n_visible[r]
+ * are left untouched.  One key per token, shared by all indexer heads.
+ *
+ *   q         [rows][H_I][d_I]   dtype
+ *   w         [rows][H_I]        fp32
+ *   k_cache   [pool_pages*64][d_I] dtype (pages as above); a page id outside
+ *             [0, pool_pages) reads as zeros and never faults
+ *   n_visible [rows]             int32, 0 <= n_visible[r] <= pages_per_seq*64
+ *   scores    [rows][scores_ld]  fp32, scores_ld >= max n_visible
+ * Products and sums are accumulated in fp32; on integer inputs with
+ * power-of-two weights (every partial sum below 2^24 units) the result is
+ * exact.  dtype SA_E4M3 with d_I = 128 runs on the tensor cores (tcgen05,
+ * kind::f8f6f4); other shapes (d_I <= 128, H_I <= 64, fp32 or e4m3) run on
+ * the CUDA cores.  Rows sharing a sequence are batched against one key tile
+ * when they are consecutive.  Alignment: k_cache and q 16-byte aligned.
+ */
+sa_status sa_index_scores(const void* q, const float* w, const void* k_cache, int64_t pool_pages,
+                          sa_dtype dtype, const int32_t* page_table, int pages_per_seq,
+                          const int32_t* seq_of_row, const int32_t* n_visible,
+                          int rows, int H_I, int d_I, int64_t scores_ld, float* scores,
+                          sa_stream_t stream);
+
+/*
+ * Exact Top-K ([Notes] §9, S_t = {s | I_{t,s} in TopK(I_{t,:}, k)}; [MLA-S]
+ * "一次错选会丢掉什么？" orders by (-score, position)):
+ * idx_out[r] receives the min(k, n_valid[r]) positions with the largest
+ * scores[r][0 .. n_valid[r]-1], equal scores going to the lower position,
+ * written in ascending position order, then -1 up to k.  -0.0 equals +0.0.
+ * Scores must be finite (precondition).
+ *   scores  [rows][scores_ld] fp32;  n_valid [rows] int32 (<= scores_ld)
+ *   idx_out [rows][k] int32
+ * Limits: 1 <= k; scores_ld <= 262144.
+ */
+sa_status sa_topk_select(const float* scores, int64_t scores_ld, const int32_t* n_valid,
+                         int rows, int k, int32_t* idx_out, sa_stream_t stream);
+
+/*
+ * Sparse MLA attention over the selected latent rows ([MLA-S] "分开以后，完整分数
+ * 怎么算？" and "“吸收矩阵”是交换线性计算的顺序"; [Notes] §2, §8):
+ *   z_j = (q_lat[r][h] . c_j + q_rope[r][h] . kr_j) * scale,   j in S_r
+ *   out[r][h] = sum_j softmax_{S_r}(z)_j * c_j         (latent aggregate; U_V is outside)
+ *   lse[r][h] = log sum_{j in S_r} exp(z_j)            (natural log; -inf if S_r is empty)
+ * S_r = the positions idx[r][0..k-1] that are >= 0, resolved to cache rows
+ * through seq(r) and the page table.  The latent row c_j is both the content
+ * key and the value; one selection is shared by all heads.
+ *
+ *   q_lat  [rows][H][d_c] bf16 (absorbed U_K^T q^C);  q_rope [rows][H][d_R] bf16 (rotated)
+ *   c_cache  rows of d_c bf16 at stride c_ld elements;  kr_cache rows of d_R bf16 at stride kr_ld;
+ *            both pools hold pool_pages*64 rows (a page id outside the pool reads row 0)
+ *   idx    [rows][k] int32 positions or -1
+ *   out    [rows][H][d_c] fp32;  lse [rows][H] fp32 or NULL
+ * Supported: d_c = 512, d_R = 64, 1 <= H <= 128; bf16 inputs, fp32 softmax
+ * and accumulation on the tensor cores.  Alignment: every base pointer and
+ * row stride a multiple of 16 bytes.
+ * _decode splits each row's k positions over several CTAs when rows are few
+ * and combines the partial softmax states in `workspace`
+ * (sa_sparse_mla_workspace_size bytes, 256-byte aligned; may be NULL when the
+ * size is 0).  _prefill keeps one row per CTA pair and needs no workspace.
+ */
+size_t sa_sparse_mla_workspace_size(int rows, int H, int k, int d_c);
+
+sa_status sa_sparse_mla_decode(const void* q_lat, const void* q_rope,
+                               const void* c_cache, int64_t c_ld, const void* kr_cache, int64_t kr_ld,
+                               int64_t pool_pages, const int32_t* page_table, int pages_per_seq,
+                               const int32_t* seq_of_row,
+                               const int32_t* idx, int rows, int H, int k, int d_c, int d_R, float scale,
+                               float* out, float* lse, void* workspace, size_t workspace_bytes,
+                               sa_stream_t stream);
+
+sa_status sa_sparse_mla_prefill(const void* q_lat, const void* q_rope,
+                                const void* c_cache, int64_t c_ld, const void* kr_cache, int64_t kr_ld,
+                                int64_t pool_pages, const int32_t* page_table, int pages_per_seq,
+                                const int32_t* seq_of_row,
+                                const int32_t* idx, int rows, int H, int k, int d_c, int d_R, float scale,
+                                float* out, float* lse, sa_stream_t stream);
+
+/*
+ * Mean-pooled block keys ([Ch11] §12.6, k_rep = k_blocks.mean(1)):
+ *   pooled[b][h][n][d] = (1/block) * sum_{i<block} K[b][n*block+i][h][d]
+ * for every complete block n < L / block.
+ *   K  bf16, element (b,t,h,d) at b*stride_b + t*stride_t + h*stride_h + d (elements)
+ *   pooled [B][H][pooled_ld][D] fp32, pooled_ld >= L / block
+ * Supported: D = 128.
+ */
+sa_status sa_block_mean_pool(const void* K, int64_t stride_b, int64_t stride_t, int64_t stride_h,
+                             int B, int L, int H, int D, int block, float* pooled, int64_t pooled_ld,
+                             sa_stream_t stream);
+
+/*
+ * Block-sparse decode for the query at position L-1 of each (sequence, head)
+ * ([Ch11] §12.5-12.6; [LLMRes] MoBA; [Notes] §4 window; [MLA-S] causality of
+ * pooling):
+ *   score_n = scale * q[b][h] . pooled[b][h][n]  over complete blocks n < L/block
+ *   chosen  = the top_blocks blocks by (-score_n, n)
+ *   U       = tokens of chosen blocks  u  [0, sink_blocks*block)  u  [L-window, L)
+ *   out[b][h] = sum_{t in U} softmax_U(scale * q . K_t) V_t
+ *   q [B][H][D] bf16; K, V as in sa_block_mean_pool; out [B][H][D] fp32;
+ *   sel_blocks [B][H][top_blocks] int32 (ascending, -1 padded) or NULL.
+ * Supported: D = 128, block = 64, 1 <= top_blocks <= 64, L/block <= 4096.
+ */
+sa_status sa_block_sparse_attn(const void* q, const float* pooled, int64_t pooled_ld,
+                               const void* K, const void* V, int64_t stride_b, int64_t stride_t,
+                               int64_t stride_h, int B, int H, int D, int L, int block,
+                               int top_blocks, int sink_blocks, int window, float scale,
+                               float* out, int32_t* sel_blocks, sa_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPARSE_ATTN_H */

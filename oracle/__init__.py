@@ -64,6 +64,7 @@ def _load():
         lib.sa_oracle_sparse_mla.argtypes = [I, I, I, I, P, P, P, P, P, I, D, P, P]
         lib.sa_oracle_block_mean_pool.argtypes = [I, I, I, P, P]
         lib.sa_oracle_block_sparse.argtypes = [I, I, I, I, I, I, D, P, P, P, P, P, P]
+        lib.sa_oracle_block_attend.argtypes = [I, I, I, P, I, I, I, D, P, P, P, P]
         lib.sa_oracle_threads.restype = I
         _lib = lib
     return _lib
@@ -164,6 +165,18 @@ def block_sparse(q, K, V, block: int, top_blocks: int, sink_blocks: int, window:
     _load().sa_oracle_block_sparse(L, D, block, top_blocks, sink_blocks, window, float(scale),
                                    _ptr(q), _ptr(K), _ptr(V), _ptr(out), _ptr(sel), _ptr(bs))
     return out, sel, bs[: L // block]
+
+
+def block_attend(q, K, V, chosen_blocks, block: int, sink_blocks: int, window: int, scale: float):
+    """Attention over the union of given chosen blocks, sink and window
+    ([Ch11] §12.5 block gather, [Notes] §2 softmax over the chosen set)."""
+    q, K, V = _f64(q), _f64(K), _f64(V)
+    L, D = K.shape
+    ch = np.ascontiguousarray(np.asarray(chosen_blocks, dtype=np.int32))
+    out = np.zeros(D)
+    _load().sa_oracle_block_attend(L, D, block, _ptr(ch), len(ch), sink_blocks, window, float(scale),
+                                   _ptr(q), _ptr(K), _ptr(V), _ptr(out))
+    return out
 
 
 # --------------------------------------------------------------------------

@@ -185,29 +185,16 @@ void sa_oracle_block_mean_pool(int L, int D, int block, const double* K, double*
         }
 }
 
-void sa_oracle_block_sparse(int L, int D, int block, int top_blocks, int sink_blocks, int window,
-                            double scale, const double* q, const double* K, const double* V,
-                            double* out, int32_t* sel, double* block_scores)
+/* Attention over the token union of given chosen blocks, the sink blocks and
+ * the window (the second half of the block-sparse decode above). */
+void sa_oracle_block_attend(int L, int D, int block, const int32_t* chosen_blocks, int n_chosen,
+                            int sink_blocks, int window, double scale,
+                            const double* q, const double* K, const double* V, double* out)
 {
     int nb = L / block;
-    double* pooled = (double*)malloc((size_t)(nb > 0 ? nb : 1) * D * sizeof(double));
-    sa_oracle_block_mean_pool(L, D, block, K, pooled);
-    sa_oracle_pair* p = (sa_oracle_pair*)malloc((size_t)(nb > 0 ? nb : 1) * sizeof(sa_oracle_pair));
-    for (int n = 0; n < nb; ++n) {
-        double dot = 0.0;
-        for (int d = 0; d < D; ++d) dot += q[d] * pooled[(int64_t)n * D + d];
-        p[n].v = dot * scale;
-        p[n].i = n;
-        if (block_scores) block_scores[n] = p[n].v;
-    }
-    qsort(p, (size_t)nb, sizeof(sa_oracle_pair), sa_oracle_cmp_desc);
-    int m = nb < top_blocks ? nb : top_blocks;
     char* chosen = (char*)calloc((size_t)(nb + 1), 1);
-    for (int j = 0; j < m; ++j) { sel[j] = (int32_t)p[j].i; chosen[p[j].i] = 1; }
-    qsort(sel, (size_t)m, sizeof(int32_t), sa_oracle_cmp_i32);
-    for (int j = m; j < top_blocks; ++j) sel[j] = -1;
-
-    /* token union: chosen blocks, sink tokens, window tokens */
+    for (int j = 0; j < n_chosen; ++j)
+        if (chosen_blocks[j] >= 0 && chosen_blocks[j] < nb) chosen[chosen_blocks[j]] = 1;
     double* z = (double*)malloc((size_t)(L > 0 ? L : 1) * sizeof(double));
     char* in_u = (char*)calloc((size_t)(L > 0 ? L : 1), 1);
     double mx = -INFINITY;
@@ -229,7 +216,31 @@ void sa_oracle_block_sparse(int L, int D, int block, int top_blocks, int sink_bl
         double a = exp(z[t] - mx) / l;
         for (int d = 0; d < D; ++d) out[d] += a * V[(int64_t)t * D + d];
     }
-    free(pooled); free(p); free(chosen); free(z); free(in_u);
+    free(chosen); free(z); free(in_u);
+}
+
+void sa_oracle_block_sparse(int L, int D, int block, int top_blocks, int sink_blocks, int window,
+                            double scale, const double* q, const double* K, const double* V,
+                            double* out, int32_t* sel, double* block_scores)
+{
+    int nb = L / block;
+    double* pooled = (double*)malloc((size_t)(nb > 0 ? nb : 1) * D * sizeof(double));
+    sa_oracle_block_mean_pool(L, D, block, K, pooled);
+    sa_oracle_pair* p = (sa_oracle_pair*)malloc((size_t)(nb > 0 ? nb : 1) * sizeof(sa_oracle_pair));
+    for (int n = 0; n < nb; ++n) {
+        double dot = 0.0;
+        for (int d = 0; d < D; ++d) dot += q[d] * pooled[(int64_t)n * D + d];
+        p[n].v = dot * scale;
+        p[n].i = n;
+        if (block_scores) block_scores[n] = p[n].v;
+    }
+    qsort(p, (size_t)nb, sizeof(sa_oracle_pair), sa_oracle_cmp_desc);
+    int m = nb < top_blocks ? nb : top_blocks;
+    for (int j = 0; j < m; ++j) sel[j] = (int32_t)p[j].i;
+    qsort(sel, (size_t)m, sizeof(int32_t), sa_oracle_cmp_i32);
+    for (int j = m; j < top_blocks; ++j) sel[j] = -1;
+    sa_oracle_block_attend(L, D, block, sel, m, sink_blocks, window, scale, q, K, V, out);
+    free(pooled); free(p);
 }
 
 /* Number of host threads OpenMP will use (reported beside the CPU timings). */

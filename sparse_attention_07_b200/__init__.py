@@ -1,0 +1,184 @@
+"""Thin Python binding of libsparse_attn.so (C ABI in include/sparse_attn.h).
+
+Argument marshalling only: every step of the hot path runs in the library's
+CUDA kernels.  PyTorch supplies device memory and the current stream.  There
+is no CPU or library fallback: if the shared library is missing or a call
+fails, an exception is raised.
+
+Functions take torch tensors on the current CUDA device and launch on
+``torch.cuda.current_stream()``; outputs are allocated with torch unless given.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsparse_attn.so")
+_lib = None
+
+SA_OK, SA_EINVAL, SA_EUNSUPPORTED, SA_ECUDA, SA_ETIMEOUT = range(5)
+SA_F32, SA_E4M3, SA_BF16 = range(3)
+
+EXPORTS = (
+    "sa_status_string", "sa_version", "sa_check_device_error", "sa_index_scores", "sa_topk_select",
+    "sa_sparse_mla_workspace_size", "sa_sparse_mla_decode", "sa_sparse_mla_prefill",
+    "sa_block_mean_pool", "sa_block_sparse_attn",
+)
+
+
+class SparseAttnError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        name = lib().sa_status_string(status).decode()
+        super().__init__(f"{fn} returned {name} ({status})")
+        self.status = status
+
+
+def lib():
+    """Load the shared library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with `python -m sparse_attention_07_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I, I64, F, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+        L.sa_status_string.restype = ctypes.c_char_p
+        L.sa_status_string.argtypes = [I]
+        L.sa_version.restype = I
+        L.sa_check_device_error.argtypes = [ctypes.POINTER(I), P]
+        L.sa_index_scores.argtypes = [P, P, P, I64, I, P, I, P, P, I, I, I, I64, P, P]
+        L.sa_topk_select.argtypes = [P, I64, P, I, I, P, P]
+        L.sa_sparse_mla_workspace_size.restype = SZ
+        L.sa_sparse_mla_workspace_size.argtypes = [I, I, I, I]
+        L.sa_sparse_mla_decode.argtypes = [P, P, P, I64, P, I64, I64, P, I, P, P, I, I, I, I, I, F, P, P, P, SZ, P]
+        L.sa_sparse_mla_prefill.argtypes = [P, P, P, I64, P, I64, I64, P, I, P, P, I, I, I, I, I, F, P, P, P]
+        L.sa_block_mean_pool.argtypes = [P, I64, I64, I64, I, I, I, I, I, P, I64, P]
+        L.sa_block_sparse_attn.argtypes = [P, P, I64, P, P, I64, I64, I64, I, I, I, I, I, I, I, I, F, P, P, P]
+        for name in EXPORTS:
+            if name not in ("sa_status_string", "sa_version", "sa_sparse_mla_workspace_size"):
+                getattr(L, name).restype = I
+        _lib = L
+    return _lib
+
+
+def _p(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _check(fn: str, st: int):
+    if st != SA_OK:
+        raise SparseAttnError(fn, st)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return SA_F32
+    if t.dtype == torch.float8_e4m3fn:
+        return SA_E4M3
+    raise TypeError(f"unsupported indexer dtype {t.dtype}")
+
+
+def check_device_error() -> int:
+    """Synchronise the current stream; return (and clear) the device error word."""
+    code = ctypes.c_int(0)
+    st = lib().sa_check_device_error(ctypes.byref(code), _stream())
+    if st not in (SA_OK, SA_ETIMEOUT):
+        raise SparseAttnError("sa_check_device_error", st)
+    return code.value
+
+
+def index_scores(q_idx, w, k_idx_cache, n_visible, pages_per_seq: int, page_table=None, seq_of_row=None,
+                 scores=None, scores_ld: Optional[int] = None):
+    """Lightning-indexer scores [rows, scores_ld] fp32 (entries past n_visible untouched)."""
+    rows, H_I, d_I = q_idx.shape
+    ld = scores_ld or pages_per_seq * 64
+    if scores is None:
+        scores = torch.empty(rows, ld, dtype=torch.float32, device=q_idx.device)
+    pool_pages = k_idx_cache.shape[0] // 64
+    st = lib().sa_index_scores(_p(q_idx), _p(w), _p(k_idx_cache), pool_pages, _dtype_code(q_idx), _p(page_table),
+                               pages_per_seq, _p(seq_of_row), _p(n_visible), rows, H_I, d_I, scores.stride(0),
+                               _p(scores), _stream())
+    _check("sa_index_scores", st)
+    return scores
+
+
+def topk_select(scores, n_valid, k: int, idx_out=None):
+    """Exact Top-K positions [rows, k] int32, ascending, -1 padded."""
+    rows = scores.shape[0]
+    if idx_out is None:
+        idx_out = torch.empty(rows, k, dtype=torch.int32, device=scores.device)
+    st = lib().sa_topk_select(_p(scores), scores.stride(0), _p(n_valid), rows, k, _p(idx_out), _stream())
+    _check("sa_topk_select", st)
+    return idx_out
+
+
+def sparse_mla_workspace_size(rows: int, H: int, k: int, d_c: int = 512) -> int:
+    return int(lib().sa_sparse_mla_workspace_size(rows, H, k, d_c))
+
+
+def _mla_args(q_lat, q_rope, c_cache, kr_cache, idx, out, lse):
+    rows, H, d_c = q_lat.shape
+    d_R = q_rope.shape[2]
+    k = idx.shape[1]
+    if out is None:
+        out = torch.empty(rows, H, d_c, dtype=torch.float32, device=q_lat.device)
+    pool_pages = c_cache.shape[0] // 64
+    return rows, H, d_c, d_R, k, out, lse, pool_pages
+
+
+def sparse_mla_decode(q_lat, q_rope, c_cache, kr_cache, idx, scale: float, pages_per_seq: int, page_table=None,
+                      seq_of_row=None, out=None, lse=None, workspace=None):
+    """Sparse MLA (latent aggregate) [rows, H, d_c] fp32; optional lse [rows, H]."""
+    rows, H, d_c, d_R, k, out, lse, pool_pages = _mla_args(q_lat, q_rope, c_cache, kr_cache, idx, out, lse)
+    need = sparse_mla_workspace_size(rows, H, k, d_c)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q_lat.device)
+    wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib().sa_sparse_mla_decode(_p(q_lat), _p(q_rope), _p(c_cache), c_cache.stride(0), _p(kr_cache),
+                                    kr_cache.stride(0), pool_pages, _p(page_table), pages_per_seq, _p(seq_of_row),
+                                    _p(idx), rows, H, k, d_c, d_R, float(scale), _p(out), _p(lse), _p(workspace),
+                                    wbytes, _stream())
+    _check("sa_sparse_mla_decode", st)
+    return out
+
+
+def sparse_mla_prefill(q_lat, q_rope, c_cache, kr_cache, idx, scale: float, pages_per_seq: int, page_table=None,
+                       seq_of_row=None, out=None, lse=None):
+    rows, H, d_c, d_R, k, out, lse, pool_pages = _mla_args(q_lat, q_rope, c_cache, kr_cache, idx, out, lse)
+    st = lib().sa_sparse_mla_prefill(_p(q_lat), _p(q_rope), _p(c_cache), c_cache.stride(0), _p(kr_cache),
+                                     kr_cache.stride(0), pool_pages, _p(page_table), pages_per_seq, _p(seq_of_row),
+                                     _p(idx), rows, H, k, d_c, d_R, float(scale), _p(out), _p(lse), _stream())
+    _check("sa_sparse_mla_prefill", st)
+    return out
+
+
+def block_mean_pool(K, block: int = 64, pooled=None):
+    """Mean-pooled complete blocks: K [B, L, H, D] bf16 -> [B, H, L//block, D] fp32."""
+    B, L, H, D = K.shape
+    nb = L // block
+    if pooled is None:
+        pooled = torch.empty(B, H, max(nb, 1), D, dtype=torch.float32, device=K.device)
+    st = lib().sa_block_mean_pool(_p(K), K.stride(0), K.stride(1), K.stride(2), B, L, H, D, block, _p(pooled),
+                                  pooled.shape[2], _stream())
+    _check("sa_block_mean_pool", st)
+    return pooled
+
+
+def block_sparse_attn(q, pooled, K, V, block: int, top_blocks: int, sink_blocks: int, window: int, scale: float,
+                      out=None, sel_blocks=None):
+    """Block-sparse decode of the query at position L-1: out [B, H, D] fp32."""
+    B, L, H, D = K.shape
+    if out is None:
+        out = torch.empty(B, H, D, dtype=torch.float32, device=q.device)
+    st = lib().sa_block_sparse_attn(_p(q), _p(pooled), pooled.shape[2], _p(K), _p(V), K.stride(0), K.stride(1),
+                                    K.stride(2), B, H, D, L, block, top_blocks, sink_blocks, window, float(scale),
+                                    _p(out), _p(sel_blocks), _stream())
+    _check("sa_block_sparse_attn", st)
+    return out

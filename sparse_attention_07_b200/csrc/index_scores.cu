@@ -1,0 +1,520 @@
+// index_scores.cu — lightning-indexer kernels.
+//
+// Computes I[r][s] = sum_j w[r][j] * ReLU(q[r][j] . k(seq(r), s)) for every
+// visible position ("Sparse Attention 数学学习笔记" §9, index score I_{t,s};
+// "MLA 与稀疏注意力" DSA section: one key per token shared by all indexer heads,
+// per-head queries and weights, no scale, no softmax).
+//
+// Tensor-core path (fp8 e4m3, d_I = 128): for one sequence the score tile of
+// 128 keys x N query-heads is the product K_tile [128 x 128] . Q^T [128 x N]
+// (N = R rows x H_I heads), issued as four tcgen05.mma kind::f8f6f4 of
+// K = 32 into a TMEM accumulator; the epilogue thread that owns a key (TMEM
+// lane) applies ReLU, the weights and the head sum in registers and writes one
+// fp32 score per row.  A persistent CTA per SM walks a balanced contiguous
+// range of (row group, key tile) items; a TMA producer warp streams 16 KB key
+// tiles (two 64-token pages) through a 6-stage ring, an MMA warp issues, and
+// 4 or 8 epilogue warps drain a double-buffered accumulator.
+//
+// CUDA-core path (fp32 or fp8, d_I <= 128, H_I <= 64): one thread per key.
+#include <cuda_fp8.h>
+
+#include "sa_device.cuh"
+#include "sa_internal.h"
+
+namespace sa {
+namespace {
+
+constexpr int kPage = 64;
+constexpr int kTileKeys = 128;
+constexpr int kStages = 6;
+constexpr int kStageBytes = kTileKeys * 128;  // 128 keys x 128 fp8
+constexpr int kMaxRows = 4096;
+
+__device__ __forceinline__ int clamp_vis(const IdxArgs& a, int r) {
+    int n = a.n_visible[r];
+    int cap = a.pages_per_seq * kPage;
+    if (cap > a.scores_ld) cap = static_cast<int>(a.scores_ld);
+    return n < 0 ? 0 : (n > cap ? cap : n);
+}
+
+__device__ __forceinline__ int seq_of(const IdxArgs& a, int r) { return a.seq_of_row ? a.seq_of_row[r] : r; }
+
+__device__ __forceinline__ int page_of(const IdxArgs& a, int seq, int p) {
+    return a.page_table ? a.page_table[static_cast<int64_t>(seq) * a.pages_per_seq + p]
+                        : seq * a.pages_per_seq + p;
+}
+
+// In-place block-wide scan over n ints in shared memory (all threads call).
+// Sum (exclusive, returns total) or max (inclusive).
+template <bool kMax>
+__device__ int block_scan(int* a, int n, int* warp_buf) {
+    const int nt = blockDim.x, tid = threadIdx.x, lane = tid & 31, wid = tid >> 5, nw = nt >> 5;
+    const int per = (n + nt - 1) / nt;
+    const int lo = min(n, tid * per), hi = min(n, lo + per);
+    int acc = kMax ? INT_MIN : 0;
+    for (int i = lo; i < hi; ++i) acc = kMax ? max(acc, a[i]) : acc + a[i];
+    int incl = acc;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl = kMax ? max(incl, v) : incl + v;
+    }
+    if (lane == 31) warp_buf[wid] = incl;
+    __syncthreads();
+    if (tid == 0) {
+        int run = kMax ? INT_MIN : 0;
+        for (int w = 0; w < nw; ++w) {
+            int v = warp_buf[w];
+            warp_buf[w] = run;
+            run = kMax ? max(run, v) : run + v;
+        }
+        warp_buf[nw] = run;
+    }
+    __syncthreads();
+    int excl_t = incl;  // exclusive prefix of this thread's chunk
+    {
+        int up = __shfl_up_sync(0xffffffffu, incl, 1);
+        int base = warp_buf[wid];
+        if (kMax)
+            excl_t = lane == 0 ? base : max(base, up);
+        else
+            excl_t = lane == 0 ? base : base + up;
+    }
+    int total = warp_buf[nw];
+    __syncthreads();
+    int run = excl_t;
+    for (int i = lo; i < hi; ++i) {
+        int v = a[i];
+        if (kMax) {
+            run = max(run, v);
+            a[i] = run;
+        } else {
+            a[i] = run;
+            run += v;
+        }
+    }
+    __syncthreads();
+    return total;
+}
+
+// Walks the (group, tile) items of one CTA in order.
+struct ItemWalk {
+    const int* prefix;  // [G+1] tile prefix
+    int G, item, end, g, t;
+    __device__ bool valid() const { return item < end; }
+    __device__ int tiles(int gg) const { return prefix[gg + 1] - prefix[gg]; }
+    __device__ void start(int begin, int end_) {
+        item = begin;
+        end = end_;
+        // largest g with prefix[g] <= item (and a nonempty group)
+        int lo = 0, hi = G;  // prefix[G] = total > item
+        while (hi - lo > 1) {
+            int mid = (lo + hi) >> 1;
+            if (prefix[mid] <= item) lo = mid; else hi = mid;
+        }
+        g = lo;
+        while (g < G && tiles(g) == 0) ++g;
+        t = item - prefix[g];
+    }
+    __device__ void next() {
+        ++item;
+        if (++t >= tiles(g)) {
+            do { ++g; } while (g < G && tiles(g) == 0);
+            t = 0;
+        }
+    }
+};
+
+template <int NH, int R, int NEPI>
+struct TcCfg {
+    static constexpr int N = R * NH;                     // MMA N (rows x heads)
+    static constexpr int kTmemCols = (2 * N <= 32) ? 32 : (2 * N <= 64 ? 64 : (2 * N <= 128 ? 128 : (2 * N <= 256 ? 256 : 512)));
+    static constexpr int kQBytes = N * 128;
+    static constexpr int kThreads = 32 * (NEPI + 2);
+    // shared layout (offsets from a 1024-aligned base)
+    static constexpr int kOffStages = 0;
+    static constexpr int kOffQ = kOffStages + kStages * kStageBytes;
+    static constexpr int kOffW = kOffQ + 2 * kQBytes;
+    static constexpr int kOffPrefix = kOffW + NEPI * R * NH * 4;
+    static constexpr int kOffGStart = kOffPrefix + (kMaxRows + 1) * 4;
+    static constexpr int kSmemBytes = kOffGStart + (kMaxRows + 1) * 4 + 1024;
+};
+
+template <int NH, int R, int NEPI>
+__global__ void __launch_bounds__(TcCfg<NH, R, NEPI>::kThreads, 1)
+    idx_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
+                  const IdxArgs a) {
+    using C = TcCfg<NH, R, NEPI>;
+    constexpr int N = C::N;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* s_stage = sm + C::kOffStages;
+    uint8_t* s_q = sm + C::kOffQ;
+    float* s_w = reinterpret_cast<float*>(sm + C::kOffW);
+    int* s_prefix = reinterpret_cast<int*>(sm + C::kOffPrefix);
+    int* s_gstart = reinterpret_cast<int*>(sm + C::kOffGStart);
+
+    __shared__ uint64_t bar_full[kStages], bar_empty[kStages], bar_qfull[2], bar_qempty[2], bar_accfull[2],
+        bar_accempty[2], bar_final;
+    __shared__ uint32_t s_tmem;
+    __shared__ int s_abort;
+    __shared__ int s_warpbuf[40];
+    __shared__ int s_G;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    WaitCtx wc{a.err, &s_abort};
+
+    if (tid == 0) {
+        s_abort = 0;
+        for (int i = 0; i < kStages; ++i) {
+            mbar_init(&bar_full[i], 1);
+            mbar_init(&bar_empty[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&bar_qfull[i], 1);
+            mbar_init(&bar_qempty[i], 1);
+            mbar_init(&bar_accfull[i], 1);
+            mbar_init(&bar_accempty[i], NEPI);
+        }
+        mbar_init(&bar_final, 1);
+        fence_mbar_init();
+    }
+    if (warp == NEPI + 1) {
+        tmem_alloc(&s_tmem, C::kTmemCols);
+        tmem_relinquish();
+    }
+    if (warp == NEPI && lane == 0) {
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_q);
+    }
+
+    // ---- group table: consecutive rows of one sequence, at most R per group
+    const int rows = a.rows;
+    int* tmp = reinterpret_cast<int*>(s_stage);  // scratch (stage ring is idle yet)
+    int G;
+    if (R == 1 || a.seq_of_row == nullptr) {
+        G = rows;
+        for (int g = tid; g <= rows; g += blockDim.x) s_gstart[g] = g;
+    } else {
+        int* flag = tmp + kMaxRows;
+        for (int r = tid; r < rows; r += blockDim.x)
+            tmp[r] = (r == 0 || a.seq_of_row[r] != a.seq_of_row[r - 1]) ? r : 0;
+        __syncthreads();
+        block_scan<true>(tmp, rows, s_warpbuf);  // run start of each row
+        for (int r = tid; r < rows; r += blockDim.x) flag[r] = ((r - tmp[r]) % R == 0) ? 1 : 0;
+        __syncthreads();
+        for (int r = tid; r < rows; r += blockDim.x) tmp[r] = flag[r];
+        __syncthreads();
+        G = block_scan<false>(tmp, rows, s_warpbuf);  // group index of group starts
+        for (int r = tid; r < rows; r += blockDim.x)
+            if (flag[r]) s_gstart[tmp[r]] = r;
+        if (tid == 0) s_gstart[G] = rows;
+        __syncthreads();
+    }
+    for (int g = tid; g < G; g += blockDim.x) {
+        int nk = 0;
+        for (int r = s_gstart[g]; r < s_gstart[g + 1]; ++r) nk = max(nk, clamp_vis(a, r));
+        s_prefix[g] = (nk + kTileKeys - 1) / kTileKeys;
+    }
+    __syncthreads();
+    const int total = block_scan<false>(s_prefix, G, s_warpbuf);
+    if (tid == 0) {
+        s_prefix[G] = total;
+        s_G = G;
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = s_tmem;
+
+    const int64_t begin = static_cast<int64_t>(blockIdx.x) * total / gridDim.x;
+    const int64_t end = static_cast<int64_t>(blockIdx.x + 1) * total / gridDim.x;
+    ItemWalk it;
+    it.prefix = s_prefix;
+    it.G = G;
+
+    if (warp == NEPI) {
+        // ------------------------------------------------ TMA producer
+        int stage = 0;
+        uint32_t phase = 0;
+        int gcount = -1, prev_g = -1;
+        int64_t n_issued = 0;
+        if (begin < end) {
+            for (it.start(static_cast<int>(begin), static_cast<int>(end)); it.valid(); it.next()) {
+                const int g = it.g, t = it.t;
+                const int r0 = s_gstart[g];
+                bool ok = true;
+                if (g != prev_g) {
+                    ++gcount;
+                    prev_g = g;
+                    const int qb = gcount & 1;
+                    if (gcount >= 2 && lane == 0) ok = mbar_wait(&bar_qempty[qb], ((gcount >> 1) - 1) & 1, wc, kErrIdxWait | 1);
+                    if (ok && lane == 0) {
+                        mbar_arrive_expect_tx(&bar_qfull[qb], C::kQBytes);
+                        tma_load_2d(s_q + qb * C::kQBytes, &tm_q, &bar_qfull[qb], 0, r0 * NH);
+                    }
+                }
+                if (ok && lane == 0) ok = mbar_wait(&bar_empty[stage], phase ^ 1, wc, kErrIdxWait | 2);
+                if (ok && lane == 0) {
+                    const int seq = seq_of(a, r0);
+                    int nk = 0;
+                    for (int r = r0; r < s_gstart[g + 1]; ++r) nk = max(nk, clamp_vis(a, r));
+                    const int p0 = 2 * t, p1 = 2 * t + 1;
+                    const bool v1 = p1 * kPage < nk;
+                    mbar_arrive_expect_tx(&bar_full[stage], (v1 ? 2 : 1) * (kStageBytes / 2));
+                    uint8_t* dst = s_stage + stage * kStageBytes;
+                    tma_load_2d(dst, &tm_k, &bar_full[stage], 0, page_of(a, seq, p0) * kPage);
+                    if (v1) tma_load_2d(dst + kStageBytes / 2, &tm_k, &bar_full[stage], 0, page_of(a, seq, p1) * kPage);
+                    ++n_issued;
+                }
+                __syncwarp();
+                if (s_abort) break;
+                if (++stage == kStages) {
+                    stage = 0;
+                    phase ^= 1;
+                }
+            }
+        }
+        // drain: every load still in flight lands before the CTA can exit
+        if (lane == 0) {
+            int dummy = 0;
+            WaitCtx dw{a.err, reinterpret_cast<volatile int*>(&dummy)};
+            for (int64_t i = n_issued - kStages; i < n_issued; ++i) {
+                if (i < 0) continue;
+                mbar_wait(&bar_full[i % kStages], static_cast<uint32_t>((i / kStages) & 1), dw, kErrIdxWait | 7);
+            }
+        }
+        __syncwarp();
+    } else if (warp == NEPI + 1) {
+        // ------------------------------------------------ MMA issuer
+        constexpr uint32_t idesc = idesc_f32acc(0, 0, false, false, 128, N);
+        int stage = 0;
+        uint32_t phase = 0;
+        int gcount = -1, prev_g = -1;
+        int64_t acc = 0;
+        if (begin < end) {
+            for (it.start(static_cast<int>(begin), static_cast<int>(end)); it.valid(); it.next()) {
+                bool ok = true;
+                if (it.g != prev_g) {
+                    if (prev_g >= 0 && lane == 0) tc_commit(&bar_qempty[gcount & 1]);
+                    ++gcount;
+                    prev_g = it.g;
+                    if (lane == 0) ok = mbar_wait(&bar_qfull[gcount & 1], (gcount >> 1) & 1, wc, kErrIdxWait | 3);
+                }
+                const int buf = static_cast<int>(acc & 1);
+                if (ok && lane == 0) ok = mbar_wait(&bar_full[stage], phase, wc, kErrIdxWait | 4);
+                if (ok && lane == 0 && acc >= 2)
+                    ok = mbar_wait(&bar_accempty[buf], static_cast<uint32_t>(((acc >> 1) - 1) & 1), wc, kErrIdxWait | 5);
+                if (ok && lane == 0) {
+                    tc_fence_after();
+                    const uint64_t da = sdesc(smem_u32(s_stage + stage * kStageBytes), 16, 1024, kSw128);
+                    const uint64_t db = sdesc(smem_u32(s_q + (gcount & 1) * C::kQBytes), 16, 1024, kSw128);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_f8_ss(tmem + buf * N, da + 2 * kk, db + 2 * kk, idesc, kk > 0 ? 1u : 0u);
+                    tc_commit(&bar_empty[stage]);
+                    tc_commit(&bar_accfull[buf]);
+                }
+                __syncwarp();
+                if (s_abort) break;
+                ++acc;
+                if (++stage == kStages) {
+                    stage = 0;
+                    phase ^= 1;
+                }
+            }
+        }
+        if (lane == 0) {  // all issued MMAs complete before TMEM is released
+            int dummy = 0;
+            WaitCtx dw{a.err, reinterpret_cast<volatile int*>(&dummy)};
+            tc_commit(&bar_final);
+            mbar_wait(&bar_final, 0, dw, kErrIdxWait | 8);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------ epilogue (warps 0..NEPI-1)
+        const int quarter = warp & 3;
+        constexpr int kHalves = NEPI / 4;
+        constexpr int kRowsPerHalf = (R + kHalves - 1) / kHalves;
+        const int half = warp >> 2;
+        int64_t acc = 0;
+        int prev_g = -1;
+        int g_r0 = 0, g_cnt = 0;
+        int nvis[kRowsPerHalf];
+        float* w_own = s_w + warp * R * NH;  // this warp's copy of the group's weights
+        if (begin < end) {
+            for (it.start(static_cast<int>(begin), static_cast<int>(end)); it.valid(); it.next()) {
+                if (it.g != prev_g) {
+                    prev_g = it.g;
+                    g_r0 = s_gstart[it.g];
+                    g_cnt = s_gstart[it.g + 1] - g_r0;
+                    __syncwarp();
+                    for (int i = lane; i < R * NH; i += 32) {
+                        const int gi = i / NH;
+                        w_own[i] = gi < g_cnt ? a.w[static_cast<int64_t>(g_r0 + gi) * NH + (i % NH)] : 0.f;
+                    }
+                    __syncwarp();
+#pragma unroll
+                    for (int j = 0; j < kRowsPerHalf; ++j) {
+                        const int gi = half * kRowsPerHalf + j;
+                        nvis[j] = gi < g_cnt ? clamp_vis(a, g_r0 + gi) : 0;
+                    }
+                }
+                const int buf = static_cast<int>(acc & 1);
+                if (!warp_wait(&bar_accfull[buf], static_cast<uint32_t>((acc >> 1) & 1), wc, kErrIdxWait | 6)) break;
+                tc_fence_after();
+                const int s = it.t * kTileKeys + quarter * 32 + lane;
+#pragma unroll
+                for (int j = 0; j < kRowsPerHalf; ++j) {
+                    const int gi = half * kRowsPerHalf + j;
+                    if (gi < R && gi < g_cnt) {
+                        float sum = 0.f;
+                        const uint32_t col = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + buf * N + gi * NH;
+                        if constexpr (NH < 32) {
+                            uint32_t v[16];
+                            tmem_ld16(col, v);
+                            tmem_ld_wait();
+#pragma unroll
+                            for (int x = 0; x < 16; ++x) sum += w_own[gi * NH + x] * fmaxf(__uint_as_float(v[x]), 0.f);
+                        } else {
+#pragma unroll
+                            for (int c = 0; c < NH; c += 32) {
+                                uint32_t v[32];
+                                tmem_ld32(col + c, v);
+                                tmem_ld_wait();
+#pragma unroll
+                                for (int x = 0; x < 32; ++x)
+                                    sum += w_own[gi * NH + c + x] * fmaxf(__uint_as_float(v[x]), 0.f);
+                            }
+                        }
+                        if (s < nvis[j]) a.scores[static_cast<int64_t>(g_r0 + gi) * a.scores_ld + s] = sum;
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bar_accempty[buf]);
+                ++acc;
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == NEPI + 1) tmem_dealloc(tmem, C::kTmemCols);
+}
+
+// ------------------------------------------------------------ CUDA-core path
+template <typename T>
+__device__ __forceinline__ float4 load4(const T* p);
+template <>
+__device__ __forceinline__ float4 load4<float>(const float* p) {
+    return *reinterpret_cast<const float4*>(p);
+}
+template <>
+__device__ __forceinline__ float4 load4<__nv_fp8_e4m3>(const __nv_fp8_e4m3* p) {
+    const uint32_t u = *reinterpret_cast<const uint32_t*>(p);
+    __nv_fp8_e4m3 b[4];
+    *reinterpret_cast<uint32_t*>(b) = u;
+    return make_float4(float(b[0]), float(b[1]), float(b[2]), float(b[3]));
+}
+
+template <typename T, int NH>
+__global__ void __launch_bounds__(128) idx_cc_kernel(const T* __restrict__ q, const T* __restrict__ kc, const IdxArgs a) {
+    __shared__ float s_q[NH * 128];
+    __shared__ float s_w[NH];
+    const int r = blockIdx.y;
+    const int d_I = a.d_I;
+    for (int i = threadIdx.x; i < NH * d_I; i += blockDim.x) {
+        const int j = i / d_I, d = i % d_I;
+        s_q[j * 128 + d] = j < a.H_I ? float(q[(static_cast<int64_t>(r) * a.H_I + j) * d_I + d]) : 0.f;
+    }
+    for (int j = threadIdx.x; j < NH; j += blockDim.x) s_w[j] = j < a.H_I ? a.w[static_cast<int64_t>(r) * a.H_I + j] : 0.f;
+    __syncthreads();
+    const int nv = clamp_vis(a, r);
+    const int s = blockIdx.x * blockDim.x + threadIdx.x;
+    if (s >= nv) return;
+    const int seq = seq_of(a, r);
+    const int page = page_of(a, seq, s / kPage);
+    if (page < 0 || page >= a.pool_pages) {  // precondition broken: no read outside the pool
+        a.scores[static_cast<int64_t>(r) * a.scores_ld + s] = 0.f;
+        return;
+    }
+    const int64_t row = static_cast<int64_t>(page) * kPage + (s % kPage);
+    const T* kp = kc + row * d_I;
+    float dot[NH];
+#pragma unroll
+    for (int j = 0; j < NH; ++j) dot[j] = 0.f;
+    for (int d = 0; d < d_I; d += 4) {
+        const float4 kv = load4<T>(kp + d);
+#pragma unroll
+        for (int j = 0; j < NH; ++j) {
+            const float* qq = s_q + j * 128 + d;
+            dot[j] += qq[0] * kv.x + qq[1] * kv.y + qq[2] * kv.z + qq[3] * kv.w;
+        }
+    }
+    float sum = 0.f;
+#pragma unroll
+    for (int j = 0; j < NH; ++j) sum += s_w[j] * fmaxf(dot[j], 0.f);
+    a.scores[static_cast<int64_t>(r) * a.scores_ld + s] = sum;
+}
+
+template <typename T, int NH>
+sa_status launch_cc(const void* q, const void* kc, const IdxArgs& a, cudaStream_t st) {
+    const int L = a.pages_per_seq * kPage;
+    dim3 grid((L + 127) / 128, a.rows);
+    idx_cc_kernel<T, NH><<<grid, 128, 0, st>>>(static_cast<const T*>(q), static_cast<const T*>(kc), a);
+    return launch_status(cudaGetLastError());
+}
+
+template <int NH, int R, int NEPI>
+sa_status launch_tc(const void* q, const void* kc, const IdxArgs& a, cudaStream_t st) {
+    using C = TcCfg<NH, R, NEPI>;
+    CUtensorMap tk, tq;
+    // keys: [pool rows][128 bytes]; rows outside the pool read as zero
+    const uint64_t kdims[2] = {128, static_cast<uint64_t>(a.pool_pages) * kPage};
+    const uint64_t kstr[1] = {128};
+    const uint32_t kbox[2] = {128, kPage};
+    if (!encode_tiled(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, kc, kdims, kstr, kbox, CU_TENSOR_MAP_SWIZZLE_128B))
+        return SA_ECUDA;
+    const uint64_t qdims[2] = {128, static_cast<uint64_t>(a.rows) * a.H_I};
+    const uint64_t qstr[1] = {128};
+    const uint32_t qbox[2] = {128, static_cast<uint32_t>(C::N)};
+    if (!encode_tiled(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, q, qdims, qstr, qbox, CU_TENSOR_MAP_SWIZZLE_128B))
+        return SA_ECUDA;
+    auto kern = idx_tc_kernel<NH, R, NEPI>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    if (e != cudaSuccess) return launch_status(e);
+    kern<<<sm_count(), C::kThreads, C::kSmemBytes, st>>>(tk, tq, a);
+    return launch_status(cudaGetLastError());
+}
+
+}  // namespace
+
+sa_status index_scores_tc(const void* q, const void* kc, const IdxArgs& a, cudaStream_t st) {
+    if (a.rows > kMaxRows) return SA_EUNSUPPORTED;
+    const bool grouped = a.seq_of_row != nullptr;
+    switch (a.H_I) {
+        case 16: return grouped ? launch_tc<16, 16, 8>(q, kc, a, st) : launch_tc<16, 1, 4>(q, kc, a, st);
+        case 32: return grouped ? launch_tc<32, 8, 8>(q, kc, a, st) : launch_tc<32, 1, 4>(q, kc, a, st);
+        case 64: return grouped ? launch_tc<64, 4, 8>(q, kc, a, st) : launch_tc<64, 1, 4>(q, kc, a, st);
+        case 128: return grouped ? launch_tc<128, 2, 8>(q, kc, a, st) : launch_tc<128, 1, 4>(q, kc, a, st);
+        default: return SA_EUNSUPPORTED;
+    }
+}
+
+sa_status index_scores_cc(const void* q, const void* kc, sa_dtype dt, const IdxArgs& a, cudaStream_t st) {
+    const int h = a.H_I;
+    if (dt == SA_F32) {
+        if (h <= 4) return launch_cc<float, 4>(q, kc, a, st);
+        if (h <= 16) return launch_cc<float, 16>(q, kc, a, st);
+        if (h <= 64) return launch_cc<float, 64>(q, kc, a, st);
+    } else if (dt == SA_E4M3) {
+        if (h <= 4) return launch_cc<__nv_fp8_e4m3, 4>(q, kc, a, st);
+        if (h <= 16) return launch_cc<__nv_fp8_e4m3, 16>(q, kc, a, st);
+        if (h <= 64) return launch_cc<__nv_fp8_e4m3, 64>(q, kc, a, st);
+    }
+    return SA_EUNSUPPORTED;
+}
+
+}  // namespace sa

@@ -1,0 +1,260 @@
+// sa_api.cu — the C ABI (include/sparse_attn.h): argument checks, then the
+// launches.  Every check happens on the host before anything is launched.
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <mutex>
+
+#include "sa_device.cuh"
+#include "sa_internal.h"
+
+namespace sa {
+namespace {
+
+constexpr int kMaxDevices = 64;
+__device__ int g_error_word;  // one per GPU that loads the library
+int* g_error_ptr[kMaxDevices] = {};
+int g_sm_count[kMaxDevices] = {};
+std::mutex g_mu;
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+int current_device() {
+    int d = 0;
+    if (cudaGetDevice(&d) != cudaSuccess) return -1;
+    return d;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+}  // namespace
+
+sa_status launch_status(cudaError_t e) { return e == cudaSuccess ? SA_OK : SA_ECUDA; }
+
+int* device_error_word() {
+    const int d = current_device();
+    if (d < 0 || d >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_error_ptr[d]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_error_word) != cudaSuccess) return nullptr;
+        g_error_ptr[d] = static_cast<int*>(p);
+    }
+    return g_error_ptr[d];
+}
+
+int sm_count() {
+    const int d = current_device();
+    if (d < 0 || d >= kMaxDevices) return 148;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_sm_count[d]) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, d) != cudaSuccess || n <= 0) n = 148;
+        g_sm_count[d] = n;
+    }
+    return g_sm_count[d];
+}
+
+bool encode_tiled(CUtensorMap* map, CUtensorMapDataType dt, int rank, const void* base, const uint64_t* dims,
+                  const uint64_t* strides_bytes, const uint32_t* box, CUtensorMapSwizzle swz) {
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (!g_encode) {
+            void* fn = nullptr;
+            cudaDriverEntryPointQueryResult q;
+            if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+                q != cudaDriverEntryPointSuccess || !fn)
+                return false;
+            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+        }
+    }
+    cuuint64_t gd[5];
+    cuuint64_t gs[4];
+    cuuint32_t bd[5], es[5];
+    for (int i = 0; i < rank; ++i) {
+        gd[i] = dims[i];
+        bd[i] = box[i];
+        es[i] = 1;
+        if (i + 1 < rank) gs[i] = strides_bytes[i];
+    }
+    const CUresult r = g_encode(map, dt, static_cast<cuuint32_t>(rank), const_cast<void*>(base), gd, gs, bd, es,
+                                CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+}  // namespace sa
+
+using namespace sa;
+
+extern "C" {
+
+const char* sa_status_string(sa_status s) {
+    switch (s) {
+        case SA_OK: return "SA_OK";
+        case SA_EINVAL: return "SA_EINVAL";
+        case SA_EUNSUPPORTED: return "SA_EUNSUPPORTED";
+        case SA_ECUDA: return "SA_ECUDA";
+        case SA_ETIMEOUT: return "SA_ETIMEOUT";
+    }
+    return "SA_UNKNOWN";
+}
+
+int sa_version(void) { return 100; }
+
+sa_status sa_check_device_error(int* code_out, sa_stream_t stream) {
+    if (!code_out) return SA_EINVAL;
+    *code_out = 0;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(st) != cudaSuccess) return SA_ECUDA;
+    int* w = device_error_word();
+    if (!w) return SA_ECUDA;
+    int v = 0;
+    if (cudaMemcpy(&v, w, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return SA_ECUDA;
+    if (v != 0) {
+        const int zero = 0;
+        if (cudaMemcpy(w, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return SA_ECUDA;
+    }
+    *code_out = v;
+    return v ? SA_ETIMEOUT : SA_OK;
+}
+
+sa_status sa_index_scores(const void* q, const float* w, const void* k_cache, int64_t pool_pages, sa_dtype dtype,
+                          const int32_t* page_table, int pages_per_seq, const int32_t* seq_of_row,
+                          const int32_t* n_visible, int rows, int H_I, int d_I, int64_t scores_ld, float* scores,
+                          sa_stream_t stream) {
+    if (rows < 0 || H_I < 1 || d_I < 1 || pages_per_seq < 1 || pool_pages < 1 || scores_ld < 1) return SA_EINVAL;
+    if (rows == 0) return SA_OK;
+    if (!q || !w || !k_cache || !n_visible || !scores) return SA_EINVAL;
+    if (dtype != SA_F32 && dtype != SA_E4M3) return SA_EUNSUPPORTED;
+    if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(w, 4) || !aligned(scores, 4)) return SA_EINVAL;
+    if (pool_pages * 64 > (int64_t(1) << 32)) return SA_EUNSUPPORTED;
+    IdxArgs a;
+    a.w = w;
+    a.page_table = page_table;
+    a.pages_per_seq = pages_per_seq;
+    a.pool_pages = pool_pages;
+    a.seq_of_row = seq_of_row;
+    a.n_visible = n_visible;
+    a.rows = rows;
+    a.H_I = H_I;
+    a.d_I = d_I;
+    a.scores = scores;
+    a.scores_ld = scores_ld;
+    a.err = device_error_word();
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const bool tc_shape = dtype == SA_E4M3 && d_I == 128 && (H_I == 16 || H_I == 32 || H_I == 64 || H_I == 128) &&
+                          rows <= 4096;
+    if (tc_shape) return index_scores_tc(q, k_cache, a, st);
+    if (d_I % 4 != 0 || d_I > 128 || H_I > 64) return SA_EUNSUPPORTED;
+    return index_scores_cc(q, k_cache, dtype, a, st);
+}
+
+sa_status sa_topk_select(const float* scores, int64_t scores_ld, const int32_t* n_valid, int rows, int k,
+                         int32_t* idx_out, sa_stream_t stream) {
+    if (rows < 0 || k < 1 || scores_ld < 1) return SA_EINVAL;
+    if (rows == 0) return SA_OK;
+    if (!scores || !n_valid || !idx_out) return SA_EINVAL;
+    if (!aligned(scores, 16) || scores_ld % 4 != 0 || !aligned(idx_out, 4)) return SA_EINVAL;
+    if (scores_ld > 262144) return SA_EUNSUPPORTED;
+    return topk_select_launch(scores, scores_ld, n_valid, rows, k, idx_out, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t sa_sparse_mla_workspace_size(int rows, int H, int k, int d_c) {
+    if (rows < 1 || H < 1 || k < 1 || d_c < 1) return 0;
+    return mla_workspace_bytes(rows, H, k, d_c, mla_decode_splits(rows, k));
+}
+
+static sa_status mla_common(const void* q_lat, const void* q_rope, const void* c_cache, int64_t c_ld,
+                            const void* kr_cache, int64_t kr_ld, int64_t pool_pages, const int32_t* page_table,
+                            int pages_per_seq, const int32_t* seq_of_row, const int32_t* idx, int rows, int H, int k,
+                            int d_c, int d_R, float scale, float* out, float* lse, MlaArgs* a) {
+    if (rows < 0 || H < 1 || k < 1 || pages_per_seq < 1 || pool_pages < 1 || !std::isfinite(scale)) return SA_EINVAL;
+    if (!q_lat || !q_rope || !c_cache || !kr_cache || !idx || !out) return SA_EINVAL;
+    if (d_c != 512 || d_R != 64 || H > 128) return SA_EUNSUPPORTED;
+    if (c_ld < d_c || kr_ld < d_R || c_ld % 8 != 0 || kr_ld % 8 != 0) return SA_EINVAL;
+    if (!aligned(q_lat, 16) || !aligned(q_rope, 16) || !aligned(c_cache, 16) || !aligned(kr_cache, 16) ||
+        !aligned(out, 16) || !aligned(idx, 4) || (lse && !aligned(lse, 4)))
+        return SA_EINVAL;
+    if (pool_pages * 64 > (int64_t(1) << 32)) return SA_EUNSUPPORTED;
+    a->q_lat = q_lat;
+    a->q_rope = q_rope;
+    a->c_cache = c_cache;
+    a->c_ld = c_ld;
+    a->kr_cache = kr_cache;
+    a->kr_ld = kr_ld;
+    a->page_table = page_table;
+    a->pages_per_seq = pages_per_seq;
+    a->pool_pages = pool_pages;
+    a->seq_of_row = seq_of_row;
+    a->idx = idx;
+    a->rows = rows;
+    a->H = H;
+    a->k = k;
+    a->d_c = d_c;
+    a->d_R = d_R;
+    a->scale = scale;
+    a->out = out;
+    a->lse = lse;
+    a->err = device_error_word();
+    return SA_OK;
+}
+
+sa_status sa_sparse_mla_decode(const void* q_lat, const void* q_rope, const void* c_cache, int64_t c_ld,
+                               const void* kr_cache, int64_t kr_ld, int64_t pool_pages, const int32_t* page_table,
+                               int pages_per_seq, const int32_t* seq_of_row, const int32_t* idx, int rows, int H,
+                               int k, int d_c, int d_R, float scale, float* out, float* lse, void* workspace,
+                               size_t workspace_bytes, sa_stream_t stream) {
+    if (rows == 0) return SA_OK;
+    MlaArgs a;
+    sa_status s = mla_common(q_lat, q_rope, c_cache, c_ld, kr_cache, kr_ld, pool_pages, page_table, pages_per_seq,
+                             seq_of_row, idx, rows, H, k, d_c, d_R, scale, out, lse, &a);
+    if (s != SA_OK) return s;
+    const int ns = mla_decode_splits(rows, k);
+    if (ns > 1 && (!workspace || !aligned(workspace, 256) ||
+                   workspace_bytes < mla_workspace_bytes(rows, H, k, d_c, ns)))
+        return SA_EINVAL;
+    return sparse_mla_launch(a, ns, workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+sa_status sa_sparse_mla_prefill(const void* q_lat, const void* q_rope, const void* c_cache, int64_t c_ld,
+                                const void* kr_cache, int64_t kr_ld, int64_t pool_pages, const int32_t* page_table,
+                                int pages_per_seq, const int32_t* seq_of_row, const int32_t* idx, int rows, int H,
+                                int k, int d_c, int d_R, float scale, float* out, float* lse, sa_stream_t stream) {
+    if (rows == 0) return SA_OK;
+    MlaArgs a;
+    sa_status s = mla_common(q_lat, q_rope, c_cache, c_ld, kr_cache, kr_ld, pool_pages, page_table, pages_per_seq,
+                             seq_of_row, idx, rows, H, k, d_c, d_R, scale, out, lse, &a);
+    if (s != SA_OK) return s;
+    return sparse_mla_launch(a, 1, nullptr, 0, reinterpret_cast<cudaStream_t>(stream));
+}
+
+sa_status sa_block_mean_pool(const void* K, int64_t stride_b, int64_t stride_t, int64_t stride_h, int B, int L,
+                             int H, int D, int block, float* pooled, int64_t pooled_ld, sa_stream_t stream) {
+    if (B < 0 || L < 0 || H < 0 || block < 1) return SA_EINVAL;
+    if (D != 128) return SA_EUNSUPPORTED;
+    if (B == 0 || H == 0 || L / block == 0) return SA_OK;
+    if (!K || !pooled || pooled_ld < L / block) return SA_EINVAL;
+    if (!aligned(K, 8) || !aligned(pooled, 16) || stride_b % 4 || stride_t % 4 || stride_h % 4) return SA_EINVAL;
+    return block_mean_pool_launch(K, stride_b, stride_t, stride_h, B, L, H, D, block, pooled, pooled_ld,
+                                  reinterpret_cast<cudaStream_t>(stream));
+}
+
+sa_status sa_block_sparse_attn(const void* q, const float* pooled, int64_t pooled_ld, const void* K, const void* V,
+                               int64_t stride_b, int64_t stride_t, int64_t stride_h, int B, int H, int D, int L,
+                               int block, int top_blocks, int sink_blocks, int window, float scale, float* out,
+                               int32_t* sel_blocks, sa_stream_t stream) {
+    if (B < 0 || H < 0 || L < 0 || block < 1 || top_blocks < 0 || sink_blocks < 0 || window < 0 ||
+        !std::isfinite(scale))
+        return SA_EINVAL;
+    if (D != 128 || block != 64 || top_blocks > 64 || L / block > 4096) return SA_EUNSUPPORTED;
+    if (B == 0 || H == 0) return SA_OK;
+    if (!q || !K || !V || !out || (L / block > 0 && !pooled) || pooled_ld < L / block) return SA_EINVAL;
+    if (!aligned(q, 2) || !aligned(K, 8) || !aligned(V, 8) || !aligned(out, 4) || (pooled && !aligned(pooled, 16)) ||
+        stride_b % 4 || stride_t % 4 || stride_h % 4)
+        return SA_EINVAL;
+    return block_sparse_launch(q, pooled, pooled_ld, K, V, stride_b, stride_t, stride_h, B, H, D, L, block,
+                               top_blocks, sink_blocks, window, scale, out, sel_blocks,
+                               reinterpret_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

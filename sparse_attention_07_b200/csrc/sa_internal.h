@@ -1,0 +1,73 @@
+// sa_internal.h — host-side declarations shared by the library's translation
+// units (launchers and helpers behind the C ABI in include/sparse_attn.h).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "sparse_attn.h"
+
+namespace sa {
+
+// Device address of this GPU's error word (kernels record wait timeouts here).
+int* device_error_word();
+// Number of SMs of the current device (cached).
+int sm_count();
+// Tensor-map encoder from the driver, fetched once through the runtime.
+bool encode_tiled(CUtensorMap* map, CUtensorMapDataType dt, int rank, const void* base, const uint64_t* dims,
+                  const uint64_t* strides_bytes, const uint32_t* box, CUtensorMapSwizzle swz);
+sa_status launch_status(cudaError_t e);
+
+struct IdxArgs {
+    const float* w;
+    const int32_t* page_table;
+    int pages_per_seq;
+    int64_t pool_pages;
+    const int32_t* seq_of_row;
+    const int32_t* n_visible;
+    int rows;
+    int H_I;
+    int d_I;
+    float* scores;
+    int64_t scores_ld;
+    int* err;
+};
+
+sa_status index_scores_tc(const void* q, const void* k_cache, const IdxArgs& a, cudaStream_t st);
+sa_status index_scores_cc(const void* q, const void* k_cache, sa_dtype dt, const IdxArgs& a, cudaStream_t st);
+
+sa_status topk_select_launch(const float* scores, int64_t ld, const int32_t* n_valid, int rows, int k,
+                             int32_t* idx_out, cudaStream_t st);
+
+struct MlaArgs {
+    const void* q_lat;
+    const void* q_rope;
+    const void* c_cache;
+    int64_t c_ld;
+    const void* kr_cache;
+    int64_t kr_ld;
+    const int32_t* page_table;
+    int pages_per_seq;
+    int64_t pool_pages;
+    const int32_t* seq_of_row;
+    const int32_t* idx;
+    int rows, H, k, d_c, d_R;
+    float scale;
+    float* out;
+    float* lse;
+    int* err;
+};
+
+size_t mla_workspace_bytes(int rows, int H, int k, int d_c, int nsplit);
+int mla_decode_splits(int rows, int k);
+sa_status sparse_mla_launch(const MlaArgs& a, int nsplit, void* ws, size_t ws_bytes, cudaStream_t st);
+
+sa_status block_mean_pool_launch(const void* K, int64_t sb, int64_t st_, int64_t sh, int B, int L, int H, int D,
+                                 int block, float* pooled, int64_t pooled_ld, cudaStream_t st);
+sa_status block_sparse_launch(const void* q, const float* pooled, int64_t pooled_ld, const void* K, const void* V,
+                              int64_t sb, int64_t st_, int64_t sh, int B, int H, int D, int L, int block,
+                              int top_blocks, int sink_blocks, int window, float scale, float* out,
+                              int32_t* sel_blocks, cudaStream_t st);
+
+}  // namespace sa

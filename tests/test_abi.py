@@ -1,0 +1,138 @@
+"""C-ABI checks that need no GPU: the library loads, exports every function
+include/sparse_attn.h declares, and rejects bad arguments on the host before
+launching anything (no pointer is dereferenced, no CUDA call is made)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import sparse_attention_07_b200 as sa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sparse_attn.h")
+
+FAKE = ctypes.c_void_p(0x1000)      # 16-byte aligned, never dereferenced on these paths
+MISALIGNED = ctypes.c_void_p(0x1004)
+
+
+@pytest.fixture(scope="module")
+def L():
+    from sparse_attention_07_b200 import build
+    build.build()
+    return sa.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(sa_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_hot_path_calls():
+    names = declared_functions()
+    for n in ("sa_index_scores", "sa_topk_select", "sa_sparse_mla_decode", "sa_sparse_mla_prefill",
+              "sa_block_sparse_attn", "sa_block_mean_pool"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    missing = [n for n in declared_functions() if not hasattr(L, n)]
+    assert not missing, missing
+    assert set(declared_functions()) <= set(sa.EXPORTS)
+
+
+def test_version_and_status_strings(L):
+    assert L.sa_version() == 100
+    assert L.sa_status_string(sa.SA_EINVAL) == b"SA_EINVAL"
+    assert L.sa_status_string(sa.SA_ETIMEOUT) == b"SA_ETIMEOUT"
+
+
+def test_index_scores_validation(L):
+    f = L.sa_index_scores
+    good = dict(q=FAKE, w=FAKE, k=FAKE, pool=4, dt=sa.SA_E4M3, pt=None, pps=4, sor=None, nv=FAKE,
+                rows=2, H_I=64, d_I=128, ld=256, out=FAKE)
+
+    def call(**kw):
+        a = {**good, **kw}
+        return f(a["q"], a["w"], a["k"], a["pool"], a["dt"], a["pt"], a["pps"], a["sor"], a["nv"], a["rows"],
+                 a["H_I"], a["d_I"], a["ld"], a["out"], None)
+
+    assert call(rows=0) == sa.SA_OK                 # nothing to do, nothing launched
+    assert call(rows=-1) == sa.SA_EINVAL
+    assert call(H_I=0) == sa.SA_EINVAL
+    assert call(pps=0) == sa.SA_EINVAL
+    assert call(pool=0) == sa.SA_EINVAL
+    assert call(q=None) == sa.SA_EINVAL
+    assert call(nv=None) == sa.SA_EINVAL
+    assert call(q=MISALIGNED) == sa.SA_EINVAL
+    assert call(dt=sa.SA_BF16) == sa.SA_EUNSUPPORTED
+    assert call(dt=sa.SA_F32, d_I=130) == sa.SA_EUNSUPPORTED   # not a multiple of 4
+    assert call(dt=sa.SA_F32, H_I=65) == sa.SA_EUNSUPPORTED
+    assert call(pool=(1 << 27)) == sa.SA_EUNSUPPORTED           # pool rows beyond a tensor map's reach
+
+
+def test_topk_validation(L):
+    f = L.sa_topk_select
+    assert f(FAKE, 1024, FAKE, 0, 8, FAKE, None) == sa.SA_OK
+    assert f(FAKE, 1024, FAKE, 2, 0, FAKE, None) == sa.SA_EINVAL
+    assert f(FAKE, 1024, FAKE, -1, 8, FAKE, None) == sa.SA_EINVAL
+    assert f(None, 1024, FAKE, 2, 8, FAKE, None) == sa.SA_EINVAL
+    assert f(FAKE, 1022, FAKE, 2, 8, FAKE, None) == sa.SA_EINVAL          # row stride not 16-byte aligned
+    assert f(MISALIGNED, 1024, FAKE, 2, 8, FAKE, None) == sa.SA_EINVAL
+    assert f(FAKE, 262148, FAKE, 2, 8, FAKE, None) == sa.SA_EUNSUPPORTED  # row longer than the cluster holds
+
+
+def _mla(L, fn, **kw):
+    a = dict(ql=FAKE, qr=FAKE, c=FAKE, cld=512, kr=FAKE, krld=64, pool=4, pt=None, pps=4, sor=None, idx=FAKE,
+             rows=2, H=128, k=2048, dc=512, dR=64, scale=0.07, out=FAKE, lse=None)
+    a.update(kw)
+    args = [a["ql"], a["qr"], a["c"], a["cld"], a["kr"], a["krld"], a["pool"], a["pt"], a["pps"], a["sor"],
+            a["idx"], a["rows"], a["H"], a["k"], a["dc"], a["dR"], a["scale"], a["out"], a["lse"]]
+    if fn == "decode":
+        return L.sa_sparse_mla_decode(*args, None, 0, None)
+    return L.sa_sparse_mla_prefill(*args, None)
+
+
+@pytest.mark.parametrize("fn", ["decode", "prefill"])
+def test_sparse_mla_validation(L, fn):
+    assert _mla(L, fn, rows=0) == sa.SA_OK
+    assert _mla(L, fn, k=0) == sa.SA_EINVAL
+    assert _mla(L, fn, H=0) == sa.SA_EINVAL
+    assert _mla(L, fn, idx=None) == sa.SA_EINVAL
+    assert _mla(L, fn, scale=float("nan")) == sa.SA_EINVAL
+    assert _mla(L, fn, dc=256) == sa.SA_EUNSUPPORTED
+    assert _mla(L, fn, dR=32) == sa.SA_EUNSUPPORTED
+    assert _mla(L, fn, H=129) == sa.SA_EUNSUPPORTED
+    assert _mla(L, fn, cld=520 + 4) == sa.SA_EINVAL            # row stride not 16-byte aligned
+    assert _mla(L, fn, c=MISALIGNED) == sa.SA_EINVAL
+    assert _mla(L, fn, cld=256) == sa.SA_EINVAL                # stride shorter than a row
+
+
+def test_block_validation(L):
+    f = L.sa_block_sparse_attn
+    args = dict(q=FAKE, pooled=FAKE, pld=2048, K=FAKE, V=FAKE, sb=8, st=8, sh=128, B=2, H=4, D=128, L=131072,
+                block=64, top=16, sink=1, win=512, scale=0.088, out=FAKE, sel=None)
+
+    def call(**kw):
+        a = {**args, **kw}
+        return f(a["q"], a["pooled"], a["pld"], a["K"], a["V"], a["sb"], a["st"], a["sh"], a["B"], a["H"], a["D"],
+                 a["L"], a["block"], a["top"], a["sink"], a["win"], a["scale"], a["out"], a["sel"], None)
+
+    assert call(B=0) == sa.SA_OK
+    assert call(D=64) == sa.SA_EUNSUPPORTED
+    assert call(block=128) == sa.SA_EUNSUPPORTED
+    assert call(top=65) == sa.SA_EUNSUPPORTED
+    assert call(L=64 * 4097) == sa.SA_EUNSUPPORTED
+    assert call(top=-1) == sa.SA_EINVAL
+    assert call(pld=100) == sa.SA_EINVAL
+    assert call(st=6) == sa.SA_EINVAL
+    assert call(K=None) == sa.SA_EINVAL
+    g = L.sa_block_mean_pool
+    assert g(FAKE, 8, 8, 128, 2, 1000, 4, 64, 64, FAKE, 15, None) == sa.SA_EUNSUPPORTED
+    assert g(FAKE, 8, 8, 128, 2, 1000, 4, 128, 64, FAKE, 10, None) == sa.SA_EINVAL   # pooled too short
+    assert g(FAKE, 8, 8, 128, 2, 1000, 4, 128, 0, FAKE, 15, None) == sa.SA_EINVAL
+
+
+def test_check_device_error_rejects_null(L):
+    assert L.sa_check_device_error(None, None) == sa.SA_EINVAL

@@ -1,0 +1,115 @@
+"""GPU parity: lightning indexer (bit-exact on integer inputs) and Top-K
+(bit-exact index sets), against the fp64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import sparse_attention_07_b200 as sa
+import workloads as W
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _oracle_scores(inp, rows):
+    return oracle.dsa_step(inp, rows)["scores"]
+
+
+def _check_scores(inp, scores, rows=None):
+    cfg = inp["cfg"]
+    rows = list(range(cfg.rows)) if rows is None else rows
+    ref = _oracle_scores(inp, rows)
+    nv = inp["n_visible"].cpu().numpy()
+    for i, r in enumerate(rows):
+        g = scores[r, : nv[r]].double().cpu().numpy()
+        assert np.array_equal(g, ref[i, : nv[r]]), f"row {r} differs"
+
+
+def test_indexer_cuda_core_tiny():
+    """fp32 inputs, H^I=4, d^I=64 (the tiny workload, full size)."""
+    inp = W.dsa_inputs(W.TINY, DEV)
+    scores = sa.index_scores(inp["q_idx"], inp["w"], inp["k_idx_cache"], inp["n_visible"], W.TINY.pages_per_seq)
+    _check_scores(inp, scores)
+    assert sa.check_device_error() == 0
+
+
+@pytest.mark.parametrize("paged", [False, True])
+@pytest.mark.parametrize("H_I", [64, 16, 32])
+def test_indexer_tensor_core_decode(paged, H_I):
+    """fp8 e4m3, d^I=128: ragged lengths (1, a page, partial tiles, several tiles)."""
+    cfg = W.small_dsa(W.LONG, n_seqs=6, rows=6, lens=(1, 63, 64, 129, 1000, 3001), H_I=H_I, topk=64, H=8,
+                      paged=paged)
+    inp = W.dsa_inputs(cfg, DEV, seed=11 + H_I)
+    scores = sa.index_scores(inp["q_idx"], inp["w"], inp["k_idx_cache"], inp["n_visible"], cfg.pages_per_seq,
+                             page_table=inp["page_table"])
+    torch.cuda.synchronize()
+    _check_scores(inp, scores)
+    assert sa.check_device_error() == 0
+
+
+def test_indexer_tensor_core_grouped_rows():
+    """Several query rows per sequence (prefill-style groups of 4 rows, runs
+    that do not start on a group boundary, one row alone)."""
+    cfg = W.small_dsa(W.LONG, n_seqs=3, lens=(700, 900, 300), rows=9, topk=64, H=8, paged=True)
+    inp = W.dsa_inputs(cfg, DEV, seed=5)
+    inp["seq_of_row"] = torch.tensor([0, 0, 0, 1, 1, 1, 1, 1, 2], dtype=torch.int32, device=DEV)
+    inp["n_visible"] = torch.tensor([650, 651, 700, 1, 64, 500, 899, 900, 300], dtype=torch.int32, device=DEV)
+    scores = sa.index_scores(inp["q_idx"], inp["w"], inp["k_idx_cache"], inp["n_visible"], cfg.pages_per_seq,
+                             page_table=inp["page_table"], seq_of_row=inp["seq_of_row"])
+    torch.cuda.synchronize()
+    _check_scores(inp, scores)
+    assert sa.check_device_error() == 0
+
+
+def test_indexer_cuda_core_fp8_small_dim():
+    cfg = W.small_dsa(W.LONG, n_seqs=2, rows=2, lens=(333, 70), d_I=64, H_I=8, topk=16, H=8)
+    inp = W.dsa_inputs(cfg, DEV, seed=3)
+    scores = sa.index_scores(inp["q_idx"], inp["w"], inp["k_idx_cache"], inp["n_visible"], cfg.pages_per_seq)
+    _check_scores(inp, scores)
+    assert sa.check_device_error() == 0
+
+
+def _topk_case(rows, n, k, seed, lo=-3, hi=3, ld=None):
+    g = torch.Generator(device=DEV)
+    g.manual_seed(seed)
+    ld = ld or ((max(n) + 3) // 4 * 4)
+    s = torch.randint(lo, hi + 1, (rows, ld), generator=g, device=DEV).float()
+    nv = torch.tensor(n, dtype=torch.int32, device=DEV)
+    got = sa.topk_select(s, nv, k).cpu().numpy()
+    want = oracle.topk(s.double().cpu().numpy(), np.array(n), k)
+    assert np.array_equal(got, want)
+    assert sa.check_device_error() == 0
+
+
+@pytest.mark.parametrize("seed", [0, 1])
+def test_topk_ties_small(seed):
+    _topk_case(6, [0, 1, 127, 128, 129, 5000], 128, seed)
+
+
+def test_topk_ties_long_rows():
+    _topk_case(4, [131072, 32768, 8193, 2049], 2048, 7)
+
+
+def test_topk_wide_value_range():
+    """Distinct-ish values spread over many exponents, including negatives."""
+    g = torch.Generator(device=DEV)
+    g.manual_seed(3)
+    s = (torch.randn(3, 40000, generator=g, device=DEV) * torch.exp(torch.randn(3, 40000, generator=g, device=DEV) * 4))
+    nv = torch.tensor([40000, 39999, 12345], dtype=torch.int32, device=DEV)
+    got = sa.topk_select(s, nv, 2048).cpu().numpy()
+    want = oracle.topk(s.double().cpu().numpy(), nv.cpu().numpy(), 2048)
+    assert np.array_equal(got, want)
+
+
+def test_topk_all_equal_and_signed_zero():
+    s = torch.zeros(2, 4096, device=DEV)
+    s[1, ::2] = -0.0
+    nv = torch.tensor([4096, 4000], dtype=torch.int32, device=DEV)
+    got = sa.topk_select(s, nv, 300).cpu().numpy()
+    assert (got == np.arange(300)).all()
+    assert sa.check_device_error() == 0
+
+
+def test_topk_max_row_length():
+    _topk_case(1, [262144], 2048, 9, lo=-100, hi=100)
