@@ -166,6 +166,42 @@ sa_status sa_sparse_mla_prefill(const void* q_lat, const void* q_rope,
                                 float* out, float* lse, sa_stream_t stream);
 
 /*
+ * Sparse MLA decode for callers that cannot allocate device memory.  The
+ * pages have no counterpart of this call: it is a deployment convenience.
+ *
+ * Some callers have no allocator to hand the library a workspace: code that
+ * runs where cudaMalloc is not allowed or not wanted (inside a host callback
+ * or a custom memory manager that owns every byte of the GPU, plugins of a
+ * framework that only passes tensors in and out).  This call computes exactly
+ * what sa_sparse_mla_decode computes, with the same arguments minus the
+ * workspace, and keeps the split-key partial states in a static device array
+ * of SA_STATIC_SCRATCH_BYTES that the library owns.  It calls no cudaMalloc,
+ * cudaFree or allocating library routine.
+ *
+ *  - Every GPU that loads the library holds that array until the process exits.
+ *  - The first call on a device looks up the array's device address (with
+ *    that device current) and caches it; make that first call before any
+ *    stream capture begins.
+ *  - Shapes whose partial states need more than SA_STATIC_SCRATCH_BYTES
+ *    (sa_sparse_mla_workspace_size(rows, H, k, d_c) > SA_STATIC_SCRATCH_BYTES)
+ *    return SA_EUNSUPPORTED and launch nothing; use sa_sparse_mla_decode with
+ *    a caller workspace for those.
+ *  - All calls share the one array.  Calls that may overlap on the GPU (on
+ *    different streams, or on different host threads without ordering)
+ *    race on it and give undefined outputs; order them on one stream.  Every
+ *    byte a call reads from the array was written earlier in the same call,
+ *    so nothing left by a previous call leaks into a result.
+ */
+#define SA_STATIC_SCRATCH_BYTES ((size_t)16 << 20)
+
+sa_status sa_sparse_mla_decode_static(const void* q_lat, const void* q_rope,
+                                      const void* c_cache, int64_t c_ld, const void* kr_cache, int64_t kr_ld,
+                                      int64_t pool_pages, const int32_t* page_table, int pages_per_seq,
+                                      const int32_t* seq_of_row,
+                                      const int32_t* idx, int rows, int H, int k, int d_c, int d_R, float scale,
+                                      float* out, float* lse, sa_stream_t stream);
+
+/*
  * Mean-pooled block keys ([Ch11] §12.6, k_rep = k_blocks.mean(1)):
  *   pooled[b][h][n][d] = (1/block) * sum_{i<block} K[b][n*block+i][h][d]
  * for every complete block n < L / block.

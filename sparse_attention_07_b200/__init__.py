@@ -26,8 +26,12 @@ SA_F32, SA_E4M3, SA_BF16 = range(3)
 EXPORTS = (
     "sa_status_string", "sa_version", "sa_check_device_error", "sa_index_scores", "sa_topk_select",
     "sa_sparse_mla_workspace_size", "sa_sparse_mla_decode", "sa_sparse_mla_prefill",
-    "sa_block_mean_pool", "sa_block_sparse_attn",
+    "sa_block_mean_pool", "sa_block_sparse_attn", "sa_sparse_mla_decode_static",
 )
+
+# Size of the library's static device array behind sparse_mla_decode_static
+# (SA_STATIC_SCRATCH_BYTES in include/sparse_attn.h).
+STATIC_SCRATCH_BYTES = 16 << 20
 
 
 class SparseAttnError(RuntimeError):
@@ -55,6 +59,7 @@ def lib():
         L.sa_sparse_mla_workspace_size.argtypes = [I, I, I, I]
         L.sa_sparse_mla_decode.argtypes = [P, P, P, I64, P, I64, I64, P, I, P, P, I, I, I, I, I, F, P, P, P, SZ, P]
         L.sa_sparse_mla_prefill.argtypes = [P, P, P, I64, P, I64, I64, P, I, P, P, I, I, I, I, I, F, P, P, P]
+        L.sa_sparse_mla_decode_static.argtypes = [P, P, P, I64, P, I64, I64, P, I, P, P, I, I, I, I, I, F, P, P, P]
         L.sa_block_mean_pool.argtypes = [P, I64, I64, I64, I, I, I, I, I, P, I64, P]
         L.sa_block_sparse_attn.argtypes = [P, P, I64, P, P, I64, I64, I64, I, I, I, I, I, I, I, I, F, P, P, P]
         for name in EXPORTS:
@@ -156,6 +161,27 @@ def sparse_mla_prefill(q_lat, q_rope, c_cache, kr_cache, idx, scale: float, page
                                      kr_cache.stride(0), pool_pages, _p(page_table), pages_per_seq, _p(seq_of_row),
                                      _p(idx), rows, H, k, d_c, d_R, float(scale), _p(out), _p(lse), _stream())
     _check("sa_sparse_mla_prefill", st)
+    return out
+
+
+def sparse_mla_decode_static(q_lat, q_rope, c_cache, kr_cache, idx, scale: float, pages_per_seq: int,
+                             page_table=None, seq_of_row=None, out=None, lse=None):
+    """sparse_mla_decode without a workspace: for callers that cannot allocate
+    device memory, the split-key partial states go to the library's static
+    device array (STATIC_SCRATCH_BYTES).  Calls share that array, so calls that
+    may overlap on the GPU must be ordered on one stream.  ``out`` and ``lse``
+    can be passed in so that the call itself allocates nothing."""
+    rows, H, d_c, d_R, k, out, lse, pool_pages = _mla_args(q_lat, q_rope, c_cache, kr_cache, idx, out, lse)
+    need = sparse_mla_workspace_size(rows, H, k, d_c)
+    if need > STATIC_SCRATCH_BYTES:
+        raise ValueError(f"sparse_mla_decode_static: {rows} rows x {H} heads x k={k} need {need} bytes of "
+                         f"split-key state, the static array holds {STATIC_SCRATCH_BYTES}; "
+                         "use sparse_mla_decode with a workspace")
+    st = lib().sa_sparse_mla_decode_static(_p(q_lat), _p(q_rope), _p(c_cache), c_cache.stride(0), _p(kr_cache),
+                                           kr_cache.stride(0), pool_pages, _p(page_table), pages_per_seq,
+                                           _p(seq_of_row), _p(idx), rows, H, k, d_c, d_R, float(scale), _p(out),
+                                           _p(lse), _stream())
+    _check("sa_sparse_mla_decode_static", st)
     return out
 
 

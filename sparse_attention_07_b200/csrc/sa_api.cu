@@ -228,6 +228,53 @@ sa_status sa_sparse_mla_prefill(const void* q_lat, const void* q_rope, const voi
     return sparse_mla_launch(a, 1, nullptr, 0, reinterpret_cast<cudaStream_t>(stream));
 }
 
+}  // extern "C"
+
+// ------------------------------------------------ decode without a caller workspace
+namespace {
+
+// Split-key partial states of sa_sparse_mla_decode_static live here; every
+// GPU that loads the library holds this array until the process exits.
+static __device__ __align__(256) unsigned char g_static_scratch[SA_STATIC_SCRATCH_BYTES];
+void* g_static_scratch_ptr[kMaxDevices] = {};
+
+// Device address of the array on the current device.  The array's name in
+// host code is only a host-side stand-in, so the address is looked up once per
+// device, with that device current, and cached.
+void* static_scratch() {
+    const int d = current_device();
+    if (d < 0 || d >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_static_scratch_ptr[d]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || p == nullptr) return nullptr;
+        g_static_scratch_ptr[d] = p;
+    }
+    return g_static_scratch_ptr[d];
+}
+
+}  // namespace
+
+extern "C" {
+
+sa_status sa_sparse_mla_decode_static(const void* q_lat, const void* q_rope, const void* c_cache, int64_t c_ld,
+                                      const void* kr_cache, int64_t kr_ld, int64_t pool_pages,
+                                      const int32_t* page_table, int pages_per_seq, const int32_t* seq_of_row,
+                                      const int32_t* idx, int rows, int H, int k, int d_c, int d_R, float scale,
+                                      float* out, float* lse, sa_stream_t stream) {
+    if (rows == 0) return SA_OK;
+    MlaArgs a;
+    sa_status s = mla_common(q_lat, q_rope, c_cache, c_ld, kr_cache, kr_ld, pool_pages, page_table, pages_per_seq,
+                             seq_of_row, idx, rows, H, k, d_c, d_R, scale, out, lse, &a);
+    if (s != SA_OK) return s;
+    const int ns = mla_decode_splits(rows, k);
+    const size_t need = mla_workspace_bytes(rows, H, k, d_c, ns);
+    if (need > SA_STATIC_SCRATCH_BYTES) return SA_EUNSUPPORTED;  // checked before any CUDA call
+    void* ws = nullptr;
+    if (need > 0 && (ws = static_scratch()) == nullptr) return SA_ECUDA;
+    return sparse_mla_launch(a, ns, ws, SA_STATIC_SCRATCH_BYTES, reinterpret_cast<cudaStream_t>(stream));
+}
+
 sa_status sa_block_mean_pool(const void* K, int64_t stride_b, int64_t stride_t, int64_t stride_h, int B, int L,
                              int H, int D, int block, float* pooled, int64_t pooled_ld, sa_stream_t stream) {
     if (B < 0 || L < 0 || H < 0 || block < 1) return SA_EINVAL;
