@@ -127,7 +127,7 @@ sa_status sa_index_scores(const void* q, const float* w, const void* k_cache, in
     if (!q || !w || !k_cache || !n_visible || !scores) return SA_EINVAL;
     if (dtype != SA_F32 && dtype != SA_E4M3) return SA_EUNSUPPORTED;
     if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(w, 4) || !aligned(scores, 4)) return SA_EINVAL;
-    if (pool_pages * 64 > (int64_t(1) << 32)) return SA_EUNSUPPORTED;
+    if (pool_pages * 64 > (int64_t(1) << 31)) return SA_EUNSUPPORTED;
     IdxArgs a;
     a.w = w;
     a.page_table = page_table;
@@ -175,7 +175,7 @@ static sa_status mla_common(const void* q_lat, const void* q_rope, const void* c
     if (!aligned(q_lat, 16) || !aligned(q_rope, 16) || !aligned(c_cache, 16) || !aligned(kr_cache, 16) ||
         !aligned(out, 16) || !aligned(idx, 4) || (lse && !aligned(lse, 4)))
         return SA_EINVAL;
-    if (pool_pages * 64 > (int64_t(1) << 32)) return SA_EUNSUPPORTED;
+    if (pool_pages * 64 > (int64_t(1) << 31)) return SA_EUNSUPPORTED;
     a->q_lat = q_lat;
     a->q_rope = q_rope;
     a->c_cache = c_cache;

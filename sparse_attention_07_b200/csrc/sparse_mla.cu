@@ -9,20 +9,31 @@
 //
 // Design (one cluster of two CTAs per (row, key split)):
 //  * The 576-wide score contraction is split across the pair: CTA 0 owns latent
-//    dims 0..255, CTA 1 owns dims 256..511 plus the 64 RoPE dims.  Each CTA
-//    keeps its slice of the 128-head query in shared memory (A operand,
-//    K-major, 128B swizzle) and gathers only its slice of every selected row
-//    with TMA tile::gather4 (4 rows x 128 B per instruction) into a 4-stage ring.
-//  * Per 32-key tile, tcgen05.mma (M=128 heads, N=32 keys, K=16) forms the
-//    CTA's partial scores in TMEM; the softmax warps (thread = head) read them,
-//    swap them with the partner through distributed shared memory and add, so
-//    both CTAs hold identical full scores and identical probabilities.
-//  * Each CTA then aggregates its own 256 latent dims: O[128 x 256] (+)= P . V
-//    with P (bf16, interleaved K-major) from shared memory and V = the gathered
-//    latent slice read MN-major — the tile gathered for the scores is reused,
-//    so every selected row is read from memory exactly once.
-//  * Online softmax in base 2 with a lazy reference: O in TMEM is rescaled
-//    only when a tile's maximum exceeds the reference by more than 2^8.
+//    dims 0..255, CTA 1 owns dims 256..511 plus the 64 RoPE dims.  Two
+//    producer warps gather only the CTA's slice of every selected row with
+//    16-byte cp.async (one warp instruction per 512-byte row slice, written in
+//    the 128-byte swizzled layout the tensor cores read) into a 3-stage ring of
+//    64-key tiles; padded slots are zero-filled without a read.  Rows of the
+//    tile kPrefetch tiles ahead are prefetched into L2, so the ring only has to
+//    cover L2 latency.
+//  * The CTA's slice of the 128-head query sits in tensor memory and is the A
+//    operand of the score MMAs (M=128 heads, N=64 keys, the smallest N at which
+//    an MMA is not dominated by its fixed issue cost).
+//  * Four exchange warps copy each tile's partial scores from TMEM to shared
+//    memory and ship them to the partner in one bulk copy that completes
+//    transaction bytes on the partner's barrier (distributed shared memory is
+//    the narrowest link of this kernel, so the copy runs off the softmax path);
+//    the partner's softmax frees the receive buffer with a remote arrive.
+//  * Eight softmax warps: thread = (head = TMEM lane, half of the tile's keys).
+//    A pair of warps shares a head range; the two halves swap their tile maxima
+//    in shared memory, so both apply the same reference.  Online base-2
+//    softmax; O is rescaled only when a tile's maximum exceeds the reference by
+//    more than 2^8.  P goes back to TMEM as bf16; both CTAs hold identical
+//    scores and probabilities.
+//  * O[128 x 256] (+)= P . V on the tensor cores with P from TMEM and V = the
+//    gathered latent slice read MN-major: the tile gathered for the scores is
+//    reused, so every selected row is read from memory once, and each CTA
+//    aggregates its own 256 latent dims.
 //  * Rows with few queries split their keys over several clusters; partial
 //    (O, m, l) states go to a workspace and a combine kernel merges them.
 #include "sa_device.cuh"
@@ -32,22 +43,34 @@ namespace sa {
 namespace {
 
 constexpr int kPage = 64;
-constexpr int kNK = 32;          // keys per tile
-constexpr int kStages = 4;
-constexpr int kBlkQ = 128 * 128;  // one 64-dim slice of the 128-head query (bytes)
-constexpr int kBlkK = kNK * 128;  // one 64-dim slice of a 32-key tile (bytes)
-constexpr int kMaxBlk = 5;
-constexpr int kOffQ = 0;
-constexpr int kOffStage = kOffQ + kMaxBlk * kBlkQ;
-constexpr int kOffX = kOffStage + kStages * kMaxBlk * kBlkK;
-constexpr int kXBytes = 128 * kNK * 4;
-constexpr int kOffP = kOffX + 2 * kXBytes;
-constexpr int kPBytes = 128 * kNK * 2;
-constexpr int kSmem = kOffP + 2 * kPBytes + 1024;
-constexpr int kThreads = 192;
+constexpr int kNK = 64;           // keys per tile
+constexpr int kHalf = kNK / 2;    // keys per softmax thread
+constexpr int kStages = 3;
+constexpr int kPrefetch = 4;      // tiles prefetched into L2 ahead of the copy
+constexpr int kBlkK = kNK * 128;  // one 64-dim slice of a tile (bytes)
+constexpr int kMaxBlk = 5;        // 64-dim slices per CTA (CTA 1: 4 latent + 1 RoPE)
+constexpr int kStageBytes = kMaxBlk * kBlkK;
+constexpr int kXBytes = 128 * kNK * 4;  // one tile of partial scores (128 heads x 64 keys fp32)
+constexpr int kOffStage = 0;
+constexpr int kOffX = kOffStage + kStages * kStageBytes;  // partner's halves, 2 buffers
+constexpr int kOffL = kOffX + 2 * kXBytes;                // this CTA's half, staged for the copy
+constexpr int kSmem = kOffL + kXBytes + 1024;
+constexpr int kSmxWarps = 8;
+constexpr int kXchgWarp0 = kSmxWarps;
+constexpr int kProdWarp0 = kXchgWarp0 + 4;
+constexpr int kProdWarps = 2;
+constexpr int kMmaWarp = kProdWarp0 + kProdWarps;
+constexpr int kThreads = 32 * (kMmaWarp + 1);
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColO = 256;
+constexpr uint32_t kColO = 0;    // O: 256 fp32 columns
+constexpr uint32_t kColS = 256;  // S: 64 fp32 columns
+constexpr uint32_t kColP = 320;  // P: 64 bf16 = 32 columns
+constexpr uint32_t kColQ = 352;  // query slice: up to 320 bf16 = 160 columns
 constexpr float kRescaleLog2 = 8.0f;
+
+static_assert(kSmem <= 232448, "shared memory budget");
+static_assert(kColQ + 160 <= kTmemCols, "tensor memory budget");
+static_assert(kStageBytes % 1024 == 0 && kXBytes % 1024 == 0, "swizzle atoms stay 1024-byte aligned");
 
 struct MlaKernelArgs {
     MlaArgs a;
@@ -64,22 +87,53 @@ __device__ __forceinline__ int64_t pool_row(const MlaArgs& a, int seq, int p) {
     return static_cast<int64_t>(pg) * kPage + (p % kPage);
 }
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
-    mla_kernel(const __grid_constant__ CUtensorMap tm_qlat, const __grid_constant__ CUtensorMap tm_qrope,
-               const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_kr,
-               const MlaKernelArgs ka) {
+__device__ __forceinline__ int idx_at(const MlaArgs& a, int r, int slot) {
+    return slot < a.k ? a.idx[static_cast<int64_t>(r) * a.k + slot] : -1;
+}
+
+template <int N>
+__device__ __forceinline__ float tree_max(float (&v)[N]) {
+#pragma unroll
+    for (int w = N / 2; w > 0; w >>= 1)
+#pragma unroll
+        for (int i = 0; i < w; ++i) v[i] = fmaxf(v[i], v[i + w]);
+    return v[0];
+}
+
+template <int N>
+__device__ __forceinline__ float tree_sum(float (&v)[N]) {
+#pragma unroll
+    for (int w = N / 2; w > 0; w >>= 1)
+#pragma unroll
+        for (int i = 0; i < w; ++i) v[i] += v[i + w];
+    return v[0];
+}
+
+// Read 64 fp32 columns of this thread's TMEM lane (two 32-column loads, one wait).
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&v)[64]) {
+    uint32_t (&v0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&v[0]);
+    uint32_t (&v1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&v[32]);
+    tmem_ld32(taddr, v0);
+    tmem_ld32(taddr + 32, v1);
+    tmem_ld_wait();
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1) mla_kernel(const MlaKernelArgs ka) {
     const MlaArgs& a = ka.a;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* sQ = sm + kOffQ;
     uint8_t* sStage = sm + kOffStage;
     uint8_t* sX = sm + kOffX;
-    uint8_t* sP = sm + kOffP;
+    uint8_t* sL = sm + kOffL;
 
-    __shared__ uint64_t bar_q, bar_full[kStages], bar_empty[kStages], bar_sfull[2], bar_sfree[2], bar_xfull[2],
-        bar_pfull[2], bar_pvdone[2], bar_final;
+    __shared__ uint64_t bar_full[kStages], bar_empty[kStages], bar_sfull, bar_sfree, bar_xfull[2], bar_xfree[2],
+        bar_pfull, bar_pvdone, bar_final;
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort;
+    __shared__ volatile int s_xfail;     // written only by exchange threads (see the exchange loop)
+    __shared__ volatile int s_pfail[4];  // written only by softmax pair q (see the softmax loop)
+    __shared__ float s_pmax[2][2][128];  // [tile parity][key half][head] tile maxima
+    __shared__ float s_psum[2][2][128];  // (l, lx) of the two key halves, for the output
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t rank = cluster_rank(), partner = rank ^ 1u;
@@ -95,118 +149,184 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
     if (tid == 0) {
         s_abort = 0;
-        mbar_init(&bar_q, 1);
+        s_xfail = 0;
+        for (int q = 0; q < 4; ++q) s_pfail[q] = 0;
         for (int i = 0; i < kStages; ++i) {
-            mbar_init(&bar_full[i], 1);
+            mbar_init(&bar_full[i], 32 * kProdWarps);
             mbar_init(&bar_empty[i], 1);
         }
+        mbar_init(&bar_sfull, 1);
+        mbar_init(&bar_sfree, kSmxWarps + 4);  // softmax and exchange warps both read S
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&bar_sfull[i], 1);
-            mbar_init(&bar_sfree[i], 4);
-            mbar_init(&bar_xfull[i], 128);
-            mbar_init(&bar_pfull[i], 4);
-            mbar_init(&bar_pvdone[i], 1);
+            mbar_init(&bar_xfull[i], 1);
+            mbar_init(&bar_xfree[i], kSmxWarps);  // the partner's softmax warps
         }
+        mbar_init(&bar_pfull, kSmxWarps);
+        mbar_init(&bar_pvdone, 1);
         mbar_init(&bar_final, 1);
         fence_mbar_init();
     }
-    if (warp == 5) {
+    if (warp == kMmaWarp) {
         tmem_alloc(&s_tmem, kTmemCols);
         tmem_relinquish();
     }
     tc_fence_before();
-    cluster_sync_all();  // partner's barriers exist before any remote arrive
+    cluster_sync_all();  // partner's barriers exist before any remote write
     tc_fence_after();
     const uint32_t tmem = s_tmem;
 
-    if (warp == 4) {
-        // ------------------------------------------------ producer: query slice + gathered rows
-        if (lane == 0) {
-            tma_prefetch_desc(&tm_c);
-            mbar_arrive_expect_tx(&bar_q, nblk * kBlkQ);
-            for (int b = 0; b < 4; ++b)
-                tma_load_3d(sQ + b * kBlkQ, &tm_qlat, &bar_q, static_cast<int>(rank) * 256 + b * 64, 0, r);
-            if (rank == 1) tma_load_3d(sQ + 4 * kBlkQ, &tm_qrope, &bar_q, 0, 0, r);
+    if (warp < 4) {
+        // The query slice of head `tid` into its TMEM lane: column c holds
+        // elements 2c, 2c+1 (rows beyond H are zero and never written out).
+        const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+        const bool live = tid < a.H;
+        const uint4* ql = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.q_lat) +
+                                                         (static_cast<int64_t>(r) * a.H + (live ? tid : 0)) * 512 +
+                                                         rank * 256);
+#pragma unroll 1
+        for (int c = 0; c < 128; c += 32) {
+            uint32_t v[32];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const uint4 u = live ? ql[c / 4 + j] : make_uint4(0u, 0u, 0u, 0u);
+                v[4 * j] = u.x;
+                v[4 * j + 1] = u.y;
+                v[4 * j + 2] = u.z;
+                v[4 * j + 3] = u.w;
+            }
+            tmem_st32(tmem + lane_base + kColQ + c, v);
+        }
+        if (rank == 1) {
+            const uint4* qr = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.q_rope) +
+                                                             (static_cast<int64_t>(r) * a.H + (live ? tid : 0)) * 64);
+            uint32_t v[32];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const uint4 u = live ? qr[j] : make_uint4(0u, 0u, 0u, 0u);
+                v[4 * j] = u.x;
+                v[4 * j + 1] = u.y;
+                v[4 * j + 2] = u.z;
+                v[4 * j + 3] = u.w;
+            }
+            tmem_st32(tmem + lane_base + kColQ + 128, v);
+        }
+        tmem_st_wait();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    if (warp >= kProdWarp0 && warp < kMmaWarp) {
+        // ------------------------------------------------ producers: gathered row slices
+        // Warp p copies keys p, p+2, ... of each tile: lane = 16-byte chunk of the
+        // 512-byte latent slice (slice b = lane / 8, chunk lane % 8); CTA 1 adds the
+        // 128-byte RoPE keys, 4 keys per instruction.  Lane i holds the pool row of
+        // the warp's i-th key (or -1 for a padded slot), for the kPrefetch tiles in
+        // flight between the L2 prefetch and the copy.
+        const int pw = warp - kProdWarp0;
+        const __nv_bfloat16* cbase = static_cast<const __nv_bfloat16*>(a.c_cache) + rank * 256 + lane * 8;
+        const __nv_bfloat16* kbase = static_cast<const __nv_bfloat16*>(a.kr_cache) + (lane & 7) * 8;
+        constexpr int kPer = kNK / kProdWarps;  // 32 keys per warp per tile
+        auto row_of = [&](int t) -> int {
+            const int p = idx_at(a, r, (t0 + t) * kNK + pw + kProdWarps * lane);
+            return p >= 0 ? static_cast<int>(pool_row(a, seq, p)) : -1;
+        };
+        auto prefetch_rows = [&](int row) {
+            if (row < 0) return;
+            const char* c = reinterpret_cast<const char*>(static_cast<const __nv_bfloat16*>(a.c_cache) +
+                                                          static_cast<int64_t>(row) * a.c_ld + rank * 256);
+#pragma unroll
+            for (int o = 0; o < 512; o += 128) prefetch_l2(c + o);
+            if (rank == 1)
+                prefetch_l2(static_cast<const __nv_bfloat16*>(a.kr_cache) + static_cast<int64_t>(row) * a.kr_ld);
+        };
+        int ring[kPrefetch];  // rows of tiles t .. t + kPrefetch - 1
+#pragma unroll
+        for (int d = 0; d < kPrefetch; ++d) {
+            ring[d] = d < nt ? row_of(d) : -1;
+            prefetch_rows(ring[d]);
         }
         int stage = 0;
         uint32_t phase = 0;
-        int64_t n_issued = 0;
         for (int t = 0; t < nt; ++t) {
             bool ok = true;
             if (lane == 0) ok = mbar_wait(&bar_empty[stage], phase ^ 1, wc, kErrMlaWait | 1);
             ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
             if (!ok) break;
-            const int slot = (t0 + t) * kNK + lane;
-            const int p = slot < a.k ? a.idx[static_cast<int64_t>(r) * a.k + slot] : -1;
-            const int row = p >= 0 ? static_cast<int>(pool_row(a, seq, p)) : 0;
-            if (lane == 0) mbar_arrive_expect_tx(&bar_full[stage], nblk * kBlkK);
-            __syncwarp();
-            const int g = lane & 7, b = lane >> 3;
-            const int y0 = __shfl_sync(0xffffffffu, row, 4 * g + 0), y1 = __shfl_sync(0xffffffffu, row, 4 * g + 1);
-            const int y2 = __shfl_sync(0xffffffffu, row, 4 * g + 2), y3 = __shfl_sync(0xffffffffu, row, 4 * g + 3);
-            uint8_t* dst = sStage + stage * (kMaxBlk * kBlkK);
-            tma_gather4(dst + b * kBlkK + g * 512, &tm_c, &bar_full[stage], static_cast<int>(rank) * 256 + b * 64, y0,
-                        y1, y2, y3);
-            if (rank == 1 && b == 0) tma_gather4(dst + 4 * kBlkK + g * 512, &tm_kr, &bar_full[stage], 0, y0, y1, y2, y3);
-            ++n_issued;
+            const int myrow = ring[0];
+            const uint32_t sbase = smem_u32(sStage + stage * kStageBytes);
+            const int b = lane >> 3, c = lane & 7;
+#pragma unroll 8
+            for (int i = 0; i < kPer; ++i) {
+                const int j = pw + kProdWarps * i;
+                const int row = __shfl_sync(0xffffffffu, myrow, i);
+                const uint32_t dst = sbase + b * kBlkK + j * 128 + ((c ^ (j & 7)) << 4);
+                cp_async16(dst, cbase + static_cast<int64_t>(row < 0 ? 0 : row) * a.c_ld, row < 0 ? 0u : 16u);
+            }
+            if (rank == 1) {
+#pragma unroll
+                for (int i0 = 0; i0 < kPer; i0 += 4) {
+                    const int i = i0 + (lane >> 3);
+                    const int j = pw + kProdWarps * i;
+                    const int row = __shfl_sync(0xffffffffu, myrow, i);
+                    const uint32_t dst = sbase + 4 * kBlkK + j * 128 + ((c ^ (j & 7)) << 4);
+                    cp_async16(dst, kbase + static_cast<int64_t>(row < 0 ? 0 : row) * a.kr_ld, row < 0 ? 0u : 16u);
+                }
+            }
+            cp_async_arrive_noinc(&bar_full[stage]);
+#pragma unroll
+            for (int d = 0; d + 1 < kPrefetch; ++d) ring[d] = ring[d + 1];
+            ring[kPrefetch - 1] = t + kPrefetch < nt ? row_of(t + kPrefetch) : -1;
+            prefetch_rows(ring[kPrefetch - 1]);
             if (++stage == kStages) {
                 stage = 0;
                 phase ^= 1;
             }
         }
-        if (lane == 0) {  // drain loads in flight
-            int dummy = 0;
-            WaitCtx dw{a.err, reinterpret_cast<volatile int*>(&dummy)};
-            mbar_wait(&bar_q, 0, dw, kErrMlaWait | 9);
-            for (int64_t i = n_issued - kStages; i < n_issued; ++i)
-                if (i >= 0) mbar_wait(&bar_full[i % kStages], static_cast<uint32_t>((i / kStages) & 1), dw, kErrMlaWait | 10);
-        }
-        __syncwarp();
-    } else if (warp == 5) {
+        cp_async_wait_all();  // every copy lands before the CTA can exit
+    } else if (warp == kMmaWarp) {
         // ------------------------------------------------ MMA issuer
         constexpr uint32_t id_qk = idesc_f32acc(1, 1, false, false, 128, kNK);
         constexpr uint32_t id_pv = idesc_f32acc(1, 1, false, true, 128, 256);
         bool ok = true;
-        if (lane == 0) ok = mbar_wait(&bar_q, 0, wc, kErrMlaWait | 2);
-        auto issue_pv = [&](int u) -> bool {
-            const int pb = u & 1;
-            if (!mbar_wait(&bar_pfull[pb], static_cast<uint32_t>((u >> 1) & 1), wc, kErrMlaWait | 3)) return false;
-            tc_fence_after();
-            const int st = u % kStages;
-            const uint64_t pd = sdesc(smem_u32(sP + pb * kPBytes), 128, 512, kSwNone);
-            const uint64_t vd = sdesc(smem_u32(sStage + st * (kMaxBlk * kBlkK)), 4096, 1024, kSw128);
-#pragma unroll
-            for (int kk = 0; kk < 2; ++kk)
-                mma_bf16_ss(tmem + kColO, pd + 16 * kk, vd + 128 * kk, id_pv, (u > 0 || kk > 0) ? 1u : 0u);
-            tc_commit(&bar_empty[st]);
-            tc_commit(&bar_pvdone[pb]);
-            return true;
-        };
-        if (lane == 0 && ok) {
+        if (lane == 0) {
             int stage = 0;
             uint32_t phase = 0;
-            for (int t = 0; t < nt && ok; ++t) {
-                ok = mbar_wait(&bar_full[stage], phase, wc, kErrMlaWait | 4);
-                const int sb = t & 1;
-                if (ok && t >= 2) ok = mbar_wait(&bar_sfree[sb], static_cast<uint32_t>(((t >> 1) - 1) & 1), wc, kErrMlaWait | 5);
-                if (!ok) break;
-                tc_fence_after();
-                uint8_t* stg = sStage + stage * (kMaxBlk * kBlkK);
-                for (int b = 0; b < nblk; ++b) {
-                    const uint64_t qd = sdesc(smem_u32(sQ + b * kBlkQ), 16, 1024, kSw128);
-                    const uint64_t kd = sdesc(smem_u32(stg + b * kBlkK), 16, 1024, kSw128);
+            for (int i = 0; i <= nt && ok; ++i) {
+                if (i < nt) {
+                    ok = mbar_wait(&bar_full[stage], phase, wc, kErrMlaWait | 4);
+                    if (ok && i >= 1) ok = mbar_wait(&bar_sfree, static_cast<uint32_t>((i - 1) & 1), wc, kErrMlaWait | 5);
+                    if (!ok) break;
+                    fence_proxy_async_smem();  // cp.async writes -> tensor-core reads
+                    tc_fence_after();
+                    uint8_t* stg = sStage + stage * kStageBytes;
+                    for (int b = 0; b < nblk; ++b) {
+                        const uint64_t kd = sdesc(smem_u32(stg + b * kBlkK), 16, 1024, kSw128);
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_bf16_ss(tmem + sb * kNK, qd + 2 * kk, kd + 2 * kk, id_qk, (b | kk) != 0 ? 1u : 0u);
+                        for (int kk = 0; kk < 4; ++kk)
+                            mma_bf16_ts(tmem + kColS, tmem + kColQ + 32 * b + 8 * kk, kd + 2 * kk, id_qk,
+                                        (b | kk) != 0 ? 1u : 0u);
+                    }
+                    tc_commit(&bar_sfull);
+                    if (++stage == kStages) {
+                        stage = 0;
+                        phase ^= 1;
+                    }
                 }
-                tc_commit(&bar_sfull[sb]);
-                if (t >= 1) ok = issue_pv(t - 1);
-                if (++stage == kStages) {
-                    stage = 0;
-                    phase ^= 1;
+                const int u = i - 1;
+                if (u >= 0) {
+                    ok = mbar_wait(&bar_pfull, static_cast<uint32_t>(u & 1), wc, kErrMlaWait | 3);
+                    if (!ok) break;
+                    tc_fence_after();
+                    const int st = u % kStages;
+                    const uint64_t vd = sdesc(smem_u32(sStage + st * kStageBytes), kBlkK, 1024, kSw128);
+#pragma unroll
+                    for (int kk = 0; kk < kNK / 16; ++kk)
+                        mma_bf16_ts(tmem + kColO, tmem + kColP + 8 * kk, vd + 128 * kk, id_pv, (u > 0 || kk > 0) ? 1u : 0u);
+                    tc_commit(&bar_empty[st]);
+                    tc_commit(&bar_pvdone);
                 }
             }
-            if (ok && nt > 0) issue_pv(nt - 1);
         }
         if (lane == 0) {
             int dummy = 0;
@@ -215,114 +335,178 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             mbar_wait(&bar_final, 0, dw, kErrMlaWait | 11);
         }
         __syncwarp();
+    } else if (warp >= kXchgWarp0) {
+        // ------------------------------------------------ exchange: this CTA's partial scores -> partner
+        // Named barrier 2 spans the 128 exchange threads.  A failed (timed-out)
+        // wait is recorded in s_xfail, which only exchange threads write, before
+        // the barrier, and every exchange thread reads it after the barrier: the
+        // four warps always leave the loop together, never one of them stuck in
+        // bar.sync.
+        const int h = tid - 32 * kXchgWarp0;
+        const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        const uint32_t x_remote = mapa_u32(smem_u32(sX), partner);
+        const uint32_t xfull_remote = mapa_u32(smem_u32(&bar_xfull[0]), partner);
+        for (int t = 0; t < nt; ++t) {
+            const int xb = t & 1;
+            uint32_t v[64];
+            const bool got = warp_wait(&bar_sfull, static_cast<uint32_t>(t & 1), wc, kErrMlaWait | 14);
+            if (got) {
+                tc_fence_after();
+                tmem_ld64(tmem + lane_base + kColS, v);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bar_sfree);
+            } else if (lane == 0) {
+                s_xfail = 1;
+            }
+            // the partner's softmax has read its buffer xb (tile t - 2); the previous copy has read L
+            if (h == 0) {
+                if (t >= 2 && !mbar_wait<true>(&bar_xfree[xb], static_cast<uint32_t>(((t >> 1) - 1) & 1), wc,
+                                               kErrMlaWait | 15))
+                    s_xfail = 1;
+                bulk_wait_read_all();
+            }
+            named_sync(2, 128);
+            if (s_xfail) break;
+            uint8_t* lrow = sL + h * 256;
+#pragma unroll
+            for (int c = 0; c < 16; ++c)
+                *reinterpret_cast<uint4*>(lrow + ((c ^ (h & 7)) << 4)) =
+                    make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+            fence_proxy_async_smem();
+            named_sync(2, 128);
+            if (h == 0) bulk_copy_to_cluster(x_remote + xb * kXBytes, sL, kXBytes, xfull_remote + 8 * xb);
+        }
+        if (h == 0) bulk_wait_all();
     } else {
-        // ------------------------------------------------ softmax + exchange + output (thread = head)
-        const int h = tid;
-        const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+        // ------------------------------------------------ softmax + output
+        // Thread = (head h = TMEM lane, key half kh).  Warps q and q + 4 form
+        // pair q and meet at named barrier 3 + q (64 threads) once per tile.  A
+        // failed wait is recorded in s_pfail[q], written only by pair q before
+        // that barrier and read by both warps after it, so the pair always
+        // leaves the loop together.
+        const int q = warp & 3, kh = warp >> 2;
+        const int h = 32 * q + lane;
+        const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
         const float c2 = a.scale * 1.4426950408889634f;  // scores in base-2 units
         float m = -INFINITY, l = 0.f, lx = 0.f;  // l: sum of bf16 P (normalises O); lx: fp32 sum (lse)
-        const uint32_t x_remote = mapa_u32(smem_u32(sX), partner);
-        const uint32_t xfull_remote0 = mapa_u32(smem_u32(&bar_xfull[0]), partner);
-        const uint32_t xfull_remote1 = mapa_u32(smem_u32(&bar_xfull[1]), partner);
+        const uint32_t xfree_remote = mapa_u32(smem_u32(&bar_xfree[0]), partner);
         bool ok = true;
+        // validity of this half's 32 slots of the next tile (slot = 32 kh + lane)
+        int i_next = nt > 0 ? idx_at(a, r, t0 * kNK + kHalf * kh + lane) : -1;
         for (int t = 0; t < nt; ++t) {
-            const int sb = t & 1;
-            if (!(ok = warp_wait(&bar_sfull[sb], static_cast<uint32_t>((t >> 1) & 1), wc, kErrMlaWait | 6))) break;
-            tc_fence_after();
-            uint32_t v[32];
-            tmem_ld32(tmem + lane_base + sb * kNK, v);
-            tmem_ld_wait();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bar_sfree[sb]);
-            // swap partial scores with the partner (row h, 8 chunks of 16 B, xor-swizzled)
-            const uint32_t xrow = x_remote + sb * kXBytes + h * 128;
+            const int xb = t & 1;
+            const unsigned vmask = __ballot_sync(0xffffffffu, i_next >= 0);
+            if (t + 1 < nt) i_next = idx_at(a, r, (t0 + t + 1) * kNK + kHalf * kh + lane);
+            if (tid == 0) mbar_arrive_expect_tx(&bar_xfull[xb], kXBytes);  // the partner's half of tile t
+            float s[kHalf];
+            bool got = warp_wait(&bar_sfull, static_cast<uint32_t>(t & 1), wc, kErrMlaWait | 6);
+            if (got) {
+                tc_fence_after();
+                uint32_t v[kHalf];
+                tmem_ld32(tmem + lane_base + kColS + kHalf * kh, v);
+                tmem_ld_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bar_sfree);
+                got = warp_wait<true>(&bar_xfull[xb], static_cast<uint32_t>((t >> 1) & 1), wc, kErrMlaWait | 7);
+                if (got) {
+                    const uint8_t* xl = sX + xb * kXBytes + h * 256;
 #pragma unroll
-            for (int c = 0; c < 8; ++c)
-                st_cluster_v4(xrow + ((c ^ (h & 7)) << 4), v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
-            mbar_arrive_cluster(sb ? xfull_remote1 : xfull_remote0);
-            if (!(ok = warp_wait<true>(&bar_xfull[sb], static_cast<uint32_t>((t >> 1) & 1), wc, kErrMlaWait | 7))) break;
-            const uint8_t* xl = sX + sb * kXBytes + h * 128;
-            float s[32];
+                    for (int c = 0; c < kHalf / 4; ++c) {
+                        const int cc = 8 * kh + c;  // 16-byte chunk of the row (4 keys)
+                        const float4 x = *reinterpret_cast<const float4*>(xl + ((cc ^ (h & 7)) << 4));
+                        const float xs[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                const float4 x = *reinterpret_cast<const float4*>(xl + ((c ^ (h & 7)) << 4));
-                s[4 * c + 0] = __uint_as_float(v[4 * c + 0]) + x.x;
-                s[4 * c + 1] = __uint_as_float(v[4 * c + 1]) + x.y;
-                s[4 * c + 2] = __uint_as_float(v[4 * c + 2]) + x.z;
-                s[4 * c + 3] = __uint_as_float(v[4 * c + 3]) + x.w;
-            }
-            const int slot = (t0 + t) * kNK + lane;
-            const bool vld = slot < a.k && a.idx[static_cast<int64_t>(r) * a.k + slot] >= 0;
-            const unsigned vmask = __ballot_sync(0xffffffffu, vld);
-            float mx = -INFINITY;
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                s[j] = ((vmask >> j) & 1u) ? s[j] * c2 : -INFINITY;
-                mx = fmaxf(mx, s[j]);
-            }
-            const bool need = mx > m + kRescaleLog2;
-            if (__any_sync(0xffffffffu, need)) {
-                const float m_new = fmaxf(m, mx);
-                const float alpha = (m == -INFINITY) ? 0.f : exp2f(m - m_new);
-                if (t > 0) {  // O holds tiles < t: wait for the last product, then scale it
-                    if (!(ok = warp_wait(&bar_pvdone[(t - 1) & 1], static_cast<uint32_t>(((t - 1) >> 1) & 1), wc,
-                                         kErrMlaWait | 8)))
-                        break;
-                    tc_fence_after();
-#pragma unroll 1
-                    for (int c = 0; c < 256; c += 32) {
-                        uint32_t o[32];
-                        tmem_ld32(tmem + lane_base + kColO + c, o);
-                        tmem_ld_wait();
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
-                        tmem_st32(tmem + lane_base + kColO + c, o);
+                        for (int e = 0; e < 4; ++e) {
+                            const int j = 4 * c + e;
+                            s[j] = ((vmask >> j) & 1u) ? (__uint_as_float(v[j]) + xs[e]) * c2 : -INFINITY;
+                        }
                     }
-                    tmem_st_wait();
-                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_cluster(xfree_remote + 8 * xb);  // the partner may refill it
+                }
+            }
+            float mx;
+            {
+                float tmp[kHalf];
+#pragma unroll
+                for (int j = 0; j < kHalf; ++j) tmp[j] = got ? s[j] : -INFINITY;
+                mx = tree_max(tmp);
+            }
+            s_pmax[t & 1][kh][h] = mx;  // by parity: the partner may still read tile t - 1
+            if (!got && lane == 0) s_pfail[q] = 1;
+            named_sync(3 + q, 64);
+            if (s_pfail[q]) {
+                ok = false;
+                break;
+            }
+            mx = fmaxf(mx, s_pmax[t & 1][kh ^ 1][h]);
+            if (__any_sync(0xffffffffu, mx > m + kRescaleLog2)) {
+                const float m_new = fmaxf(m, mx);
+                const float alpha = (m == -INFINITY) ? 0.f : fast_exp2(m - m_new);
+                if (t > 0) {  // O holds tiles < t: wait for the last product, then scale this half of it
+                    if (warp_wait(&bar_pvdone, static_cast<uint32_t>((t - 1) & 1), wc, kErrMlaWait | 8)) {
+                        tc_fence_after();
+#pragma unroll 1
+                        for (int c = 128 * kh; c < 128 * kh + 128; c += 32) {
+                            uint32_t o[32];
+                            tmem_ld32(tmem + lane_base + kColO + c, o);
+                            tmem_ld_wait();
+#pragma unroll
+                            for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+                            tmem_st32(tmem + lane_base + kColO + c, o);
+                        }
+                        tmem_st_wait();
+                    }
                 }
                 l *= alpha;
                 lx *= alpha;
                 m = m_new;
             }
-            uint32_t pk[16];
+            // masked slots are -inf and give exactly 0; a fully masked prefix keeps m at -inf
+            const float mref = (m == -INFINITY) ? 0.f : m;
+            uint32_t pk[kHalf / 2];
+            float lb[kHalf / 2], lf[kHalf / 2];
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                // masked slots contribute exactly 0 (also while m is still -inf)
-                const float p0 = ((vmask >> (2 * j)) & 1u) ? exp2f(s[2 * j] - m) : 0.f;
-                const float p1 = ((vmask >> (2 * j + 1)) & 1u) ? exp2f(s[2 * j + 1] - m) : 0.f;
+            for (int j = 0; j < kHalf / 2; ++j) {
+                const float p0 = fast_exp2(s[2 * j] - mref);
+                const float p1 = fast_exp2(s[2 * j + 1] - mref);
                 const __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
-                l += __low2float(b2) + __high2float(b2);
-                lx += p0 + p1;
+                lb[j] = __low2float(b2) + __high2float(b2);
+                lf[j] = p0 + p1;
                 pk[j] = *reinterpret_cast<const uint32_t*>(&b2);
             }
-            const int pb = t & 1;
-            if (t >= 2 &&
-                !(ok = warp_wait(&bar_pvdone[pb], static_cast<uint32_t>(((t >> 1) - 1) & 1), wc, kErrMlaWait | 12)))
-                break;
-            uint8_t* prow = sP + pb * kPBytes + (h >> 3) * 512 + (h & 7) * 16;
-#pragma unroll
-            for (int c = 0; c < 4; ++c)
-                *reinterpret_cast<uint4*>(prow + c * 128) = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-            fence_proxy_async_smem();
+            l += tree_sum(lb);
+            lx += tree_sum(lf);
+            // the product of tile t - 1 has read P before it is overwritten
+            if (t >= 1) warp_wait(&bar_pvdone, static_cast<uint32_t>((t - 1) & 1), wc, kErrMlaWait | 12);
+            tc_fence_after();
+            tmem_st16(tmem + lane_base + kColP + (kHalf / 2) * kh, pk);
+            tmem_st_wait();
+            tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bar_pfull[pb]);
+            if (lane == 0) mbar_arrive(&bar_pfull);
         }
-        // ---- output: this CTA's 256 latent dims of every head
+        // ---- output: this thread's half (128 latent dims) of the CTA's 256 dims of head h
+        s_psum[kh][0][h] = l;
+        s_psum[kh][1][h] = lx;
+        named_sync(3 + q, 64);
+        const float lt = s_psum[0][0][h] + s_psum[1][0][h];
+        const float lxt = s_psum[0][1][h] + s_psum[1][1][h];
         if (ok && nt > 0)
-            ok = warp_wait(&bar_pvdone[(nt - 1) & 1], static_cast<uint32_t>(((nt - 1) >> 1) & 1), wc, kErrMlaWait | 13);
-        if (ok) {
+            ok = warp_wait(&bar_pvdone, static_cast<uint32_t>((nt - 1) & 1), wc, kErrMlaWait | 13);
+        if (ok && !s_abort) {
             tc_fence_after();
             const bool partial = ka.nsplit > 1;
-            const float inv = (l > 0.f && !partial) ? 1.f / l : 1.f;
+            const float inv = (lt > 0.f && !partial) ? 1.f / lt : 1.f;
             float* dst;
             if (partial)
                 dst = ka.ws_o + ((static_cast<int64_t>(r) * ka.nsplit + split) * a.H + h) * 512 + rank * 256;
             else
                 dst = a.out + (static_cast<int64_t>(r) * a.H + h) * a.d_c + rank * 256;
 #pragma unroll 1
-            for (int c = 0; c < 256; c += 32) {
+            for (int c = 128 * kh; c < 128 * kh + 128; c += 32) {
                 uint32_t o[32];
                 if (nt > 0) {
                     tmem_ld32(tmem + lane_base + kColO + c, o);
@@ -332,7 +516,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     for (int j = 0; j < 32; ++j) o[j] = 0u;
                 }
                 if (h < a.H) {
-                    const bool empty = !(l > 0.f);
+                    const bool empty = !(lt > 0.f);
 #pragma unroll
                     for (int j = 0; j < 32; j += 4) {
                         float4 f;
@@ -344,14 +528,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     }
                 }
             }
-            if (h < a.H && rank == 0) {
+            if (h < a.H && rank == 0 && kh == 0) {
                 if (partial) {
                     float* ml = ka.ws_ml + ((static_cast<int64_t>(r) * ka.nsplit + split) * a.H + h) * 4;
                     ml[0] = m;
-                    ml[1] = l;
-                    ml[2] = lx;
+                    ml[1] = lt;
+                    ml[2] = lxt;
                 } else if (a.lse) {
-                    a.lse[static_cast<int64_t>(r) * a.H + h] = l > 0.f ? (m + log2f(lx)) * 0.6931471805599453f : -INFINITY;
+                    a.lse[static_cast<int64_t>(r) * a.H + h] = lt > 0.f ? (m + log2f(lxt)) * 0.6931471805599453f : -INFINITY;
                 }
             }
         }
@@ -361,7 +545,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     __syncthreads();
     cluster_sync_all();  // the partner no longer writes into this CTA's shared memory
     tc_fence_after();
-    if (warp == 5) tmem_dealloc(tmem, kTmemCols);
+    if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
 }
 
 // Merge the split partial states of every (row, head).
@@ -429,39 +613,9 @@ sa_status sparse_mla_launch(const MlaArgs& a, int nsplit, void* ws, size_t ws_by
         ka.ws_o = static_cast<float*>(ws);
         ka.ws_ml = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + ((o + 255) & ~size_t(255)));
     }
-    const uint64_t pool_rows = static_cast<uint64_t>(a.pool_pages) * kPage;
-    CUtensorMap tq, tqr, tc, tkr;
-    {
-        const uint64_t dims[3] = {512, static_cast<uint64_t>(a.H), static_cast<uint64_t>(a.rows)};
-        const uint64_t str[2] = {512 * 2, static_cast<uint64_t>(a.H) * 512 * 2};
-        const uint32_t box[3] = {64, 128, 1};
-        if (!encode_tiled(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, a.q_lat, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
-            return SA_ECUDA;
-    }
-    {
-        const uint64_t dims[3] = {64, static_cast<uint64_t>(a.H), static_cast<uint64_t>(a.rows)};
-        const uint64_t str[2] = {64 * 2, static_cast<uint64_t>(a.H) * 64 * 2};
-        const uint32_t box[3] = {64, 128, 1};
-        if (!encode_tiled(&tqr, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, a.q_rope, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
-            return SA_ECUDA;
-    }
-    {
-        const uint64_t dims[2] = {512, pool_rows};
-        const uint64_t str[1] = {static_cast<uint64_t>(a.c_ld) * 2};
-        const uint32_t box[2] = {64, 1};
-        if (!encode_tiled(&tc, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.c_cache, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
-            return SA_ECUDA;
-    }
-    {
-        const uint64_t dims[2] = {64, pool_rows};
-        const uint64_t str[1] = {static_cast<uint64_t>(a.kr_ld) * 2};
-        const uint32_t box[2] = {64, 1};
-        if (!encode_tiled(&tkr, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.kr_cache, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
-            return SA_ECUDA;
-    }
     cudaError_t e = cudaFuncSetAttribute(mla_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
     if (e != cudaSuccess) return launch_status(e);
-    mla_kernel<<<2 * a.rows * nsplit, kThreads, kSmem, st>>>(tq, tqr, tc, tkr, ka);
+    mla_kernel<<<2 * a.rows * nsplit, kThreads, kSmem, st>>>(ka);
     e = cudaGetLastError();
     if (e != cudaSuccess) return launch_status(e);
     if (nsplit > 1) {
