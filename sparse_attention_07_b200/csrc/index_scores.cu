@@ -13,7 +13,9 @@
 // fp32 score per row.  A persistent CTA per SM walks a balanced contiguous
 // range of (row group, key tile) items; a TMA producer warp streams 16 KB key
 // tiles (two 64-token pages) through a 6-stage ring, an MMA warp issues, and
-// 4 or 8 epilogue warps drain a double-buffered accumulator.
+// 4 or 8 epilogue warps drain a ring of 2 or 4 TMEM accumulators.  The producer
+// looks up 32 items at a time (one per lane), so its issue loop holds no
+// dependent global loads.
 //
 // CUDA-core path (fp32 or fp8, d_I <= 128, H_I <= 64): one thread per key.
 #include <cuda_fp8.h>
@@ -128,7 +130,9 @@ struct ItemWalk {
 template <int NH, int R, int NEPI>
 struct TcCfg {
     static constexpr int N = R * NH;                     // MMA N (rows x heads)
-    static constexpr int kTmemCols = (2 * N <= 32) ? 32 : (2 * N <= 64 ? 64 : (2 * N <= 128 ? 128 : (2 * N <= 256 ? 256 : 512)));
+    // accumulator buffers: four where they fit in TMEM (the MMA runs further ahead of the epilogue)
+    static constexpr int kAcc = (4 * N <= 512) ? 4 : 2;
+    static constexpr int kTmemCols = (kAcc * N <= 32) ? 32 : (kAcc * N <= 64 ? 64 : (kAcc * N <= 128 ? 128 : (kAcc * N <= 256 ? 256 : 512)));
     static constexpr int kQBytes = N * 128;
     static constexpr int kThreads = 32 * (NEPI + 2);
     // shared layout (offsets from a 1024-aligned base)
@@ -137,7 +141,8 @@ struct TcCfg {
     static constexpr int kOffW = kOffQ + 2 * kQBytes;
     static constexpr int kOffPrefix = kOffW + NEPI * R * NH * 4;
     static constexpr int kOffGStart = kOffPrefix + (kMaxRows + 1) * 4;
-    static constexpr int kSmemBytes = kOffGStart + (kMaxRows + 1) * 4 + 1024;
+    static constexpr int kOffGnk = kOffGStart + (kMaxRows + 1) * 4;
+    static constexpr int kSmemBytes = kOffGnk + (kMaxRows + 1) * 4 + 1024;
 };
 
 template <int NH, int R, int NEPI>
@@ -153,9 +158,10 @@ __global__ void __launch_bounds__(TcCfg<NH, R, NEPI>::kThreads, 1)
     float* s_w = reinterpret_cast<float*>(sm + C::kOffW);
     int* s_prefix = reinterpret_cast<int*>(sm + C::kOffPrefix);
     int* s_gstart = reinterpret_cast<int*>(sm + C::kOffGStart);
+    int* s_gnk = reinterpret_cast<int*>(sm + C::kOffGnk);  // longest visible length in the group
 
-    __shared__ uint64_t bar_full[kStages], bar_empty[kStages], bar_qfull[2], bar_qempty[2], bar_accfull[2],
-        bar_accempty[2], bar_final;
+    __shared__ uint64_t bar_full[kStages], bar_empty[kStages], bar_qfull[2], bar_qempty[2], bar_accfull[C::kAcc],
+        bar_accempty[C::kAcc], bar_final;
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort;
     __shared__ int s_warpbuf[40];
@@ -173,6 +179,8 @@ __global__ void __launch_bounds__(TcCfg<NH, R, NEPI>::kThreads, 1)
         for (int i = 0; i < 2; ++i) {
             mbar_init(&bar_qfull[i], 1);
             mbar_init(&bar_qempty[i], 1);
+        }
+        for (int i = 0; i < C::kAcc; ++i) {
             mbar_init(&bar_accfull[i], 1);
             mbar_init(&bar_accempty[i], NEPI);
         }
@@ -214,6 +222,7 @@ __global__ void __launch_bounds__(TcCfg<NH, R, NEPI>::kThreads, 1)
     for (int g = tid; g < G; g += blockDim.x) {
         int nk = 0;
         for (int r = s_gstart[g]; r < s_gstart[g + 1]; ++r) nk = max(nk, clamp_vis(a, r));
+        s_gnk[g] = nk;
         s_prefix[g] = (nk + kTileKeys - 1) / kTileKeys;
     }
     __syncthreads();
@@ -235,40 +244,56 @@ __global__ void __launch_bounds__(TcCfg<NH, R, NEPI>::kThreads, 1)
 
     if (warp == NEPI) {
         // ------------------------------------------------ TMA producer
+        // The warp describes the next 32 items at once (lane i: item + i: its
+        // group, key tile and the physical pages of the tile's two 64-key pages),
+        // so lane 0's issue loop holds no dependent global loads.
         int stage = 0;
         uint32_t phase = 0;
         int gcount = -1, prev_g = -1;
         int64_t n_issued = 0;
-        if (begin < end) {
-            for (it.start(static_cast<int>(begin), static_cast<int>(end)); it.valid(); it.next()) {
-                const int g = it.g, t = it.t;
-                const int r0 = s_gstart[g];
-                bool ok = true;
-                if (g != prev_g) {
-                    ++gcount;
-                    prev_g = g;
-                    const int qb = gcount & 1;
-                    if (gcount >= 2 && lane == 0) ok = mbar_wait(&bar_qempty[qb], ((gcount >> 1) - 1) & 1, wc, kErrIdxWait | 1);
-                    if (ok && lane == 0) {
-                        mbar_arrive_expect_tx(&bar_qfull[qb], C::kQBytes);
-                        tma_load_2d(s_q + qb * C::kQBytes, &tm_q, &bar_qfull[qb], 0, r0 * NH);
+        bool ok = true;
+        for (int item = static_cast<int>(begin); ok && item < static_cast<int>(end); item += 32) {
+            const int my_item = item + lane;
+            int my_g = 0, my_p0 = 0, my_p1 = -1;
+            if (my_item < end) {
+                int lo = 0, hi = G;  // largest g with prefix[g] <= my_item (a non-empty group)
+                while (hi - lo > 1) {
+                    const int mid = (lo + hi) >> 1;
+                    if (s_prefix[mid] <= my_item) lo = mid; else hi = mid;
+                }
+                my_g = lo;
+                const int t = my_item - s_prefix[lo];
+                const int seq = seq_of(a, s_gstart[lo]);
+                my_p0 = page_of(a, seq, 2 * t);
+                if ((2 * t + 1) * kPage < s_gnk[lo]) my_p1 = page_of(a, seq, 2 * t + 1);
+            }
+            const int n = min(32, static_cast<int>(end) - item);
+            for (int i = 0; i < n; ++i) {
+                const int g = __shfl_sync(0xffffffffu, my_g, i);
+                const int p0 = __shfl_sync(0xffffffffu, my_p0, i);
+                const int p1 = __shfl_sync(0xffffffffu, my_p1, i);
+                if (lane == 0) {
+                    if (g != prev_g) {
+                        ++gcount;
+                        prev_g = g;
+                        const int qb = gcount & 1;
+                        if (gcount >= 2) ok = mbar_wait(&bar_qempty[qb], ((gcount >> 1) - 1) & 1, wc, kErrIdxWait | 1);
+                        if (ok) {
+                            mbar_arrive_expect_tx(&bar_qfull[qb], C::kQBytes);
+                            tma_load_2d(s_q + qb * C::kQBytes, &tm_q, &bar_qfull[qb], 0, s_gstart[g] * NH);
+                        }
+                    }
+                    if (ok) ok = mbar_wait(&bar_empty[stage], phase ^ 1, wc, kErrIdxWait | 2);
+                    if (ok) {
+                        mbar_arrive_expect_tx(&bar_full[stage], (p1 >= 0 ? 2 : 1) * (kStageBytes / 2));
+                        uint8_t* dst = s_stage + stage * kStageBytes;
+                        tma_load_2d(dst, &tm_k, &bar_full[stage], 0, p0 * kPage);
+                        if (p1 >= 0) tma_load_2d(dst + kStageBytes / 2, &tm_k, &bar_full[stage], 0, p1 * kPage);
+                        ++n_issued;
                     }
                 }
-                if (ok && lane == 0) ok = mbar_wait(&bar_empty[stage], phase ^ 1, wc, kErrIdxWait | 2);
-                if (ok && lane == 0) {
-                    const int seq = seq_of(a, r0);
-                    int nk = 0;
-                    for (int r = r0; r < s_gstart[g + 1]; ++r) nk = max(nk, clamp_vis(a, r));
-                    const int p0 = 2 * t, p1 = 2 * t + 1;
-                    const bool v1 = p1 * kPage < nk;
-                    mbar_arrive_expect_tx(&bar_full[stage], (v1 ? 2 : 1) * (kStageBytes / 2));
-                    uint8_t* dst = s_stage + stage * kStageBytes;
-                    tma_load_2d(dst, &tm_k, &bar_full[stage], 0, page_of(a, seq, p0) * kPage);
-                    if (v1) tma_load_2d(dst + kStageBytes / 2, &tm_k, &bar_full[stage], 0, page_of(a, seq, p1) * kPage);
-                    ++n_issued;
-                }
-                __syncwarp();
-                if (s_abort) break;
+                ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+                if (!ok) break;
                 if (++stage == kStages) {
                     stage = 0;
                     phase ^= 1;
@@ -301,10 +326,10 @@ __global__ void __launch_bounds__(TcCfg<NH, R, NEPI>::kThreads, 1)
                     prev_g = it.g;
                     if (lane == 0) ok = mbar_wait(&bar_qfull[gcount & 1], (gcount >> 1) & 1, wc, kErrIdxWait | 3);
                 }
-                const int buf = static_cast<int>(acc & 1);
+                const int buf = static_cast<int>(acc % C::kAcc);
                 if (ok && lane == 0) ok = mbar_wait(&bar_full[stage], phase, wc, kErrIdxWait | 4);
-                if (ok && lane == 0 && acc >= 2)
-                    ok = mbar_wait(&bar_accempty[buf], static_cast<uint32_t>(((acc >> 1) - 1) & 1), wc, kErrIdxWait | 5);
+                if (ok && lane == 0 && acc >= C::kAcc)
+                    ok = mbar_wait(&bar_accempty[buf], static_cast<uint32_t>((acc / C::kAcc - 1) & 1), wc, kErrIdxWait | 5);
                 if (ok && lane == 0) {
                     tc_fence_after();
                     const uint64_t da = sdesc(smem_u32(s_stage + stage * kStageBytes), 16, 1024, kSw128);
@@ -341,6 +366,7 @@ __global__ void __launch_bounds__(TcCfg<NH, R, NEPI>::kThreads, 1)
         int prev_g = -1;
         int g_r0 = 0, g_cnt = 0;
         int nvis[kRowsPerHalf];
+        float wr[R == 1 ? NH : 1];  // one-row groups: the row's weights
         float* w_own = s_w + warp * R * NH;  // this warp's copy of the group's weights
         if (begin < end) {
             for (it.start(static_cast<int>(begin), static_cast<int>(end)); it.valid(); it.next()) {
@@ -348,6 +374,10 @@ __global__ void __launch_bounds__(TcCfg<NH, R, NEPI>::kThreads, 1)
                     prev_g = it.g;
                     g_r0 = s_gstart[it.g];
                     g_cnt = s_gstart[it.g + 1] - g_r0;
+                    if constexpr (R == 1) {
+#pragma unroll
+                        for (int x = 0; x < NH; ++x) wr[x] = a.w[static_cast<int64_t>(g_r0) * NH + x];
+                    }
                     __syncwarp();
                     for (int i = lane; i < R * NH; i += 32) {
                         const int gi = i / NH;
@@ -360,10 +390,42 @@ __global__ void __launch_bounds__(TcCfg<NH, R, NEPI>::kThreads, 1)
                         nvis[j] = gi < g_cnt ? clamp_vis(a, g_r0 + gi) : 0;
                     }
                 }
-                const int buf = static_cast<int>(acc & 1);
-                if (!warp_wait(&bar_accfull[buf], static_cast<uint32_t>((acc >> 1) & 1), wc, kErrIdxWait | 6)) break;
+                const int buf = static_cast<int>(acc % C::kAcc);
+                if (!warp_wait(&bar_accfull[buf], static_cast<uint32_t>((acc / C::kAcc) & 1), wc, kErrIdxWait | 6)) break;
                 tc_fence_after();
                 const int s = it.t * kTileKeys + quarter * 32 + lane;
+                if constexpr (R == 1) {
+                    // one row per group: its weights sit in registers; four independent
+                    // accumulators (on integer inputs every partial sum is exact, so the
+                    // order of the additions does not change the result)
+                    float acc4[4] = {0.f, 0.f, 0.f, 0.f};
+                    const uint32_t col = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + buf * N;
+                    if constexpr (NH == 16) {
+                        uint32_t v[16];
+                        tmem_ld16(col, v);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int x = 0; x < 16; ++x) acc4[x & 3] = fmaf(wr[x], fmaxf(__uint_as_float(v[x]), 0.f), acc4[x & 3]);
+                    } else {
+#pragma unroll
+                        for (int c = 0; c < NH; c += 64) {
+                            uint32_t v0[32], v1[32];
+                            tmem_ld32(col + c, v0);
+                            if (c + 32 < NH) tmem_ld32(col + c + 32, v1);
+                            tmem_ld_wait();
+#pragma unroll
+                            for (int x = 0; x < 32; ++x)
+                                acc4[x & 3] = fmaf(wr[c + x], fmaxf(__uint_as_float(v0[x]), 0.f), acc4[x & 3]);
+                            if (c + 32 < NH) {
+#pragma unroll
+                                for (int x = 0; x < 32; ++x)
+                                    acc4[x & 3] = fmaf(wr[c + 32 + x], fmaxf(__uint_as_float(v1[x]), 0.f), acc4[x & 3]);
+                            }
+                        }
+                    }
+                    if (s < nvis[0] && g_cnt > 0)
+                        a.scores[static_cast<int64_t>(g_r0) * a.scores_ld + s] = (acc4[0] + acc4[1]) + (acc4[2] + acc4[3]);
+                } else {
 #pragma unroll
                 for (int j = 0; j < kRowsPerHalf; ++j) {
                     const int gi = half * kRowsPerHalf + j;
@@ -389,6 +451,7 @@ __global__ void __launch_bounds__(TcCfg<NH, R, NEPI>::kThreads, 1)
                         }
                         if (s < nvis[j]) a.scores[static_cast<int64_t>(g_r0 + gi) * a.scores_ld + s] = sum;
                     }
+                }
                 }
                 tc_fence_before();
                 __syncwarp();
