@@ -172,9 +172,12 @@ class DecodeStep:
         self.out = torch.empty(cfg.rows, cfg.H, cfg.d_c, dtype=torch.float32, device=dev)
         self.lse = torch.empty(cfg.rows, cfg.H, dtype=torch.float32, device=dev)
         self.prefill = cfg.prefill_start >= 0
-        ws = 0 if self.prefill else sa.sparse_mla_workspace_size(cfg.rows, cfg.H, cfg.topk, cfg.d_c)
-        self.ws = torch.empty(max(ws, 256), dtype=torch.uint8, device=dev) if ws else None
-        self.launches_per_step = 3 + (1 if ws else 0)
+        size = sa.sparse_mla_prefill_workspace_size if self.prefill else sa.sparse_mla_workspace_size
+        self.ws = torch.empty(size(cfg.rows, cfg.H, cfg.topk, cfg.d_c), dtype=torch.uint8, device=dev)
+        # decode splits keys (and adds the combine launch) when its workspace holds partial states
+        combine = not self.prefill and (sa.sparse_mla_workspace_size(cfg.rows, cfg.H, cfg.topk, cfg.d_c) >
+                                        sa.sparse_mla_prefill_workspace_size(cfg.rows, cfg.H, cfg.topk, cfg.d_c))
+        self.launches_per_step = 3 + (1 if combine else 0)
 
     def indexer(self):
         i, c = self.inp, self.cfg
@@ -187,7 +190,7 @@ class DecodeStep:
         if self.prefill:
             self.sa.sparse_mla_prefill(i["q_lat"], i["q_rope"], i["c_cache"], i["kr_cache"], self.idx, c.scale,
                                        c.pages_per_seq, page_table=i["page_table"], seq_of_row=i["seq_of_row"],
-                                       out=self.out, lse=self.lse)
+                                       out=self.out, lse=self.lse, workspace=self.ws)
         else:
             self.sa.sparse_mla_decode(i["q_lat"], i["q_rope"], i["c_cache"], i["kr_cache"], self.idx, c.scale,
                                       c.pages_per_seq, page_table=i["page_table"], seq_of_row=i["seq_of_row"],

@@ -143,12 +143,19 @@ sa_status sa_topk_select(const float* scores, int64_t scores_ld, const int32_t* 
  * Supported: d_c = 512, d_R = 64, 1 <= H <= 128; bf16 inputs, fp32 softmax
  * and accumulation on the tensor cores.  Alignment: every base pointer and
  * row stride a multiple of 16 bytes.
- * _decode splits each row's k positions over several CTAs when rows are few
- * and combines the partial softmax states in `workspace`
- * (sa_sparse_mla_workspace_size bytes, 256-byte aligned; may be NULL when the
- * size is 0).  _prefill keeps one row per CTA pair and needs no workspace.
+ * Both calls need a caller workspace (256-byte aligned, contents need no
+ * initialisation and are scratch after the call): the two CTAs that share a
+ * row exchange their partial scores through it (an L2-resident area of
+ * sa_sparse_mla_prefill_workspace_size bytes, one slot per SM), and _decode,
+ * which splits each row's k positions over several CTA pairs when rows are
+ * few, also keeps the partial softmax states there
+ * (sa_sparse_mla_workspace_size bytes in all).  A smaller or missing
+ * workspace returns SA_EINVAL.  _prefill keeps one row per CTA pair and
+ * supports k <= 4096; _decode splits larger k.  Concurrent calls (different
+ * streams) need separate workspaces.
  */
 size_t sa_sparse_mla_workspace_size(int rows, int H, int k, int d_c);
+size_t sa_sparse_mla_prefill_workspace_size(int rows, int H, int k, int d_c);
 
 sa_status sa_sparse_mla_decode(const void* q_lat, const void* q_rope,
                                const void* c_cache, int64_t c_ld, const void* kr_cache, int64_t kr_ld,
@@ -163,7 +170,8 @@ sa_status sa_sparse_mla_prefill(const void* q_lat, const void* q_rope,
                                 int64_t pool_pages, const int32_t* page_table, int pages_per_seq,
                                 const int32_t* seq_of_row,
                                 const int32_t* idx, int rows, int H, int k, int d_c, int d_R, float scale,
-                                float* out, float* lse, sa_stream_t stream);
+                                float* out, float* lse, void* workspace, size_t workspace_bytes,
+                                sa_stream_t stream);
 
 /*
  * Sparse MLA decode for callers that cannot allocate device memory.  The
@@ -174,8 +182,9 @@ sa_status sa_sparse_mla_prefill(const void* q_lat, const void* q_rope,
  * or a custom memory manager that owns every byte of the GPU, plugins of a
  * framework that only passes tensors in and out).  This call computes exactly
  * what sa_sparse_mla_decode computes, with the same arguments minus the
- * workspace, and keeps the split-key partial states in a static device array
- * of SA_STATIC_SCRATCH_BYTES that the library owns.  It calls no cudaMalloc,
+ * workspace, and keeps its scratch (the partial-score exchange area and the
+ * split-key partial states) in a static device array of
+ * SA_STATIC_SCRATCH_BYTES that the library owns.  It calls no cudaMalloc,
  * cudaFree or allocating library routine.
  *
  *  - Every GPU that loads the library holds that array until the process exits.
@@ -192,7 +201,7 @@ sa_status sa_sparse_mla_prefill(const void* q_lat, const void* q_rope,
  *    byte a call reads from the array was written earlier in the same call,
  *    so nothing left by a previous call leaks into a result.
  */
-#define SA_STATIC_SCRATCH_BYTES ((size_t)16 << 20)
+#define SA_STATIC_SCRATCH_BYTES ((size_t)40 << 20)
 
 sa_status sa_sparse_mla_decode_static(const void* q_lat, const void* q_rope,
                                       const void* c_cache, int64_t c_ld, const void* kr_cache, int64_t kr_ld,

@@ -25,13 +25,14 @@ SA_F32, SA_E4M3, SA_BF16 = range(3)
 
 EXPORTS = (
     "sa_status_string", "sa_version", "sa_check_device_error", "sa_index_scores", "sa_topk_select",
-    "sa_sparse_mla_workspace_size", "sa_sparse_mla_decode", "sa_sparse_mla_prefill",
+    "sa_sparse_mla_workspace_size", "sa_sparse_mla_prefill_workspace_size", "sa_sparse_mla_decode",
+    "sa_sparse_mla_prefill",
     "sa_block_mean_pool", "sa_block_sparse_attn", "sa_sparse_mla_decode_static",
 )
 
 # Size of the library's static device array behind sparse_mla_decode_static
 # (SA_STATIC_SCRATCH_BYTES in include/sparse_attn.h).
-STATIC_SCRATCH_BYTES = 16 << 20
+STATIC_SCRATCH_BYTES = 40 << 20
 
 
 class SparseAttnError(RuntimeError):
@@ -58,12 +59,15 @@ def lib():
         L.sa_sparse_mla_workspace_size.restype = SZ
         L.sa_sparse_mla_workspace_size.argtypes = [I, I, I, I]
         L.sa_sparse_mla_decode.argtypes = [P, P, P, I64, P, I64, I64, P, I, P, P, I, I, I, I, I, F, P, P, P, SZ, P]
-        L.sa_sparse_mla_prefill.argtypes = [P, P, P, I64, P, I64, I64, P, I, P, P, I, I, I, I, I, F, P, P, P]
+        L.sa_sparse_mla_prefill_workspace_size.restype = SZ
+        L.sa_sparse_mla_prefill_workspace_size.argtypes = [I, I, I, I]
+        L.sa_sparse_mla_prefill.argtypes = [P, P, P, I64, P, I64, I64, P, I, P, P, I, I, I, I, I, F, P, P, P, SZ, P]
         L.sa_sparse_mla_decode_static.argtypes = [P, P, P, I64, P, I64, I64, P, I, P, P, I, I, I, I, I, F, P, P, P]
         L.sa_block_mean_pool.argtypes = [P, I64, I64, I64, I, I, I, I, I, P, I64, P]
         L.sa_block_sparse_attn.argtypes = [P, P, I64, P, P, I64, I64, I64, I, I, I, I, I, I, I, I, F, P, P, P]
         for name in EXPORTS:
-            if name not in ("sa_status_string", "sa_version", "sa_sparse_mla_workspace_size"):
+            if name not in ("sa_status_string", "sa_version", "sa_sparse_mla_workspace_size",
+                            "sa_sparse_mla_prefill_workspace_size"):
                 getattr(L, name).restype = I
         _lib = L
     return _lib
@@ -154,12 +158,21 @@ def sparse_mla_decode(q_lat, q_rope, c_cache, kr_cache, idx, scale: float, pages
     return out
 
 
+def sparse_mla_prefill_workspace_size(rows: int, H: int, k: int, d_c: int = 512) -> int:
+    return int(lib().sa_sparse_mla_prefill_workspace_size(rows, H, k, d_c))
+
+
 def sparse_mla_prefill(q_lat, q_rope, c_cache, kr_cache, idx, scale: float, pages_per_seq: int, page_table=None,
-                       seq_of_row=None, out=None, lse=None):
+                       seq_of_row=None, out=None, lse=None, workspace=None):
     rows, H, d_c, d_R, k, out, lse, pool_pages = _mla_args(q_lat, q_rope, c_cache, kr_cache, idx, out, lse)
+    if workspace is None and rows > 0:
+        workspace = torch.empty(sparse_mla_prefill_workspace_size(rows, H, k, d_c), dtype=torch.uint8,
+                                device=q_lat.device)
+    wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     st = lib().sa_sparse_mla_prefill(_p(q_lat), _p(q_rope), _p(c_cache), c_cache.stride(0), _p(kr_cache),
                                      kr_cache.stride(0), pool_pages, _p(page_table), pages_per_seq, _p(seq_of_row),
-                                     _p(idx), rows, H, k, d_c, d_R, float(scale), _p(out), _p(lse), _stream())
+                                     _p(idx), rows, H, k, d_c, d_R, float(scale), _p(out), _p(lse), _p(workspace),
+                                     wbytes, _stream())
     _check("sa_sparse_mla_prefill", st)
     return out
 

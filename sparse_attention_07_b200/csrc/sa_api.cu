@@ -210,22 +210,30 @@ sa_status sa_sparse_mla_decode(const void* q_lat, const void* q_rope, const void
                              seq_of_row, idx, rows, H, k, d_c, d_R, scale, out, lse, &a);
     if (s != SA_OK) return s;
     const int ns = mla_decode_splits(rows, k);
-    if (ns > 1 && (!workspace || !aligned(workspace, 256) ||
-                   workspace_bytes < mla_workspace_bytes(rows, H, k, d_c, ns)))
+    if (!workspace || !aligned(workspace, 256) || workspace_bytes < mla_workspace_bytes(rows, H, k, d_c, ns))
         return SA_EINVAL;
     return sparse_mla_launch(a, ns, workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t sa_sparse_mla_prefill_workspace_size(int rows, int H, int k, int d_c) {
+    if (rows < 1 || H < 1 || k < 1 || d_c < 1) return 0;
+    return mla_workspace_bytes(rows, H, k, d_c, 1);
 }
 
 sa_status sa_sparse_mla_prefill(const void* q_lat, const void* q_rope, const void* c_cache, int64_t c_ld,
                                 const void* kr_cache, int64_t kr_ld, int64_t pool_pages, const int32_t* page_table,
                                 int pages_per_seq, const int32_t* seq_of_row, const int32_t* idx, int rows, int H,
-                                int k, int d_c, int d_R, float scale, float* out, float* lse, sa_stream_t stream) {
+                                int k, int d_c, int d_R, float scale, float* out, float* lse, void* workspace,
+                                size_t workspace_bytes, sa_stream_t stream) {
     if (rows == 0) return SA_OK;
     MlaArgs a;
     sa_status s = mla_common(q_lat, q_rope, c_cache, c_ld, kr_cache, kr_ld, pool_pages, page_table, pages_per_seq,
                              seq_of_row, idx, rows, H, k, d_c, d_R, scale, out, lse, &a);
     if (s != SA_OK) return s;
-    return sparse_mla_launch(a, 1, nullptr, 0, reinterpret_cast<cudaStream_t>(stream));
+    if (k > 64 * kMaxTilesPerCta) return SA_EUNSUPPORTED;
+    if (!workspace || !aligned(workspace, 256) || workspace_bytes < mla_workspace_bytes(rows, H, k, d_c, 1))
+        return SA_EINVAL;
+    return sparse_mla_launch(a, 1, workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"
@@ -270,8 +278,8 @@ sa_status sa_sparse_mla_decode_static(const void* q_lat, const void* q_rope, con
     const int ns = mla_decode_splits(rows, k);
     const size_t need = mla_workspace_bytes(rows, H, k, d_c, ns);
     if (need > SA_STATIC_SCRATCH_BYTES) return SA_EUNSUPPORTED;  // checked before any CUDA call
-    void* ws = nullptr;
-    if (need > 0 && (ws = static_scratch()) == nullptr) return SA_ECUDA;
+    void* ws = static_scratch();
+    if (ws == nullptr) return SA_ECUDA;
     return sparse_mla_launch(a, ns, ws, SA_STATIC_SCRATCH_BYTES, reinterpret_cast<cudaStream_t>(stream));
 }
 

@@ -59,6 +59,15 @@ struct MlaArgs {
     int* err;
 };
 
+// Sparse MLA: the two CTAs of a pair exchange partial scores through an
+// L2-resident scratch area with one slot per SM (a CTA uses the slot of the SM
+// it runs on; one CTA fits on an SM), kMlaXBuf tiles of kMlaXBytes per slot.
+constexpr int kMlaXBuf = 4;
+constexpr int kMlaXBytes = 128 * 64 * 4;
+constexpr int kMlaScratchSlots = 160;
+constexpr int kMaxTilesPerCta = 64;  // 64-key tiles per CTA (the row table in shared memory)
+
+size_t mla_exchange_bytes();
 size_t mla_workspace_bytes(int rows, int H, int k, int d_c, int nsplit);
 int mla_decode_splits(int rows, int k);
 sa_status sparse_mla_launch(const MlaArgs& a, int nsplit, void* ws, size_t ws_bytes, cudaStream_t st);

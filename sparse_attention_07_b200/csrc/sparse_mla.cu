@@ -9,31 +9,33 @@
 //
 // Design (one cluster of two CTAs per (row, key split)):
 //  * The 576-wide score contraction is split across the pair: CTA 0 owns latent
-//    dims 0..255, CTA 1 owns dims 256..511 plus the 64 RoPE dims.  Two
-//    producer warps gather only the CTA's slice of every selected row with
+//    dims 0..255, CTA 1 owns dims 256..511 plus the 64 RoPE dims, and each CTA
+//    aggregates its own 256 latent dims of the output, so every selected row is
+//    read from memory once.
+//  * Prologue: the pool rows of all of the CTA's selected slots go into a table
+//    in shared memory (-1 for padded slots); the gather loop then does no
+//    dependent global loads.
+//  * Six producer warps gather the CTA's slice of every selected row with
 //    16-byte cp.async (one warp instruction per 512-byte row slice, written in
-//    the 128-byte swizzled layout the tensor cores read) into a 3-stage ring of
-//    64-key tiles; padded slots are zero-filled without a read.  Rows of the
-//    tile kPrefetch tiles ahead are prefetched into L2, so the ring only has to
-//    cover L2 latency.
+//    the 128-byte swizzled layout the tensor cores read) into a 5-stage ring of
+//    64-key tiles; padded slots are zero-filled without a read.
 //  * The CTA's slice of the 128-head query sits in tensor memory and is the A
-//    operand of the score MMAs (M=128 heads, N=64 keys, the smallest N at which
-//    an MMA is not dominated by its fixed issue cost).
-//  * Four exchange warps copy each tile's partial scores from TMEM to shared
-//    memory and ship them to the partner in one bulk copy that completes
-//    transaction bytes on the partner's barrier (distributed shared memory is
-//    the narrowest link of this kernel, so the copy runs off the softmax path);
-//    the partner's softmax frees the receive buffer with a remote arrive.
-//  * Eight softmax warps: thread = (head = TMEM lane, half of the tile's keys).
-//    A pair of warps shares a head range; the two halves swap their tile maxima
-//    in shared memory, so both apply the same reference.  Online base-2
-//    softmax; O is rescaled only when a tile's maximum exceeds the reference by
-//    more than 2^8.  P goes back to TMEM as bf16; both CTAs hold identical
-//    scores and probabilities.
+//    operand of the score MMAs (M=128 heads, N=64 keys).
+//  * Four exchange warps copy each tile's partial scores from tensor memory
+//    (which frees the score accumulator for the next tile at once) to this
+//    CTA's slot of an L2-resident scratch buffer and signal both softmaxes: this
+//    CTA's through a local barrier, the partner's through a remote arrive.
+//    Distributed shared memory carries only those barrier arrivals.
+//  * Four softmax warps, thread = head = TMEM lane: the thread adds the two
+//    partial scores of its head for the tile's 64 keys, runs an online base-2
+//    softmax (O is rescaled only when a tile's maximum exceeds the reference by
+//    more than 2^8) and writes P as bf16 to tensor memory.  Both CTAs compute
+//    the same P.
 //  * O[128 x 256] (+)= P . V on the tensor cores with P from TMEM and V = the
-//    gathered latent slice read MN-major: the tile gathered for the scores is
-//    reused, so every selected row is read from memory once, and each CTA
-//    aggregates its own 256 latent dims.
+//    gathered latent slice read MN-major.  The MMA warp issues whichever of the
+//    next score MMA and the next aggregation is ready, so the scores of later
+//    tiles run ahead of the softmax.
+//  * The output leaves through shared memory, one bulk copy per head.
 //  * Rows with few queries split their keys over several clusters; partial
 //    (O, m, l) states go to a workspace and a combine kernel merges them.
 #include "sa_device.cuh"
@@ -44,21 +46,18 @@ namespace {
 
 constexpr int kPage = 64;
 constexpr int kNK = 64;           // keys per tile
-constexpr int kHalf = kNK / 2;    // keys per softmax thread
-constexpr int kStages = 3;
-constexpr int kPrefetch = 4;      // tiles prefetched into L2 ahead of the copy
+constexpr int kStages = 5;
 constexpr int kBlkK = kNK * 128;  // one 64-dim slice of a tile (bytes)
 constexpr int kMaxBlk = 5;        // 64-dim slices per CTA (CTA 1: 4 latent + 1 RoPE)
 constexpr int kStageBytes = kMaxBlk * kBlkK;
-constexpr int kXBytes = 128 * kNK * 4;  // one tile of partial scores (128 heads x 64 keys fp32)
 constexpr int kOffStage = 0;
-constexpr int kOffX = kOffStage + kStages * kStageBytes;  // partner's halves, 2 buffers
-constexpr int kOffL = kOffX + 2 * kXBytes;                // this CTA's half, staged for the copy
-constexpr int kSmem = kOffL + kXBytes + 1024;
-constexpr int kSmxWarps = 8;
+constexpr int kOffRows = kOffStage + kStages * kStageBytes;  // [kMaxTilesPerCta * kNK] pool rows
+constexpr int kSmem = kOffRows + kMaxTilesPerCta * kNK * 4 + 1024;
+constexpr int kORowBytes = 256 * 4 + 16;  // one head's output row staged in shared memory (padded)
+constexpr int kSmxWarps = 4;
 constexpr int kXchgWarp0 = kSmxWarps;
 constexpr int kProdWarp0 = kXchgWarp0 + 4;
-constexpr int kProdWarps = 2;
+constexpr int kProdWarps = 6;
 constexpr int kMmaWarp = kProdWarp0 + kProdWarps;
 constexpr int kThreads = 32 * (kMmaWarp + 1);
 constexpr uint32_t kTmemCols = 512;
@@ -67,14 +66,18 @@ constexpr uint32_t kColS = 256;  // S: 64 fp32 columns
 constexpr uint32_t kColP = 320;  // P: 64 bf16 = 32 columns
 constexpr uint32_t kColQ = 352;  // query slice: up to 320 bf16 = 160 columns
 constexpr float kRescaleLog2 = 8.0f;
+constexpr int kXFloats = kMlaXBytes / 4;  // floats per exchange buffer
 
-static_assert(kSmem <= 232448, "shared memory budget");
+static_assert(kSmem <= 232448 - 2048, "shared memory budget");
 static_assert(kColQ + 160 <= kTmemCols, "tensor memory budget");
-static_assert(kStageBytes % 1024 == 0 && kXBytes % 1024 == 0, "swizzle atoms stay 1024-byte aligned");
+static_assert(kStageBytes % 1024 == 0, "swizzle atoms stay 1024-byte aligned");
+static_assert(128 * kORowBytes <= kStages * kStageBytes, "the output rows fit in the stage ring");
+static_assert(kMlaXBytes == 128 * kNK * 4, "one exchange buffer holds a tile of fp32 partial scores");
 
 struct MlaKernelArgs {
     MlaArgs a;
     int nsplit;
+    float* xs;     // exchange scratch: [kMlaScratchSlots][kMlaXBuf][16 chunks][128 heads][4] fp32
     float* ws_o;   // [rows][nsplit][H][512] partial outputs (nsplit > 1)
     float* ws_ml;  // [rows][nsplit][H][4] partial (m, l of bf16 P, l of fp32 P, unused)
 };
@@ -118,22 +121,25 @@ __device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&v)[64]) {
     tmem_ld_wait();
 }
 
+__device__ __forceinline__ uint32_t sm_id() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%smid;" : "=r"(r));
+    return r;
+}
+
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1) mla_kernel(const MlaKernelArgs ka) {
     const MlaArgs& a = ka.a;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sStage = sm + kOffStage;
-    uint8_t* sX = sm + kOffX;
-    uint8_t* sL = sm + kOffL;
+    int* sRows = reinterpret_cast<int*>(sm + kOffRows);
 
-    __shared__ uint64_t bar_full[kStages], bar_empty[kStages], bar_sfull, bar_sfree, bar_xfull[2], bar_xfree[2],
-        bar_pfull, bar_pvdone, bar_final;
+    __shared__ uint64_t bar_full[kStages], bar_empty[kStages], bar_sfull, bar_sfree, bar_lfull[kMlaXBuf],
+        bar_lfree[kMlaXBuf], bar_xfull[kMlaXBuf], bar_xfree[kMlaXBuf], bar_pfull, bar_pvdone, bar_final;
     __shared__ uint32_t s_tmem;
+    __shared__ uint32_t s_slot;  // this CTA's scratch slot (its SM id); the partner reads it remotely
     __shared__ int s_abort;
-    __shared__ volatile int s_xfail;     // written only by exchange threads (see the exchange loop)
-    __shared__ volatile int s_pfail[4];  // written only by softmax pair q (see the softmax loop)
-    __shared__ float s_pmax[2][2][128];  // [tile parity][key half][head] tile maxima
-    __shared__ float s_psum[2][2][128];  // (l, lx) of the two key halves, for the output
+    __shared__ volatile int s_xfail;  // written only by exchange threads (see the exchange loop)
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t rank = cluster_rank(), partner = rank ^ 1u;
@@ -143,22 +149,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1) mla_ker
     const int T = (a.k + kNK - 1) / kNK;
     const int t0 = static_cast<int>(static_cast<int64_t>(split) * T / ka.nsplit);
     const int t1 = static_cast<int>(static_cast<int64_t>(split + 1) * T / ka.nsplit);
-    const int nt = t1 - t0;
+    const int nt = t1 - t0;  // at most kMaxTilesPerCta (the host picks the splits)
     const int seq = a.seq_of_row ? a.seq_of_row[r] : r;
     WaitCtx wc{a.err, &s_abort};
 
     if (tid == 0) {
+        const uint32_t slot = sm_id();
+        s_slot = slot;
         s_abort = 0;
         s_xfail = 0;
-        for (int q = 0; q < 4; ++q) s_pfail[q] = 0;
+        if (slot >= static_cast<uint32_t>(kMlaScratchSlots) || nt > kMaxTilesPerCta) {
+            record_error(a.err, kErrMlaWait | 20);  // no scratch slot for this SM: do nothing
+            s_abort = 1;
+        }
         for (int i = 0; i < kStages; ++i) {
             mbar_init(&bar_full[i], 32 * kProdWarps);
             mbar_init(&bar_empty[i], 1);
         }
         mbar_init(&bar_sfull, 1);
-        mbar_init(&bar_sfree, kSmxWarps + 4);  // softmax and exchange warps both read S
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&bar_xfull[i], 1);
+        mbar_init(&bar_sfree, 4);  // the exchange warps read S
+        for (int i = 0; i < kMlaXBuf; ++i) {
+            mbar_init(&bar_lfull[i], 1);          // exchange thread 0, after its fence
+            mbar_init(&bar_lfree[i], kSmxWarps);  // this CTA's softmax warps
+            mbar_init(&bar_xfull[i], 1);          // the partner's exchange thread 0
             mbar_init(&bar_xfree[i], kSmxWarps);  // the partner's softmax warps
         }
         mbar_init(&bar_pfull, kSmxWarps);
@@ -170,10 +183,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1) mla_ker
         tmem_alloc(&s_tmem, kTmemCols);
         tmem_relinquish();
     }
+    // pool rows of every slot of this CTA's tiles (-1: padded slot)
+    for (int i = tid; i < nt * kNK && nt <= kMaxTilesPerCta; i += kThreads) {
+        const int p = idx_at(a, r, t0 * kNK + i);
+        sRows[i] = p >= 0 ? static_cast<int>(pool_row(a, seq, p)) : -1;
+    }
     tc_fence_before();
-    cluster_sync_all();  // partner's barriers exist before any remote write
+    cluster_sync_all();  // barriers, row table and slot are in place, and the partner has started
     tc_fence_after();
     const uint32_t tmem = s_tmem;
+    const uint32_t my_slot = s_slot;
+    const uint32_t peer_slot = ld_cluster_u32(mapa_u32(smem_u32(&s_slot), partner));
+    // both CTAs skip the work alike when either has no scratch slot (recorded above)
+    const bool run = my_slot < static_cast<uint32_t>(kMlaScratchSlots) &&
+                     peer_slot < static_cast<uint32_t>(kMlaScratchSlots) && nt <= kMaxTilesPerCta;
 
     if (warp < 4) {
         // The query slice of head `tid` into its TMEM lane: column c holds
@@ -216,36 +239,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1) mla_ker
     __syncthreads();
     tc_fence_after();
 
-    if (warp >= kProdWarp0 && warp < kMmaWarp) {
+    if (!run) {
+        // nothing to do: fall through to the teardown
+    } else if (warp >= kProdWarp0 && warp < kMmaWarp) {
         // ------------------------------------------------ producers: gathered row slices
-        // Warp p copies keys p, p+2, ... of each tile: lane = 16-byte chunk of the
-        // 512-byte latent slice (slice b = lane / 8, chunk lane % 8); CTA 1 adds the
-        // 128-byte RoPE keys, 4 keys per instruction.  Lane i holds the pool row of
-        // the warp's i-th key (or -1 for a padded slot), for the kPrefetch tiles in
-        // flight between the L2 prefetch and the copy.
+        // Warp p copies keys p, p + 6, ... of each tile: lane = 16-byte chunk of the
+        // 512-byte latent slice (slice b = lane / 8, chunk lane % 8).  CTA 1 adds the
+        // 128-byte RoPE keys, 4 keys per instruction.
         const int pw = warp - kProdWarp0;
         const __nv_bfloat16* cbase = static_cast<const __nv_bfloat16*>(a.c_cache) + rank * 256 + lane * 8;
         const __nv_bfloat16* kbase = static_cast<const __nv_bfloat16*>(a.kr_cache) + (lane & 7) * 8;
-        constexpr int kPer = kNK / kProdWarps;  // 32 keys per warp per tile
-        auto row_of = [&](int t) -> int {
-            const int p = idx_at(a, r, (t0 + t) * kNK + pw + kProdWarps * lane);
-            return p >= 0 ? static_cast<int>(pool_row(a, seq, p)) : -1;
-        };
-        auto prefetch_rows = [&](int row) {
-            if (row < 0) return;
-            const char* c = reinterpret_cast<const char*>(static_cast<const __nv_bfloat16*>(a.c_cache) +
-                                                          static_cast<int64_t>(row) * a.c_ld + rank * 256);
-#pragma unroll
-            for (int o = 0; o < 512; o += 128) prefetch_l2(c + o);
-            if (rank == 1)
-                prefetch_l2(static_cast<const __nv_bfloat16*>(a.kr_cache) + static_cast<int64_t>(row) * a.kr_ld);
-        };
-        int ring[kPrefetch];  // rows of tiles t .. t + kPrefetch - 1
-#pragma unroll
-        for (int d = 0; d < kPrefetch; ++d) {
-            ring[d] = d < nt ? row_of(d) : -1;
-            prefetch_rows(ring[d]);
-        }
+        const int b = lane >> 3, c = lane & 7;
         int stage = 0;
         uint32_t phase = 0;
         for (int t = 0; t < nt; ++t) {
@@ -253,31 +257,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1) mla_ker
             if (lane == 0) ok = mbar_wait(&bar_empty[stage], phase ^ 1, wc, kErrMlaWait | 1);
             ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
             if (!ok) break;
-            const int myrow = ring[0];
+            const int* trow = sRows + t * kNK;
             const uint32_t sbase = smem_u32(sStage + stage * kStageBytes);
-            const int b = lane >> 3, c = lane & 7;
-#pragma unroll 8
-            for (int i = 0; i < kPer; ++i) {
-                const int j = pw + kProdWarps * i;
-                const int row = __shfl_sync(0xffffffffu, myrow, i);
+#pragma unroll 4
+            for (int j = pw; j < kNK; j += kProdWarps) {
+                const int row = trow[j];
                 const uint32_t dst = sbase + b * kBlkK + j * 128 + ((c ^ (j & 7)) << 4);
                 cp_async16(dst, cbase + static_cast<int64_t>(row < 0 ? 0 : row) * a.c_ld, row < 0 ? 0u : 16u);
             }
             if (rank == 1) {
-#pragma unroll
-                for (int i0 = 0; i0 < kPer; i0 += 4) {
-                    const int i = i0 + (lane >> 3);
-                    const int j = pw + kProdWarps * i;
-                    const int row = __shfl_sync(0xffffffffu, myrow, i);
+                for (int j0 = 4 * pw; j0 < kNK; j0 += 4 * kProdWarps) {
+                    const int j = j0 + (lane >> 3);
+                    const int row = trow[j];
                     const uint32_t dst = sbase + 4 * kBlkK + j * 128 + ((c ^ (j & 7)) << 4);
                     cp_async16(dst, kbase + static_cast<int64_t>(row < 0 ? 0 : row) * a.kr_ld, row < 0 ? 0u : 16u);
                 }
             }
             cp_async_arrive_noinc(&bar_full[stage]);
-#pragma unroll
-            for (int d = 0; d + 1 < kPrefetch; ++d) ring[d] = ring[d + 1];
-            ring[kPrefetch - 1] = t + kPrefetch < nt ? row_of(t + kPrefetch) : -1;
-            prefetch_rows(ring[kPrefetch - 1]);
             if (++stage == kStages) {
                 stage = 0;
                 phase ^= 1;
@@ -286,49 +282,62 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1) mla_ker
         cp_async_wait_all();  // every copy lands before the CTA can exit
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------ MMA issuer
+        // Polls (without blocking) for the next score tile (its rows landed and the
+        // exchange warps have read the previous scores) and for the next
+        // aggregation (its P is written), and issues whichever is ready.
         constexpr uint32_t id_qk = idesc_f32acc(1, 1, false, false, 128, kNK);
         constexpr uint32_t id_pv = idesc_f32acc(1, 1, false, true, 128, 256);
-        bool ok = true;
         if (lane == 0) {
-            int stage = 0;
-            uint32_t phase = 0;
-            for (int i = 0; i <= nt && ok; ++i) {
-                if (i < nt) {
-                    ok = mbar_wait(&bar_full[stage], phase, wc, kErrMlaWait | 4);
-                    if (ok && i >= 1) ok = mbar_wait(&bar_sfree, static_cast<uint32_t>((i - 1) & 1), wc, kErrMlaWait | 5);
-                    if (!ok) break;
+            int iq = 0, ip = 0;  // next score tile, next aggregation tile
+            int qstage = 0;
+            uint32_t qphase = 0;
+            unsigned long long t_last = global_ns();
+            while (ip < nt) {
+                bool did = false;
+                if (iq < nt && mbar_test_wait(&bar_full[qstage], qphase) &&
+                    (iq == 0 || mbar_test_wait(&bar_sfree, static_cast<uint32_t>((iq - 1) & 1)))) {
                     fence_proxy_async_smem();  // cp.async writes -> tensor-core reads
                     tc_fence_after();
-                    uint8_t* stg = sStage + stage * kStageBytes;
-                    for (int b = 0; b < nblk; ++b) {
-                        const uint64_t kd = sdesc(smem_u32(stg + b * kBlkK), 16, 1024, kSw128);
+                    uint8_t* stg = sStage + qstage * kStageBytes;
+                    for (int bb = 0; bb < nblk; ++bb) {
+                        const uint64_t kd = sdesc(smem_u32(stg + bb * kBlkK), 16, 1024, kSw128);
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk)
-                            mma_bf16_ts(tmem + kColS, tmem + kColQ + 32 * b + 8 * kk, kd + 2 * kk, id_qk,
-                                        (b | kk) != 0 ? 1u : 0u);
+                            mma_bf16_ts(tmem + kColS, tmem + kColQ + 32 * bb + 8 * kk, kd + 2 * kk, id_qk,
+                                        (bb | kk) != 0 ? 1u : 0u);
                     }
                     tc_commit(&bar_sfull);
-                    if (++stage == kStages) {
-                        stage = 0;
-                        phase ^= 1;
+                    ++iq;
+                    if (++qstage == kStages) {
+                        qstage = 0;
+                        qphase ^= 1;
                     }
+                    did = true;
                 }
-                const int u = i - 1;
-                if (u >= 0) {
-                    ok = mbar_wait(&bar_pfull, static_cast<uint32_t>(u & 1), wc, kErrMlaWait | 3);
-                    if (!ok) break;
+                if (ip < iq && mbar_test_wait(&bar_pfull, static_cast<uint32_t>(ip & 1))) {
                     tc_fence_after();
-                    const int st = u % kStages;
+                    const int st = ip % kStages;
                     const uint64_t vd = sdesc(smem_u32(sStage + st * kStageBytes), kBlkK, 1024, kSw128);
 #pragma unroll
                     for (int kk = 0; kk < kNK / 16; ++kk)
-                        mma_bf16_ts(tmem + kColO, tmem + kColP + 8 * kk, vd + 128 * kk, id_pv, (u > 0 || kk > 0) ? 1u : 0u);
+                        mma_bf16_ts(tmem + kColO, tmem + kColP + 8 * kk, vd + 128 * kk, id_pv,
+                                    (ip > 0 || kk > 0) ? 1u : 0u);
                     tc_commit(&bar_empty[st]);
                     tc_commit(&bar_pvdone);
+                    ++ip;
+                    did = true;
+                }
+                if (did) {
+                    t_last = global_ns();
+                } else {
+                    if (*wc.abort) break;
+                    if (global_ns() - t_last > kWaitLimitNs) {
+                        record_error(a.err, kErrMlaWait | 4);
+                        s_abort = 1;
+                        break;
+                    }
                 }
             }
-        }
-        if (lane == 0) {
             int dummy = 0;
             WaitCtx dw{a.err, reinterpret_cast<volatile int*>(&dummy)};
             tc_commit(&bar_final);
@@ -336,18 +345,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1) mla_ker
         }
         __syncwarp();
     } else if (warp >= kXchgWarp0) {
-        // ------------------------------------------------ exchange: this CTA's partial scores -> partner
-        // Named barrier 2 spans the 128 exchange threads.  A failed (timed-out)
-        // wait is recorded in s_xfail, which only exchange threads write, before
-        // the barrier, and every exchange thread reads it after the barrier: the
-        // four warps always leave the loop together, never one of them stuck in
-        // bar.sync.
+        // ------------------------------------------------ exchange: partial scores -> L2 scratch
+        // Thread h moves head h's 64 partial scores of tile t into buffer t % kMlaXBuf
+        // of this CTA's scratch slot (layout [16-byte chunk][head], so each warp
+        // store covers 512 contiguous bytes).  Named barrier 2 spans the 128
+        // exchange threads.  A failed (timed-out) wait is recorded in s_xfail,
+        // which only exchange threads write, before the barrier, and every
+        // exchange thread reads it after the barrier: the four warps always leave
+        // the loop together, never one of them stuck in bar.sync.
         const int h = tid - 32 * kXchgWarp0;
         const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-        const uint32_t x_remote = mapa_u32(smem_u32(sX), partner);
+        float* myx = ka.xs + static_cast<size_t>(my_slot) * kMlaXBuf * kXFloats;
         const uint32_t xfull_remote = mapa_u32(smem_u32(&bar_xfull[0]), partner);
         for (int t = 0; t < nt; ++t) {
-            const int xb = t & 1;
+            const int xb = t % kMlaXBuf;
             uint32_t v[64];
             const bool got = warp_wait(&bar_sfull, static_cast<uint32_t>(t & 1), wc, kErrMlaWait | 14);
             if (got) {
@@ -359,106 +370,93 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1) mla_ker
             } else if (lane == 0) {
                 s_xfail = 1;
             }
-            // the partner's softmax has read its buffer xb (tile t - 2); the previous copy has read L
-            if (h == 0) {
-                if (t >= 2 && !mbar_wait<true>(&bar_xfree[xb], static_cast<uint32_t>(((t >> 1) - 1) & 1), wc,
-                                               kErrMlaWait | 15))
-                    s_xfail = 1;
-                bulk_wait_read_all();
+            // buffer xb last held tile t - kMlaXBuf: both softmaxes must have read it
+            if (h == 0 && t >= kMlaXBuf) {
+                const uint32_t par = static_cast<uint32_t>((t / kMlaXBuf - 1) & 1);
+                if (!mbar_wait(&bar_lfree[xb], par, wc, kErrMlaWait | 16)) s_xfail = 1;
+                if (!mbar_wait<true>(&bar_xfree[xb], par, wc, kErrMlaWait | 15)) s_xfail = 1;
             }
             named_sync(2, 128);
             if (s_xfail) break;
-            uint8_t* lrow = sL + h * 256;
+            float4* dst = reinterpret_cast<float4*>(myx + xb * kXFloats);
 #pragma unroll
-            for (int c = 0; c < 16; ++c)
-                *reinterpret_cast<uint4*>(lrow + ((c ^ (h & 7)) << 4)) =
-                    make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
-            fence_proxy_async_smem();
+            for (int c = 0; c < 16; ++c) st_cg_v4(dst + c * 128 + h, v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
             named_sync(2, 128);
-            if (h == 0) bulk_copy_to_cluster(x_remote + xb * kXBytes, sL, kXBytes, xfull_remote + 8 * xb);
+            if (h == 0) {
+                __threadfence();  // the partial scores are in L2 before either softmax is told
+                mbar_arrive(&bar_lfull[xb]);
+                mbar_arrive_cluster(xfull_remote + 8 * xb);
+            }
         }
-        if (h == 0) bulk_wait_all();
     } else {
-        // ------------------------------------------------ softmax + output
-        // Thread = (head h = TMEM lane, key half kh).  Warps q and q + 4 form
-        // pair q and meet at named barrier 3 + q (64 threads) once per tile.  A
-        // failed wait is recorded in s_pfail[q], written only by pair q before
-        // that barrier and read by both warps after it, so the pair always
-        // leaves the loop together.
-        const int q = warp & 3, kh = warp >> 2;
-        const int h = 32 * q + lane;
-        const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+        // ------------------------------------------------ softmax + output (thread = head h)
+        const int h = tid;
+        const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
         const float c2 = a.scale * 1.4426950408889634f;  // scores in base-2 units
         float m = -INFINITY, l = 0.f, lx = 0.f;  // l: sum of bf16 P (normalises O); lx: fp32 sum (lse)
+        const float4* myx = reinterpret_cast<const float4*>(ka.xs + static_cast<size_t>(my_slot) * kMlaXBuf * kXFloats);
+        const float4* px = reinterpret_cast<const float4*>(ka.xs + static_cast<size_t>(peer_slot) * kMlaXBuf * kXFloats);
         const uint32_t xfree_remote = mapa_u32(smem_u32(&bar_xfree[0]), partner);
         bool ok = true;
-        // validity of this half's 32 slots of the next tile (slot = 32 kh + lane)
-        int i_next = nt > 0 ? idx_at(a, r, t0 * kNK + kHalf * kh + lane) : -1;
         for (int t = 0; t < nt; ++t) {
-            const int xb = t & 1;
-            const unsigned vmask = __ballot_sync(0xffffffffu, i_next >= 0);
-            if (t + 1 < nt) i_next = idx_at(a, r, (t0 + t + 1) * kNK + kHalf * kh + lane);
-            if (tid == 0) mbar_arrive_expect_tx(&bar_xfull[xb], kXBytes);  // the partner's half of tile t
-            float s[kHalf];
-            bool got = warp_wait(&bar_sfull, static_cast<uint32_t>(t & 1), wc, kErrMlaWait | 6);
-            if (got) {
-                tc_fence_after();
-                uint32_t v[kHalf];
-                tmem_ld32(tmem + lane_base + kColS + kHalf * kh, v);
-                tmem_ld_wait();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&bar_sfree);
-                got = warp_wait<true>(&bar_xfull[xb], static_cast<uint32_t>((t >> 1) & 1), wc, kErrMlaWait | 7);
-                if (got) {
-                    const uint8_t* xl = sX + xb * kXBytes + h * 256;
+            const int xb = t % kMlaXBuf;
+            const uint32_t par = static_cast<uint32_t>((t / kMlaXBuf) & 1);
+            // which of the tile's 64 slots hold a key
+            const unsigned vm0 = __ballot_sync(0xffffffffu, sRows[t * kNK + lane] >= 0);
+            const unsigned vm1 = __ballot_sync(0xffffffffu, sRows[t * kNK + 32 + lane] >= 0);
+            ok = warp_wait(&bar_lfull[xb], par, wc, kErrMlaWait | 6);
+            if (ok) ok = warp_wait<true>(&bar_xfull[xb], par, wc, kErrMlaWait | 7);
+            if (!ok) break;
+            float s[kNK];
+            {
+                const float4* ow = myx + xb * (kXFloats / 4) + h;
+                const float4* pw4 = px + xb * (kXFloats / 4) + h;
 #pragma unroll
-                    for (int c = 0; c < kHalf / 4; ++c) {
-                        const int cc = 8 * kh + c;  // 16-byte chunk of the row (4 keys)
-                        const float4 x = *reinterpret_cast<const float4*>(xl + ((cc ^ (h & 7)) << 4));
-                        const float xs[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int j = 4 * c + e;
-                            s[j] = ((vmask >> j) & 1u) ? (__uint_as_float(v[j]) + xs[e]) * c2 : -INFINITY;
-                        }
-                    }
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive_cluster(xfree_remote + 8 * xb);  // the partner may refill it
+                for (int c = 0; c < 16; ++c) {
+                    const float4 u = ld_cg_v4(ow + c * 128);
+                    const float4 w = ld_cg_v4(pw4 + c * 128);
+                    s[4 * c + 0] = (u.x + w.x) * c2;
+                    s[4 * c + 1] = (u.y + w.y) * c2;
+                    s[4 * c + 2] = (u.z + w.z) * c2;
+                    s[4 * c + 3] = (u.w + w.w) * c2;
                 }
+            }
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&bar_lfree[xb]);
+                mbar_arrive_cluster(xfree_remote + 8 * xb);  // the partner may refill its buffer
+            }
+#pragma unroll
+            for (int j = 0; j < kNK; ++j) {
+                const unsigned bit = j < 32 ? (vm0 >> j) & 1u : (vm1 >> (j - 32)) & 1u;
+                if (!bit) s[j] = -INFINITY;
             }
             float mx;
             {
-                float tmp[kHalf];
+                float tmp[kNK];
 #pragma unroll
-                for (int j = 0; j < kHalf; ++j) tmp[j] = got ? s[j] : -INFINITY;
+                for (int j = 0; j < kNK; ++j) tmp[j] = s[j];
                 mx = tree_max(tmp);
             }
-            s_pmax[t & 1][kh][h] = mx;  // by parity: the partner may still read tile t - 1
-            if (!got && lane == 0) s_pfail[q] = 1;
-            named_sync(3 + q, 64);
-            if (s_pfail[q]) {
-                ok = false;
-                break;
-            }
-            mx = fmaxf(mx, s_pmax[t & 1][kh ^ 1][h]);
             if (__any_sync(0xffffffffu, mx > m + kRescaleLog2)) {
                 const float m_new = fmaxf(m, mx);
                 const float alpha = (m == -INFINITY) ? 0.f : fast_exp2(m - m_new);
-                if (t > 0) {  // O holds tiles < t: wait for the last product, then scale this half of it
-                    if (warp_wait(&bar_pvdone, static_cast<uint32_t>((t - 1) & 1), wc, kErrMlaWait | 8)) {
-                        tc_fence_after();
-#pragma unroll 1
-                        for (int c = 128 * kh; c < 128 * kh + 128; c += 32) {
-                            uint32_t o[32];
-                            tmem_ld32(tmem + lane_base + kColO + c, o);
-                            tmem_ld_wait();
-#pragma unroll
-                            for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
-                            tmem_st32(tmem + lane_base + kColO + c, o);
-                        }
-                        tmem_st_wait();
+                if (t > 0) {  // O holds tiles < t: wait for the last product, then scale this head's row
+                    if (!warp_wait(&bar_pvdone, static_cast<uint32_t>((t - 1) & 1), wc, kErrMlaWait | 8)) {
+                        ok = false;
+                        break;
                     }
+                    tc_fence_after();
+#pragma unroll 1
+                    for (int c = 0; c < 256; c += 32) {
+                        uint32_t o[32];
+                        tmem_ld32(tmem + lane_base + kColO + c, o);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+                        tmem_st32(tmem + lane_base + kColO + c, o);
+                    }
+                    tmem_st_wait();
                 }
                 l *= alpha;
                 lx *= alpha;
@@ -466,10 +464,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1) mla_ker
             }
             // masked slots are -inf and give exactly 0; a fully masked prefix keeps m at -inf
             const float mref = (m == -INFINITY) ? 0.f : m;
-            uint32_t pk[kHalf / 2];
-            float lb[kHalf / 2], lf[kHalf / 2];
+            uint32_t pk[kNK / 2];
+            float lb[kNK / 2], lf[kNK / 2];
 #pragma unroll
-            for (int j = 0; j < kHalf / 2; ++j) {
+            for (int j = 0; j < kNK / 2; ++j) {
                 const float p0 = fast_exp2(s[2 * j] - mref);
                 const float p1 = fast_exp2(s[2 * j + 1] - mref);
                 const __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
@@ -480,33 +478,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1) mla_ker
             l += tree_sum(lb);
             lx += tree_sum(lf);
             // the product of tile t - 1 has read P before it is overwritten
-            if (t >= 1) warp_wait(&bar_pvdone, static_cast<uint32_t>((t - 1) & 1), wc, kErrMlaWait | 12);
+            if (t >= 1 && !warp_wait(&bar_pvdone, static_cast<uint32_t>((t - 1) & 1), wc, kErrMlaWait | 12)) {
+                ok = false;
+                break;
+            }
             tc_fence_after();
-            tmem_st16(tmem + lane_base + kColP + (kHalf / 2) * kh, pk);
+            tmem_st32(tmem + lane_base + kColP, pk);
             tmem_st_wait();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar_pfull);
         }
-        // ---- output: this thread's half (128 latent dims) of the CTA's 256 dims of head h
-        s_psum[kh][0][h] = l;
-        s_psum[kh][1][h] = lx;
-        named_sync(3 + q, 64);
-        const float lt = s_psum[0][0][h] + s_psum[1][0][h];
-        const float lxt = s_psum[0][1][h] + s_psum[1][1][h];
+        // ---- output: head h's 256 latent dims of this CTA, staged in the idle stage
+        // ring (padded rows: no bank conflicts) and sent with one bulk copy per head
         if (ok && nt > 0)
             ok = warp_wait(&bar_pvdone, static_cast<uint32_t>((nt - 1) & 1), wc, kErrMlaWait | 13);
-        if (ok && !s_abort) {
+        if (ok && !*wc.abort) {
             tc_fence_after();
             const bool partial = ka.nsplit > 1;
-            const float inv = (lt > 0.f && !partial) ? 1.f / lt : 1.f;
-            float* dst;
-            if (partial)
-                dst = ka.ws_o + ((static_cast<int64_t>(r) * ka.nsplit + split) * a.H + h) * 512 + rank * 256;
-            else
-                dst = a.out + (static_cast<int64_t>(r) * a.H + h) * a.d_c + rank * 256;
+            const bool empty = !(l > 0.f);
+            const float inv = (!empty && !partial) ? 1.f / l : 1.f;
+            float* srow = reinterpret_cast<float*>(sStage + h * kORowBytes);
 #pragma unroll 1
-            for (int c = 128 * kh; c < 128 * kh + 128; c += 32) {
+            for (int c = 0; c < 256; c += 32) {
                 uint32_t o[32];
                 if (nt > 0) {
                     tmem_ld32(tmem + lane_base + kColO + c, o);
@@ -515,35 +509,40 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1) mla_ker
 #pragma unroll
                     for (int j = 0; j < 32; ++j) o[j] = 0u;
                 }
-                if (h < a.H) {
-                    const bool empty = !(lt > 0.f);
 #pragma unroll
-                    for (int j = 0; j < 32; j += 4) {
-                        float4 f;
-                        f.x = empty ? 0.f : __uint_as_float(o[j + 0]) * inv;
-                        f.y = empty ? 0.f : __uint_as_float(o[j + 1]) * inv;
-                        f.z = empty ? 0.f : __uint_as_float(o[j + 2]) * inv;
-                        f.w = empty ? 0.f : __uint_as_float(o[j + 3]) * inv;
-                        *reinterpret_cast<float4*>(dst + c + j) = f;
-                    }
+                for (int j = 0; j < 32; j += 4) {
+                    float4 f;
+                    f.x = empty ? 0.f : __uint_as_float(o[j + 0]) * inv;
+                    f.y = empty ? 0.f : __uint_as_float(o[j + 1]) * inv;
+                    f.z = empty ? 0.f : __uint_as_float(o[j + 2]) * inv;
+                    f.w = empty ? 0.f : __uint_as_float(o[j + 3]) * inv;
+                    *reinterpret_cast<float4*>(srow + c + j) = f;
                 }
             }
-            if (h < a.H && rank == 0 && kh == 0) {
-                if (partial) {
-                    float* ml = ka.ws_ml + ((static_cast<int64_t>(r) * ka.nsplit + split) * a.H + h) * 4;
-                    ml[0] = m;
-                    ml[1] = lt;
-                    ml[2] = lxt;
-                } else if (a.lse) {
-                    a.lse[static_cast<int64_t>(r) * a.H + h] = lt > 0.f ? (m + log2f(lxt)) * 0.6931471805599453f : -INFINITY;
+            fence_proxy_async_smem();  // generic-proxy writes -> bulk-copy reads
+            if (h < a.H) {
+                float* dst = partial ? ka.ws_o + ((static_cast<int64_t>(r) * ka.nsplit + split) * a.H + h) * 512 + rank * 256
+                                     : a.out + (static_cast<int64_t>(r) * a.H + h) * a.d_c + rank * 256;
+                bulk_copy_s2g(dst, srow, 256 * 4);
+                if (rank == 0) {
+                    if (partial) {
+                        float* ml = ka.ws_ml + ((static_cast<int64_t>(r) * ka.nsplit + split) * a.H + h) * 4;
+                        ml[0] = m;
+                        ml[1] = l;
+                        ml[2] = lx;
+                    } else if (a.lse) {
+                        a.lse[static_cast<int64_t>(r) * a.H + h] =
+                            l > 0.f ? (m + log2f(lx)) * 0.6931471805599453f : -INFINITY;
+                    }
                 }
+                bulk_wait_all();
             }
         }
     }
 
     tc_fence_before();
     __syncthreads();
-    cluster_sync_all();  // the partner no longer writes into this CTA's shared memory
+    cluster_sync_all();  // the partner no longer arrives on this CTA's barriers
     tc_fence_after();
     if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
 }
@@ -586,18 +585,25 @@ __global__ void __launch_bounds__(128) mla_combine_kernel(const MlaKernelArgs ka
 int mla_decode_splits(int rows, int k) {
     const int T = (k + kNK - 1) / kNK;
     int ns = sm_count() / (2 * rows);
-    if (ns < 1) ns = 1;
     if (ns > T) ns = T;
     if (ns > 16) ns = 16;
+    const int need = (T + kMaxTilesPerCta - 1) / kMaxTilesPerCta;  // tiles per CTA fit the row table
+    if (ns < need) ns = need;
+    if (ns < 1) ns = 1;
     return ns;
 }
 
+size_t mla_exchange_bytes() { return static_cast<size_t>(kMlaScratchSlots) * kMlaXBuf * kMlaXBytes; }
+
 size_t mla_workspace_bytes(int rows, int H, int k, int d_c, int nsplit) {
     (void)k;
-    if (nsplit <= 1) return 0;
-    const size_t o = static_cast<size_t>(rows) * nsplit * H * d_c * 4;
-    const size_t ml = static_cast<size_t>(rows) * nsplit * H * 4 * 4;
-    return ((o + 255) & ~size_t(255)) + ((ml + 255) & ~size_t(255));
+    size_t total = mla_exchange_bytes();
+    if (nsplit > 1) {
+        const size_t o = static_cast<size_t>(rows) * nsplit * H * d_c * 4;
+        const size_t ml = static_cast<size_t>(rows) * nsplit * H * 4 * 4;
+        total += ((o + 255) & ~size_t(255)) + ((ml + 255) & ~size_t(255));
+    }
+    return total;
 }
 
 sa_status sparse_mla_launch(const MlaArgs& a, int nsplit, void* ws, size_t ws_bytes, cudaStream_t st) {
@@ -606,12 +612,18 @@ sa_status sparse_mla_launch(const MlaArgs& a, int nsplit, void* ws, size_t ws_by
     ka.nsplit = nsplit;
     ka.ws_o = nullptr;
     ka.ws_ml = nullptr;
+    const int T = (a.k + kNK - 1) / kNK;
+    if ((T + nsplit - 1) / nsplit > kMaxTilesPerCta) return SA_EUNSUPPORTED;
+    if (sm_count() > kMlaScratchSlots) return SA_EUNSUPPORTED;
+    const size_t need = mla_workspace_bytes(a.rows, a.H, a.k, a.d_c, nsplit);
+    if (ws == nullptr || ws_bytes < need) return SA_EINVAL;
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    ka.xs = reinterpret_cast<float*>(w);
+    w += mla_exchange_bytes();
     if (nsplit > 1) {
-        const size_t need = mla_workspace_bytes(a.rows, a.H, a.k, a.d_c, nsplit);
-        if (ws == nullptr || ws_bytes < need) return SA_EINVAL;
         const size_t o = static_cast<size_t>(a.rows) * nsplit * a.H * a.d_c * 4;
-        ka.ws_o = static_cast<float*>(ws);
-        ka.ws_ml = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + ((o + 255) & ~size_t(255)));
+        ka.ws_o = reinterpret_cast<float*>(w);
+        ka.ws_ml = reinterpret_cast<float*>(w + ((o + 255) & ~size_t(255)));
     }
     cudaError_t e = cudaFuncSetAttribute(mla_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
     if (e != cudaSuccess) return launch_status(e);

@@ -5,15 +5,22 @@
 // position ("MLA 与稀疏注意力", selected_positions), written in ascending order.
 //
 // One cluster of 8 CTAs per row.  Each CTA copies 1/8 of the row into shared
-// memory as order-preserving 32-bit keys (one read of the scores), then the
-// cluster runs a most-significant-digit-first radix select with 8-bit digits:
-// every CTA builds a histogram of the digit over the keys still in the
-// candidate class, the 8 histograms are summed through distributed shared
-// memory, and the class shrinks to the digit holding the k-th largest key.
-// The search stops as soon as the whole remaining class is taken.  Finally an
-// ordered compaction (warp ballots + prefix counts across warps and CTAs)
-// writes every key above the class plus the first `remaining` keys of the
-// class in position order — ascending output without a sort.
+// memory as order-preserving 32-bit keys (the only read of the scores) and
+// selects with a most-significant-digit-first radix search:
+//  1. First digit = key bits 31..20 (sign, exponent, three mantissa bits).
+//     Every CTA builds a 4096-bin histogram while it loads.  The cluster
+//     reduces it scatter-wise: CTA r sums bins 512r..512r+511 over the eight
+//     CTAs and scans them, the eight block totals are exchanged, and the CTA
+//     that holds the boundary bin (the bin of the k-th largest key) broadcasts
+//     the digit, the count above it and the count inside it.
+//  2. Each CTA lists its keys that carry the boundary digit (the candidates).
+//     The remaining digits (bits 19..12, 11..4, 3..0) are resolved by radix
+//     passes over the candidates only; every pass sums its 256-bin histograms
+//     through distributed shared memory.  The search stops as soon as the whole
+//     remaining class is taken.
+//  3. Ordered compaction (warp ballots + prefix counts across warps and CTAs)
+//     writes every key above the final class plus the first `remaining` keys
+//     of the class in position order: ascending output without a sort.
 #include "sa_device.cuh"
 #include "sa_internal.h"
 
@@ -23,6 +30,10 @@ namespace {
 constexpr int kCluster = 8;
 constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
+constexpr int kBins0 = 4096;                 // first digit: key bits 31..20
+constexpr int kOwn = kBins0 / kCluster;      // first-digit bins reduced by each CTA
+constexpr int kCandCap = 4096;               // candidate slots per CTA
+static_assert(kOwn == kThreads, "one owned bin per thread");
 
 // fp32 -> uint32 whose unsigned order is the float order; -0 and +0 map alike.
 __device__ __forceinline__ uint32_t order_key(float f) {
@@ -31,16 +42,40 @@ __device__ __forceinline__ uint32_t order_key(float f) {
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// Histogram increment by a whole warp: lanes with equal digits add once.
+__device__ __forceinline__ void hist_add(int* hist, bool active, uint32_t digit, int lane) {
+    const unsigned am = __ballot_sync(0xffffffffu, active);
+    if (active) {
+        const unsigned peers = __match_any_sync(am, digit);
+        if (lane == __ffs(peers) - 1) atomicAdd(&hist[digit], __popc(peers));
+    }
+}
+
+// Lane i receives the sum of lanes i..31.
+__device__ __forceinline__ int warp_suffix(int v, int lane) {
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_down_sync(0xffffffffu, v, o);
+        if (lane + o < 32) v += t;
+    }
+    return v;
+}
+
 __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
-    topk_kernel(const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ n_valid, int k,
+    topk_kernel(const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ n_valid, int k, int chunk,
                 int32_t* __restrict__ out) {
-    extern __shared__ uint32_t s_keys[];
+    extern __shared__ __align__(16) uint32_t s_keys[];  // [chunk] keys of this CTA's slice
+    __shared__ int s_hist0[kBins0];
     __shared__ int s_hist[2][256];
     __shared__ int s_suf[257];
-    __shared__ int s_wsum[8];
+    __shared__ int s_wsum[kWarps];
+    __shared__ int s_btot[kCluster];  // first-digit block totals, written by every CTA
+    __shared__ int s_sel0[3];         // boundary digit, count above, count inside (written by its owner)
+    __shared__ int s_sel[3];
+    __shared__ int s_ncand;
+    __shared__ uint16_t s_cand[kCandCap];  // local positions of the candidates
     __shared__ int s_warp_gt[kWarps], s_warp_eq[kWarps];
     __shared__ int s_counts[2];
-    __shared__ int s_sel[3];  // digit, count above the digit, count of the digit
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int row = blockIdx.x / kCluster;
@@ -54,86 +89,164 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
         return;
     }
 
-    const int chunk = (((n + kCluster - 1) / kCluster) + 3) & ~3;
     const int lo = static_cast<int>(rank) * chunk;
     const int cnt = max(0, min(n, lo + chunk) - lo);
     const float* src = scores + static_cast<int64_t>(row) * ld + lo;
-    {
-        const int n4 = cnt >> 2;
-        for (int i = tid; i < n4; i += kThreads) {
-            const float4 v = reinterpret_cast<const float4*>(src)[i];
-            s_keys[4 * i + 0] = order_key(v.x);
-            s_keys[4 * i + 1] = order_key(v.y);
-            s_keys[4 * i + 2] = order_key(v.z);
-            s_keys[4 * i + 3] = order_key(v.w);
-        }
-        for (int i = 4 * n4 + tid; i < cnt; i += kThreads) s_keys[i] = order_key(src[i]);
-    }
 
-    uint32_t prefix = 0, mask = 0;
-    int remaining = k;
-    const int cnt_round = ((cnt + kThreads - 1) / kThreads) * kThreads;
-    for (int pass = 0; pass < 4; ++pass) {
-        const int shift = 24 - 8 * pass;
-        int* hist = s_hist[pass & 1];
-        if (tid < 256) hist[tid] = 0;
-        __syncthreads();
+    for (int i = tid; i < kBins0; i += kThreads) s_hist0[i] = 0;
+    if (tid == 0) s_ncand = 0;
+    __syncthreads();
+
+    // ---- 1. load the slice and histogram its first digit
+    // four vector loads in flight per thread before any of them is consumed
+    const int n4 = cnt >> 2;
+    constexpr int kVec = 4;
+    for (int base = 0; base < n4; base += kVec * kThreads) {
+        float4 v[kVec];
+#pragma unroll
+        for (int u = 0; u < kVec; ++u) {
+            const int i = base + u * kThreads + tid;
+            if (i < n4) v[u] = reinterpret_cast<const float4*>(src)[i];
+        }
+#pragma unroll
+        for (int u = 0; u < kVec; ++u) {
+            const int i = base + u * kThreads + tid;
+            const bool ok = i < n4;
+            uint4 kk = make_uint4(0u, 0u, 0u, 0u);
+            if (ok) {
+                kk = make_uint4(order_key(v[u].x), order_key(v[u].y), order_key(v[u].z), order_key(v[u].w));
+                reinterpret_cast<uint4*>(s_keys)[i] = kk;
+            }
+            hist_add(s_hist0, ok, kk.x >> 20, lane);
+            hist_add(s_hist0, ok, kk.y >> 20, lane);
+            hist_add(s_hist0, ok, kk.z >> 20, lane);
+            hist_add(s_hist0, ok, kk.w >> 20, lane);
+        }
+    }
+    if (warp == 0) {  // up to three keys after the last full vector
+        const int i = 4 * n4 + lane;
+        const bool ok = i < cnt;
+        uint32_t key = 0u;
+        if (ok) {
+            key = order_key(src[i]);
+            s_keys[i] = key;
+        }
+        hist_add(s_hist0, ok, key >> 20, lane);
+    }
+    cluster_sync_all();
+
+    // CTA `rank` reduces bins rank*512 .. rank*512+511 over the cluster
+    const int g = static_cast<int>(rank) * kOwn + tid;
+    int tot = 0;
+    {
+        const uint32_t a = smem_u32(&s_hist0[g]);
+        uint32_t v[kCluster];
+#pragma unroll
+        for (int r = 0; r < kCluster; ++r) v[r] = ld_cluster_u32(mapa_u32(a, static_cast<uint32_t>(r)));
+#pragma unroll
+        for (int r = 0; r < kCluster; ++r) tot += static_cast<int>(v[r]);
+    }
+    int incl = warp_suffix(tot, lane);
+    if (lane == 0) s_wsum[warp] = incl;
+    __syncthreads();
+    for (int w = warp + 1; w < kWarps; ++w) incl += s_wsum[w];  // keys in bins g.. of this CTA's range
+    if (tid < kCluster) {
+        int t = 0;
+        for (int w = 0; w < kWarps; ++w) t += s_wsum[w];
+        st_cluster_u32(mapa_u32(smem_u32(&s_btot[rank]), static_cast<uint32_t>(tid)), static_cast<uint32_t>(t));
+    }
+    cluster_sync_all();
+    for (int r = static_cast<int>(rank) + 1; r < kCluster; ++r) incl += s_btot[r];
+    {
+        const int above = incl - tot;  // keys in bins above g, cluster-wide
+        if (tot > 0 && incl >= k && above < k) {
+            for (int r = 0; r < kCluster; ++r) {
+                const uint32_t a = mapa_u32(smem_u32(&s_sel0[0]), static_cast<uint32_t>(r));
+                st_cluster_u32(a, static_cast<uint32_t>(g));
+                st_cluster_u32(a + 4, static_cast<uint32_t>(above));
+                st_cluster_u32(a + 8, static_cast<uint32_t>(tot));
+            }
+        }
+    }
+    cluster_sync_all();
+
+    uint32_t prefix = static_cast<uint32_t>(s_sel0[0]) << 20, mask = 0xFFF00000u;
+    int remaining = k - s_sel0[1];
+    if (s_sel0[2] != remaining) {
+        // ---- 2. list the candidates (keys carrying the boundary digit) and refine
+        const uint32_t d0 = static_cast<uint32_t>(s_sel0[0]);
+        const int cnt_round = ((cnt + kThreads - 1) / kThreads) * kThreads;
         for (int base = 0; base < cnt_round; base += kThreads) {
             const int i = base + tid;
-            bool active = false;
-            uint32_t digit = 0;
-            if (i < cnt) {
-                const uint32_t key = s_keys[i];
-                active = (key & mask) == prefix;
-                digit = (key >> shift) & 255u;
-            }
-            const unsigned am = __ballot_sync(0xffffffffu, active);
-            if (active) {
-                const unsigned peers = __match_any_sync(am, digit);
-                if (lane == __ffs(peers) - 1) atomicAdd(&hist[digit], __popc(peers));
-            }
+            const bool c = i < cnt && (s_keys[i] >> 20) == d0;
+            const unsigned b = __ballot_sync(0xffffffffu, c);
+            int wbase = 0;
+            if (lane == 0 && b) wbase = atomicAdd(&s_ncand, __popc(b));
+            wbase = __shfl_sync(0xffffffffu, wbase, 0);
+            const int slot = wbase + __popc(b & ((1u << lane) - 1u));
+            if (c && slot < kCandCap) s_cand[slot] = static_cast<uint16_t>(i);
         }
         __syncthreads();
-        cluster_sync_all();
-        // cluster-wide histogram and its suffix sums (bins 255 .. 0)
-        if (tid < 256) {
-            const uint32_t my = smem_u32(&hist[tid]);
-            int tot = 0;
+        // a CTA whose candidates overflow the list scans all of its keys instead
+        const bool listed = s_ncand <= kCandCap;
+        const int nscan = listed ? s_ncand : cnt;
+        const int nscan_round = ((nscan + kThreads - 1) / kThreads) * kThreads;
+        for (int pass = 0; pass < 3; ++pass) {
+            const int shift = pass == 0 ? 12 : (pass == 1 ? 4 : 0);
+            const uint32_t dmask = pass == 2 ? 15u : 255u;
+            int* hist = s_hist[pass & 1];
+            if (tid < 256) hist[tid] = 0;
+            __syncthreads();
+            for (int base = 0; base < nscan_round; base += kThreads) {
+                const int i = base + tid;
+                bool active = false;
+                uint32_t digit = 0;
+                if (i < nscan) {
+                    const uint32_t key = s_keys[listed ? static_cast<int>(s_cand[i]) : i];
+                    active = (key & mask) == prefix;
+                    digit = (key >> shift) & dmask;
+                }
+                hist_add(hist, active, digit, lane);
+            }
+            cluster_sync_all();
+            // cluster-wide histogram and its suffix sums (bins 255 .. 0)
+            if (tid < 256) {
+                const uint32_t my = smem_u32(&hist[tid]);
+                uint32_t v[kCluster];
 #pragma unroll
-            for (uint32_t r = 0; r < kCluster; ++r) tot += static_cast<int>(ld_cluster_u32(mapa_u32(my, r)));
-            int incl = tot;  // suffix within the warp's 32 bins
+                for (int r = 0; r < kCluster; ++r) v[r] = ld_cluster_u32(mapa_u32(my, static_cast<uint32_t>(r)));
+                int t = 0;
 #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int t = __shfl_down_sync(0xffffffffu, incl, o);
-                if (lane + o < 32) incl += t;
+                for (int r = 0; r < kCluster; ++r) t += static_cast<int>(v[r]);
+                const int in = warp_suffix(t, lane);
+                s_suf[tid] = in;
+                if (lane == 0) s_wsum[warp] = in;
             }
-            s_suf[tid] = incl;
-            if (lane == 0) s_wsum[warp] = incl;
-        }
-        __syncthreads();
-        if (tid < 256) {
-            int add = 0;
-            for (int w = warp + 1; w < 8; ++w) add += s_wsum[w];
-            s_suf[tid] += add;
-            if (tid == 0) s_suf[256] = 0;
-        }
-        __syncthreads();
-        if (tid < 256) {
-            const int here = s_suf[tid], above = s_suf[tid + 1];
-            if (here >= remaining && above < remaining) {
-                s_sel[0] = tid;
-                s_sel[1] = above;
-                s_sel[2] = here - above;
+            __syncthreads();
+            if (tid < 256) {
+                int add = 0;
+                for (int w = warp + 1; w < 8; ++w) add += s_wsum[w];
+                s_suf[tid] += add;
+                if (tid == 0) s_suf[256] = 0;
             }
+            __syncthreads();
+            if (tid < 256) {
+                const int here = s_suf[tid], above = s_suf[tid + 1];
+                if (here >= remaining && above < remaining) {
+                    s_sel[0] = tid;
+                    s_sel[1] = above;
+                    s_sel[2] = here - above;
+                }
+            }
+            __syncthreads();
+            remaining -= s_sel[1];
+            prefix |= static_cast<uint32_t>(s_sel[0]) << shift;
+            mask |= dmask << shift;
+            if (s_sel[2] == remaining) break;  // the whole class is taken
         }
-        __syncthreads();
-        remaining -= s_sel[1];
-        prefix |= static_cast<uint32_t>(s_sel[0]) << shift;
-        mask |= 255u << shift;
-        if (s_sel[2] == remaining) break;  // the whole class is taken
     }
 
-    // ---- ordered compaction
+    // ---- 3. ordered compaction
     const int seg = (cnt + kWarps - 1) / kWarps;
     const int ws = min(cnt, warp * seg), we = min(cnt, ws + seg);
     int gt_w = 0, eq_w = 0;
@@ -154,23 +267,23 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
     }
     __syncthreads();
     if (tid == 0) {
-        int g = 0, e = 0;
+        int gsum = 0, esum = 0;
         for (int w = 0; w < kWarps; ++w) {
-            g += s_warp_gt[w];
-            e += s_warp_eq[w];
+            gsum += s_warp_gt[w];
+            esum += s_warp_eq[w];
         }
-        s_counts[0] = g;
-        s_counts[1] = e;
+        s_counts[0] = gsum;
+        s_counts[1] = esum;
     }
     cluster_sync_all();
     // offsets of this CTA: ranks below take their "above" keys and their share of the class
     int off = 0, eq_before = 0;
     for (uint32_t r = 0; r < rank; ++r) {
-        const int g = static_cast<int>(ld_cluster_u32(mapa_u32(smem_u32(&s_counts[0]), r)));
-        const int e = static_cast<int>(ld_cluster_u32(mapa_u32(smem_u32(&s_counts[1]), r)));
-        const int take = max(0, min(e, remaining - eq_before));
-        off += g + take;
-        eq_before += e;
+        const int gr = static_cast<int>(ld_cluster_u32(mapa_u32(smem_u32(&s_counts[0]), r)));
+        const int er = static_cast<int>(ld_cluster_u32(mapa_u32(smem_u32(&s_counts[1]), r)));
+        const int take = max(0, min(er, remaining - eq_before));
+        off += gr + take;
+        eq_before += er;
     }
     const int take_c = max(0, min(s_counts[1], remaining - eq_before));
     // offsets of this warp inside the CTA
@@ -209,7 +322,7 @@ sa_status topk_select_launch(const float* scores, int64_t ld, const int32_t* n_v
     cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return launch_status(e);
-    topk_kernel<<<rows * kCluster, kThreads, smem, st>>>(scores, ld, n_valid, k, idx_out);
+    topk_kernel<<<rows * kCluster, kThreads, smem, st>>>(scores, ld, n_valid, k, chunk, idx_out);
     return launch_status(cudaGetLastError());
 }
 

@@ -39,7 +39,8 @@ def assert_lse_close(got, want, what=""):
     want = np.asarray(want, dtype=np.float64)
     both_inf = np.isneginf(got) & np.isneginf(want)
     assert (np.isneginf(got) == np.isneginf(want)).all(), f"{what}: -inf pattern differs"
-    assert np.abs(np.where(both_inf, 0, got - want)).max() <= LSE_ABS, what
+    err = np.abs(np.where(both_inf, 0, got - want))
+    assert err.max() <= LSE_ABS, f"{what}: max abs error {err.max():.3e}"
 
 
 def check_rows(inp, rows, scores, idx, out, lse):

@@ -91,7 +91,7 @@ def _mla(L, fn, **kw):
             a["idx"], a["rows"], a["H"], a["k"], a["dc"], a["dR"], a["scale"], a["out"], a["lse"]]
     if fn == "decode":
         return L.sa_sparse_mla_decode(*args, None, 0, None)
-    return L.sa_sparse_mla_prefill(*args, None)
+    return L.sa_sparse_mla_prefill(*args, None, 0, None)
 
 
 @pytest.mark.parametrize("fn", ["decode", "prefill"])
@@ -107,6 +107,7 @@ def test_sparse_mla_validation(L, fn):
     assert _mla(L, fn, cld=520 + 4) == sa.SA_EINVAL            # row stride not 16-byte aligned
     assert _mla(L, fn, c=MISALIGNED) == sa.SA_EINVAL
     assert _mla(L, fn, cld=256) == sa.SA_EINVAL                # stride shorter than a row
+    assert _mla(L, fn) == sa.SA_EINVAL                         # no workspace
 
 
 def test_block_validation(L):

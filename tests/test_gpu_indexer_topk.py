@@ -113,3 +113,10 @@ def test_topk_all_equal_and_signed_zero():
 
 def test_topk_max_row_length():
     _topk_case(1, [262144], 2048, 9, lo=-100, hi=100)
+
+
+def test_topk_many_candidates():
+    """Two values only: the boundary digit holds about half of every slice,
+    more keys than a CTA lists as candidates, so the refinement scans the slice."""
+    _topk_case(3, [131072, 100000, 65536], 2048, 11, lo=0, hi=1)
+    _topk_case(2, [131072, 70001], 60000, 12, lo=0, hi=1)

@@ -1,8 +1,9 @@
 """sa_sparse_mla_decode_static: sparse MLA decode for callers that cannot
 allocate device memory (no allocator of their own to hand the library a
 workspace, or code running where cudaMalloc is not allowed).  The call keeps
-its split-key partial states in the library's static device array, so its
-results must match sa_sparse_mla_decode given a caller workspace.
+its scratch (the partial-score exchange area and the split-key partial
+states) in the library's static device array, so its results must match
+sa_sparse_mla_decode given a caller workspace.
 
 This file is named so that pytest collects it last: a run that stops at the
 first failure has run every other test before it reaches this one."""
@@ -54,18 +55,19 @@ def test_static_scratch_decode_matches_workspace_decode():
 
 
 def test_static_scratch_rejects_shapes_beyond_the_array():
-    """Shapes whose partial states exceed the static array are refused on the
-    host, before any launch (no device pointer is touched)."""
+    """Shapes whose scratch (exchange area plus split-key partial states)
+    exceeds the static array are refused on the host, before any launch (no
+    device pointer is touched)."""
     from sparse_attention_07_b200 import build
     build.build()
     L = sa.lib()
     rejected = 0
-    for rows in (1, 2, 4, 8, 16, 37):
-        need = sa.sparse_mla_workspace_size(rows, 128, 2048, 512)
+    for rows, k in ((1, 2048), (37, 4096), (74, 8192), (100, 8192)):
+        need = sa.sparse_mla_workspace_size(rows, 128, k, 512)
         if need <= sa.STATIC_SCRATCH_BYTES:
             continue
         st = L.sa_sparse_mla_decode_static(FAKE, FAKE, FAKE, 512, FAKE, 64, 1024, None, 16, None, FAKE, rows, 128,
-                                           2048, 512, 64, 0.07, FAKE, None, None)
+                                           k, 512, 64, 0.07, FAKE, None, None)
         assert st == sa.SA_EUNSUPPORTED
         rejected += 1
     assert rejected > 0, "no shape exceeded the static array"
