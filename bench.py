@@ -36,11 +36,11 @@ import workloads as W  # noqa: E402
 DECODE_METRIC = "sparse-MLA decode queries/s (indexer+topk+attn) at L=32K/128K; % HBM roofline"
 L2_FLUSH_BYTES = 256 << 20  # > 126 MB L2
 
-# dram__bytes_read.sum + dram__bytes_write.sum of the indexer kernel, per launch,
-# from one ncu capture of the long-decode workload, with the sha256 of the
+# dram__bytes_read.sum + dram__bytes_write.sum per launch of the roofline
+# kernel of a workload, from one ncu capture, with the sha256 prefix of the
 # kernel source it was taken on (the figure is reported only while they match).
 TRAFFIC = {
-    "long": {"bytes_per_launch": None, "src_sha": None},
+    "long": {"kernel": "sparse_mla.cu", "bytes_per_launch": None, "src_sha": None},
 }
 
 
@@ -185,8 +185,14 @@ class DecodeStep:
                              page_table=i["page_table"], seq_of_row=i["seq_of_row"], scores=self.scores)
 
     def rest(self):
+        self.topk()
+        self.attn()
+
+    def topk(self):
+        self.sa.topk_select(self.scores, self.inp["n_visible"], self.cfg.topk, idx_out=self.idx)
+
+    def attn(self):
         i, c = self.inp, self.cfg
-        self.sa.topk_select(self.scores, i["n_visible"], c.topk, idx_out=self.idx)
         if self.prefill:
             self.sa.sparse_mla_prefill(i["q_lat"], i["q_rope"], i["c_cache"], i["kr_cache"], self.idx, c.scale,
                                        c.pages_per_seq, page_table=i["page_table"], seq_of_row=i["seq_of_row"],
@@ -213,22 +219,31 @@ class BlockStep:
     def rest(self):
         pass
 
+    def topk(self):
+        pass
+
+    def attn(self):
+        pass
+
 
 def time_steps(step, K: int, flush):
-    """K steps, each bracketed by CUDA events on the launching stream; the L2
-    flush runs between steps outside the events.  Returns per-step and
-    first-kernel times (ms)."""
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
-           torch.cuda.Event(enable_timing=True)) for _ in range(K)]
-    for e0, e1, e2 in ev:
+    """K steps, each bracketed by CUDA events on the launching stream (torch's
+    current stream, which the library calls use); the L2 flush runs between
+    steps outside the events.  Returns per-step times and the per-step times of
+    the three stages (indexer, Top-K, attention) in ms."""
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    for e in ev:
         flush.zero_()
-        e0.record()
+        e[0].record()
         step.indexer()
-        e1.record()
-        step.rest()
-        e2.record()
+        e[1].record()
+        step.topk()
+        e[2].record()
+        step.attn()
+        e[3].record()
     torch.cuda.synchronize()
-    return [e0.elapsed_time(e2) for e0, e1, e2 in ev], [e0.elapsed_time(e1) for e0, e1, e2 in ev]
+    return ([e[0].elapsed_time(e[3]) for e in ev],
+            [[e[j].elapsed_time(e[j + 1]) for e in ev] for j in range(3)])
 
 
 def e2e_steps(step, K: int, flush):
@@ -340,7 +355,7 @@ def run_native(args):
         torch.distributed.barrier()
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
-        step_ms, first_ms = time_steps(step, args.steps, flush)
+        step_ms, stage_ms = time_steps(step, args.steps, flush)
     if ws > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
@@ -350,9 +365,10 @@ def run_native(args):
         raise RuntimeError(f"device error word 0x{err:x}")
 
     ms = statistics.mean(step_ms)
-    first = statistics.mean(first_ms)
+    t_idx, t_topk, t_attn = (statistics.mean(x) for x in stage_ms)
     e2e = statistics.mean(e2e_ms)
-    ms, first, e2e = reduce_max([ms, first, e2e], ws, dev)
+    ms, t_idx, t_topk, t_attn, e2e = reduce_max([ms, t_idx, t_topk, t_attn, e2e], ws, dev)
+    first = t_idx
 
     hbm, bf16_burst, bf16_sus, peak_src = peaks()
     res = {"impl": "native"}
@@ -362,27 +378,49 @@ def run_native(args):
         unit = "tokens/s" if prefill else "queries/s"
         metric = "sparse-MLA prefill tokens/s (indexer+topk+attn)" if prefill else DECODE_METRIC
         keys_b, rows_b = decode_bytes(cfg)
+        score_b = int(cfg.n_visible().sum()) * 4
+        fi, fm = prefill_flops(cfg)
+        # a prefill step lasts milliseconds (sustained peak); a decode step is a short burst
+        bf16_peak = bf16_sus if prefill else bf16_burst
+        fp8_peak = bf16_peak * 2.0  # fp8 dense rate = 2x bf16 (nominal ratio)
+        kern = {
+            "indexer": {"kernel": "idx_tc_kernel" if cfg.idx_dtype == "e4m3" else "idx_cc_kernel", "us": t_idx * 1e3,
+                        "bytes": keys_b, "flop": fi, "flop_peak": fp8_peak},
+            "topk": {"kernel": "topk_kernel", "us": t_topk * 1e3, "bytes": score_b},
+            "attn": {"kernel": "mla_kernel" + ("" if prefill else " (+ mla_combine_kernel)"), "us": t_attn * 1e3,
+                     "bytes": rows_b, "flop": fm, "flop_peak": bf16_peak},
+        }
+        for v in kern.values():
+            v["hbm_gbs"] = round(v["bytes"] / (v["us"] * 1e-6) / 1e9, 1)
+            v["hbm_frac"] = round(v["hbm_gbs"] / hbm, 4)
+            if "flop" in v:
+                v["tflops"] = round(v["flop"] / (v["us"] * 1e-6) / 1e12, 1)
+            v["us"] = round(v["us"], 2)
+        dom_name = max(kern, key=lambda n: kern[n]["us"])
+        dom = kern[dom_name]
+        tr = TRAFFIC.get(args.config, {})
+        traffic = None
+        if tr.get("bytes_per_launch") and tr.get("src_sha") == src_sha(
+                "sparse_attention_07_b200/csrc/" + tr.get("kernel", "")) and dom_name == "attn":
+            traffic = tr["bytes_per_launch"]
         if prefill:
-            fi, fm = prefill_flops(cfg)
-            fp8_peak = bf16_burst * 2.0  # fp8 dense rate = 2x bf16 (nominal ratio)
-            ach = fi / (first * 1e-3) / 1e12
-            roof = {"bound": "tensor", "achieved": round(ach, 1), "peak": fp8_peak, "unit": "TFLOP/s",
-                    "frac": round(ach / fp8_peak, 4), "traffic": None,
-                    "kernel": "idx_tc_kernel (fp8 kind::f8f6f4)",
-                    "peak_source": f"{peak_src} bf16 burst x 2 (nominal fp8/bf16 ratio)"}
+            # both big kernels are contractions: the roofline is the tensor pipe
+            peak = dom["flop_peak"]
+            roof = {"bound": "tensor", "achieved": dom["tflops"], "peak": peak, "unit": "TFLOP/s",
+                    "frac": round(dom["tflops"] / peak, 4), "traffic": traffic, "kernel": dom["kernel"],
+                    "peak_source": (f"{peak_src} bf16 sustained x 2 (nominal fp8/bf16 ratio)"
+                                    if dom_name == "indexer" else f"{peak_src} bf16 sustained")}
         else:
-            ach = keys_b / (first * 1e-3) / 1e9
-            tr = TRAFFIC.get(args.config, {})
-            traffic = tr.get("bytes_per_launch") if tr.get("src_sha") == src_sha(
-                "sparse_attention_07_b200/csrc/index_scores.cu") else None
-            roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": hbm, "unit": "GB/s",
-                    "frac": round(ach / hbm, 4), "traffic": traffic,
-                    "kernel": "idx_tc_kernel" if cfg.idx_dtype == "e4m3" else "idx_cc_kernel",
+            roof = {"bound": "hbm", "achieved": dom["hbm_gbs"], "peak": hbm, "unit": "GB/s",
+                    "frac": dom["hbm_frac"], "traffic": traffic, "kernel": dom["kernel"],
                     "peak_source": f"{peak_src} hbm_gbs"}
+        for v in kern.values():
+            v.pop("flop_peak", None)
         step_gbs = (keys_b + rows_b) / (ms * 1e-3) / 1e9
         res["step_roofline"] = {"bytes_per_step": keys_b + rows_b, "indexer_key_bytes": keys_b,
                                 "gathered_row_bytes": rows_b, "achieved": round(step_gbs, 1), "peak": hbm,
                                 "unit": "GB/s", "frac": round(step_gbs / hbm, 4)}
+        res["kernels"] = kern
     else:
         units = cfg.B * ws
         unit = "queries/s"

@@ -102,6 +102,24 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t* b, uint32_t parity) {
     return ok != 0;
 }
 
+__device__ __forceinline__ bool mbar_test_wait_acq_cluster(uint64_t* b, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(b)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Arrive on an mbarrier of a CTA of the cluster without ordering this thread's
+// earlier memory accesses (for "I have finished reading" signals whose reads
+// have already returned their values).
+__device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
 // Context for bounded waits: the device error word and the CTA's abort flag.
 struct WaitCtx {
     int* err;             // global error word (may be null)
