@@ -453,6 +453,88 @@ def run_native(args):
         torch.distributed.destroy_process_group()
 
 
+# history lengths of the dual-mode measurement (long-decode shapes otherwise)
+CROSSOVER_L = (1024, 2048, 3072, 4096, 6144, 8192, 12288, 16384)
+
+
+def run_crossover(args):
+    """Short-sequence mode vs DSA: the step time of the DSA path (indexer ->
+    Top-K -> sparse MLA) and of dense MLA over every visible position, for the
+    long-decode shapes at growing history lengths; `value` is the length above
+    which DSA is faster (linear interpolation between measured lengths)."""
+    ws, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    import sparse_attention_07_b200 as sa
+    sa.lib()
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    table = []
+    launches = 0
+    for L in CROSSOVER_L:
+        cfg = W.small_dsa(W.LONG, lens=(L,) * W.LONG.n_seqs)
+        inp = W.dsa_inputs(cfg, dev, seed=rank_seed(cfg.seed + L, rank))
+        dsa = DecodeStep(inp, sa)
+        nv = inp["n_visible"]
+        out = torch.empty(cfg.rows, cfg.H, cfg.d_c, dtype=torch.float32, device=dev)
+        wsd = torch.empty(sa.dense_mla_workspace_size(cfg.rows, cfg.H, L, cfg.d_c), dtype=torch.uint8, device=dev)
+
+        def dense():
+            sa.dense_mla_decode(inp["q_lat"], inp["q_rope"], inp["c_cache"], inp["kr_cache"], nv, L, cfg.scale,
+                                cfg.pages_per_seq, page_table=inp["page_table"], out=out, workspace=wsd)
+
+        def time_fn(fn):
+            for _ in range(args.warmup):
+                flush.zero_()
+                fn()
+            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(args.steps)]
+            for a, b in ev:
+                flush.zero_()
+                a.record()
+                fn()
+                b.record()
+            torch.cuda.synchronize()
+            return statistics.mean(a.elapsed_time(b) for a, b in ev)
+
+        t_dsa = time_fn(lambda: (dsa.indexer(), dsa.rest()))
+        t_dense = time_fn(dense)
+        launches += args.steps * (dsa.launches_per_step + 1 + (1 if sa.dense_mla_workspace_size(
+            cfg.rows, cfg.H, L, cfg.d_c) > 0 else 0))
+        table.append({"L": L, "dsa_us": round(t_dsa * 1e3, 2), "dense_us": round(t_dense * 1e3, 2)})
+        del inp, dsa, wsd
+        torch.cuda.empty_cache()
+    if sa.check_device_error() != 0:
+        raise RuntimeError("device error word set")
+    cross = None
+    for a, b in zip(table, table[1:]):
+        da, db = a["dsa_us"] - a["dense_us"], b["dsa_us"] - b["dense_us"]
+        if da >= 0 > db:
+            cross = round(a["L"] + (b["L"] - a["L"]) * da / (da - db))
+            break
+    if cross is None and table and table[0]["dsa_us"] < table[0]["dense_us"]:
+        cross = table[0]["L"]
+    hbm, _, _, peak_src = peaks()
+    last = table[-1]
+    dense_bytes = W.LONG.n_seqs * last["L"] * (W.LONG.d_c + W.LONG.d_R) * 2
+    ach = dense_bytes / (last["dense_us"] * 1e-6) / 1e9
+    res = {
+        "impl": "native", "metric": "DSA vs dense MLA decode crossover (history length above which DSA is faster)",
+        "value": cross, "unit": "tokens", "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": None, "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
+        "dtype": "e4m3 indexer / bf16 MLA, fp32 accumulate", "data": "synthetic (seeded)",
+        "config": {"workload": "long-decode shapes (32 queries, H^I=64 e4m3, top-2048, 128-head MLA) at history "
+                               "lengths " + ",".join(str(x) for x in CROSSOVER_L),
+                   "l2": f"flushed between steps ({L2_FLUSH_BYTES >> 20} MiB write, outside the events)"},
+        "crossover": table,
+        "roofline": {"bound": "hbm", "achieved": round(ach, 1), "peak": hbm, "unit": "GB/s", "frac": round(ach / hbm, 4),
+                     "traffic": None, "kernel": f"mla_kernel, dense mode at L={last['L']}",
+                     "peak_source": f"{peak_src} hbm_gbs"},
+        "e2e": None, "gpu_launches": launches,
+    }
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+
+
 def run_reference(args):
     """The oracle as the reference arm, timed on the host cores."""
     ws, rank, local = dist_env()
@@ -507,12 +589,19 @@ def main(argv=None):
     p.add_argument("--steps", type=int, default=200)
     p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--impl", choices=["native", "reference"], default="native")
-    p.add_argument("--config", default="long", choices=sorted(list(W.DSA_CONFIGS) + list(W.BLOCK_CONFIGS)))
+    p.add_argument("--config", default="long",
+                   choices=sorted(list(W.DSA_CONFIGS) + list(W.BLOCK_CONFIGS) + ["crossover"]))
     p.add_argument("--no-cpu-baseline", action="store_true")
     args = p.parse_args(argv)
     if args.warmup < 3 and args.impl == "native":
         args.warmup = 3
-    if args.impl == "reference":
+    if args.config == "crossover":
+        if args.impl == "reference":
+            print(json.dumps({"impl": "reference", "unavailable": "the crossover mode times two GPU paths; "
+                              "the oracle arm covers the workload configs"}), flush=True)
+        else:
+            run_crossover(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_native(args)

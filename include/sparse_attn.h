@@ -174,6 +174,26 @@ sa_status sa_sparse_mla_prefill(const void* q_lat, const void* q_rope,
                                 sa_stream_t stream);
 
 /*
+ * Dense MLA decode: the same attention as sa_sparse_mla_decode over every
+ * visible position instead of a selection (row r attends to positions
+ * 0 .. n_visible[r]-1 of its sequence).  It is the short-sequence mode of the
+ * dual-mode system of [LLMRes] "DeepSeek Sparse Attention (DSA)": below a few
+ * thousand tokens the indexer and Top-K cost more than attending to every
+ * position, so the caller runs this call without either of them.
+ *   n_visible [rows] int32, each <= L_max and inside the page table;
+ *   workspace: sa_dense_mla_workspace_size(rows, H, L_max, d_c) bytes.
+ * Other arguments, layouts, limits and errors as sa_sparse_mla_decode.
+ */
+size_t sa_dense_mla_workspace_size(int rows, int H, int L_max, int d_c);
+
+sa_status sa_dense_mla_decode(const void* q_lat, const void* q_rope,
+                              const void* c_cache, int64_t c_ld, const void* kr_cache, int64_t kr_ld,
+                              int64_t pool_pages, const int32_t* page_table, int pages_per_seq,
+                              const int32_t* seq_of_row, const int32_t* n_visible, int rows, int H, int L_max,
+                              int d_c, int d_R, float scale, float* out, float* lse, void* workspace,
+                              size_t workspace_bytes, sa_stream_t stream);
+
+/*
  * Sparse MLA decode for callers that cannot allocate device memory.  The
  * pages have no counterpart of this call: it is a deployment convenience.
  *

@@ -28,6 +28,7 @@ EXPORTS = (
     "sa_sparse_mla_workspace_size", "sa_sparse_mla_prefill_workspace_size", "sa_sparse_mla_decode",
     "sa_sparse_mla_prefill",
     "sa_block_mean_pool", "sa_block_sparse_attn", "sa_sparse_mla_decode_static",
+    "sa_dense_mla_workspace_size", "sa_dense_mla_decode",
 )
 
 # Size of the library's static device array behind sparse_mla_decode_static
@@ -62,12 +63,15 @@ def lib():
         L.sa_sparse_mla_prefill_workspace_size.restype = SZ
         L.sa_sparse_mla_prefill_workspace_size.argtypes = [I, I, I, I]
         L.sa_sparse_mla_prefill.argtypes = [P, P, P, I64, P, I64, I64, P, I, P, P, I, I, I, I, I, F, P, P, P, SZ, P]
+        L.sa_dense_mla_workspace_size.restype = SZ
+        L.sa_dense_mla_workspace_size.argtypes = [I, I, I, I]
+        L.sa_dense_mla_decode.argtypes = [P, P, P, I64, P, I64, I64, P, I, P, P, I, I, I, I, I, F, P, P, P, SZ, P]
         L.sa_sparse_mla_decode_static.argtypes = [P, P, P, I64, P, I64, I64, P, I, P, P, I, I, I, I, I, F, P, P, P]
         L.sa_block_mean_pool.argtypes = [P, I64, I64, I64, I, I, I, I, I, P, I64, P]
         L.sa_block_sparse_attn.argtypes = [P, P, I64, P, P, I64, I64, I64, I, I, I, I, I, I, I, I, F, P, P, P]
         for name in EXPORTS:
             if name not in ("sa_status_string", "sa_version", "sa_sparse_mla_workspace_size",
-                            "sa_sparse_mla_prefill_workspace_size"):
+                            "sa_sparse_mla_prefill_workspace_size", "sa_dense_mla_workspace_size"):
                 getattr(L, name).restype = I
         _lib = L
     return _lib
@@ -174,6 +178,31 @@ def sparse_mla_prefill(q_lat, q_rope, c_cache, kr_cache, idx, scale: float, page
                                      _p(idx), rows, H, k, d_c, d_R, float(scale), _p(out), _p(lse), _p(workspace),
                                      wbytes, _stream())
     _check("sa_sparse_mla_prefill", st)
+    return out
+
+
+def dense_mla_workspace_size(rows: int, H: int, L_max: int, d_c: int = 512) -> int:
+    return int(lib().sa_dense_mla_workspace_size(rows, H, L_max, d_c))
+
+
+def dense_mla_decode(q_lat, q_rope, c_cache, kr_cache, n_visible, L_max: int, scale: float, pages_per_seq: int,
+                     page_table=None, seq_of_row=None, out=None, lse=None, workspace=None):
+    """Dense MLA over every visible position (the short-sequence mode): row r
+    attends to positions 0 .. n_visible[r]-1.  [rows, H, d_c] fp32."""
+    rows, H, d_c = q_lat.shape
+    d_R = q_rope.shape[2]
+    if out is None:
+        out = torch.empty(rows, H, d_c, dtype=torch.float32, device=q_lat.device)
+    pool_pages = c_cache.shape[0] // 64
+    if workspace is None and rows > 0:
+        workspace = torch.empty(dense_mla_workspace_size(rows, H, L_max, d_c), dtype=torch.uint8,
+                                device=q_lat.device)
+    wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib().sa_dense_mla_decode(_p(q_lat), _p(q_rope), _p(c_cache), c_cache.stride(0), _p(kr_cache),
+                                   kr_cache.stride(0), pool_pages, _p(page_table), pages_per_seq, _p(seq_of_row),
+                                   _p(n_visible), rows, H, L_max, d_c, d_R, float(scale), _p(out), _p(lse),
+                                   _p(workspace), wbytes, _stream())
+    _check("sa_dense_mla_decode", st)
     return out
 
 

@@ -169,11 +169,11 @@ static sa_status mla_common(const void* q_lat, const void* q_rope, const void* c
                             int pages_per_seq, const int32_t* seq_of_row, const int32_t* idx, int rows, int H, int k,
                             int d_c, int d_R, float scale, float* out, float* lse, MlaArgs* a) {
     if (rows < 0 || H < 1 || k < 1 || pages_per_seq < 1 || pool_pages < 1 || !std::isfinite(scale)) return SA_EINVAL;
-    if (!q_lat || !q_rope || !c_cache || !kr_cache || !idx || !out) return SA_EINVAL;
+    if (!q_lat || !q_rope || !c_cache || !kr_cache || !out) return SA_EINVAL;
     if (d_c != 512 || d_R != 64 || H > 128) return SA_EUNSUPPORTED;
     if (c_ld < d_c || kr_ld < d_R || c_ld % 8 != 0 || kr_ld % 8 != 0) return SA_EINVAL;
     if (!aligned(q_lat, 16) || !aligned(q_rope, 16) || !aligned(c_cache, 16) || !aligned(kr_cache, 16) ||
-        !aligned(out, 16) || !aligned(idx, 4) || (lse && !aligned(lse, 4)))
+        !aligned(out, 16) || (idx && !aligned(idx, 4)) || (lse && !aligned(lse, 4)))
         return SA_EINVAL;
     if (pool_pages * 64 > (int64_t(1) << 31)) return SA_EUNSUPPORTED;
     a->q_lat = q_lat;
@@ -187,6 +187,7 @@ static sa_status mla_common(const void* q_lat, const void* q_rope, const void* c
     a->pool_pages = pool_pages;
     a->seq_of_row = seq_of_row;
     a->idx = idx;
+    a->n_visible = nullptr;
     a->rows = rows;
     a->H = H;
     a->k = k;
@@ -205,6 +206,7 @@ sa_status sa_sparse_mla_decode(const void* q_lat, const void* q_rope, const void
                                int k, int d_c, int d_R, float scale, float* out, float* lse, void* workspace,
                                size_t workspace_bytes, sa_stream_t stream) {
     if (rows == 0) return SA_OK;
+    if (!idx) return SA_EINVAL;
     MlaArgs a;
     sa_status s = mla_common(q_lat, q_rope, c_cache, c_ld, kr_cache, kr_ld, pool_pages, page_table, pages_per_seq,
                              seq_of_row, idx, rows, H, k, d_c, d_R, scale, out, lse, &a);
@@ -226,6 +228,7 @@ sa_status sa_sparse_mla_prefill(const void* q_lat, const void* q_rope, const voi
                                 int k, int d_c, int d_R, float scale, float* out, float* lse, void* workspace,
                                 size_t workspace_bytes, sa_stream_t stream) {
     if (rows == 0) return SA_OK;
+    if (!idx) return SA_EINVAL;
     MlaArgs a;
     sa_status s = mla_common(q_lat, q_rope, c_cache, c_ld, kr_cache, kr_ld, pool_pages, page_table, pages_per_seq,
                              seq_of_row, idx, rows, H, k, d_c, d_R, scale, out, lse, &a);
@@ -234,6 +237,28 @@ sa_status sa_sparse_mla_prefill(const void* q_lat, const void* q_rope, const voi
     if (!workspace || !aligned(workspace, 256) || workspace_bytes < mla_workspace_bytes(rows, H, k, d_c, 1))
         return SA_EINVAL;
     return sparse_mla_launch(a, 1, workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t sa_dense_mla_workspace_size(int rows, int H, int L_max, int d_c) {
+    return sa_sparse_mla_workspace_size(rows, H, L_max, d_c);
+}
+
+sa_status sa_dense_mla_decode(const void* q_lat, const void* q_rope, const void* c_cache, int64_t c_ld,
+                              const void* kr_cache, int64_t kr_ld, int64_t pool_pages, const int32_t* page_table,
+                              int pages_per_seq, const int32_t* seq_of_row, const int32_t* n_visible, int rows,
+                              int H, int L_max, int d_c, int d_R, float scale, float* out, float* lse,
+                              void* workspace, size_t workspace_bytes, sa_stream_t stream) {
+    if (rows == 0) return SA_OK;
+    if (!n_visible || !aligned(n_visible, 4)) return SA_EINVAL;
+    MlaArgs a;
+    sa_status s = mla_common(q_lat, q_rope, c_cache, c_ld, kr_cache, kr_ld, pool_pages, page_table, pages_per_seq,
+                             seq_of_row, nullptr, rows, H, L_max, d_c, d_R, scale, out, lse, &a);
+    if (s != SA_OK) return s;
+    a.n_visible = n_visible;
+    const int ns = mla_decode_splits(rows, L_max);
+    if (!workspace || !aligned(workspace, 256) || workspace_bytes < mla_workspace_bytes(rows, H, L_max, d_c, ns))
+        return SA_EINVAL;
+    return sparse_mla_launch(a, ns, workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"
@@ -271,6 +296,7 @@ sa_status sa_sparse_mla_decode_static(const void* q_lat, const void* q_rope, con
                                       const int32_t* idx, int rows, int H, int k, int d_c, int d_R, float scale,
                                       float* out, float* lse, sa_stream_t stream) {
     if (rows == 0) return SA_OK;
+    if (!idx) return SA_EINVAL;
     MlaArgs a;
     sa_status s = mla_common(q_lat, q_rope, c_cache, c_ld, kr_cache, kr_ld, pool_pages, page_table, pages_per_seq,
                              seq_of_row, idx, rows, H, k, d_c, d_R, scale, out, lse, &a);

@@ -51,7 +51,8 @@ struct MlaArgs {
     int pages_per_seq;
     int64_t pool_pages;
     const int32_t* seq_of_row;
-    const int32_t* idx;
+    const int32_t* idx;        // [rows][k] selected positions; null: dense mode
+    const int32_t* n_visible;  // dense mode: row r attends to positions 0 .. n_visible[r]-1
     int rows, H, k, d_c, d_R;
     float scale;
     float* out;

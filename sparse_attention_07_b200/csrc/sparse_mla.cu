@@ -90,8 +90,12 @@ __device__ __forceinline__ int64_t pool_row(const MlaArgs& a, int seq, int p) {
     return static_cast<int64_t>(pg) * kPage + (p % kPage);
 }
 
+// Position held by slot `slot` of row r: the selection, or in dense mode (no
+// selection) every visible position in order.
 __device__ __forceinline__ int idx_at(const MlaArgs& a, int r, int slot) {
-    return slot < a.k ? a.idx[static_cast<int64_t>(r) * a.k + slot] : -1;
+    if (slot >= a.k) return -1;
+    if (a.idx) return a.idx[static_cast<int64_t>(r) * a.k + slot];
+    return slot < a.n_visible[r] ? slot : -1;
 }
 
 template <int N>
