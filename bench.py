@@ -246,6 +246,39 @@ def time_steps(step, K: int, flush):
             [[e[j].elapsed_time(e[j + 1]) for e in ev] for j in range(3)])
 
 
+def time_projections(step, K: int, flush, hbm: float):
+    """The per-head projections around sparse MLA (query absorption with U_K,
+    up-projection with U_V), timed on their own with synthetic weights of the
+    workload's shapes (d_C=128, d_v=128): outside the metric's step, which
+    starts from the absorbed query and ends at the latent output."""
+    import sparse_attention_07_b200 as sa
+    cfg, dev = step.cfg, step.out.device
+    g = torch.Generator(device=dev)
+    g.manual_seed(cfg.seed + 77)
+    q_c = (torch.randn(cfg.rows, cfg.H, cfg.d_C, generator=g, device=dev)).to(torch.bfloat16)
+    U_K = (torch.randn(cfg.H, cfg.d_C, cfg.d_c, generator=g, device=dev) / cfg.d_C ** 0.5).to(torch.bfloat16)
+    U_V = (torch.randn(cfg.H, 128, cfg.d_c, generator=g, device=dev) / cfg.d_c ** 0.5).to(torch.bfloat16)
+    q_lat = torch.empty(cfg.rows, cfg.H, cfg.d_c, dtype=torch.bfloat16, device=dev)
+    out = torch.empty(cfg.rows, cfg.H, 128, dtype=torch.float32, device=dev)
+    res = {}
+    for name, fn, w in (("absorb", lambda: sa.mla_absorb_query(q_c, U_K, q_lat=q_lat), U_K),
+                        ("up_project", lambda: sa.mla_up_project(step.out, U_V, out=out), U_V)):
+        for _ in range(3):
+            fn()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+        for a, b in ev:
+            flush.zero_()
+            a.record()
+            fn()
+            b.record()
+        torch.cuda.synchronize()
+        us = statistics.mean(a.elapsed_time(b) for a, b in ev) * 1e3
+        nbytes = w.numel() * 2  # the weights are read once; the activations are a few hundred KB
+        res[name] = {"kernel": "head_gemm_kernel", "us": round(us, 2), "weight_bytes": nbytes,
+                     "hbm_gbs": round(nbytes / (us * 1e-6) / 1e9, 1), "hbm_frac": round(nbytes / (us * 1e-6) / 1e9 / hbm, 4)}
+    return res
+
+
 def e2e_steps(step, K: int, flush):
     """Same step through the public API with the step's query inputs copied in
     from pinned host memory and the output read back, inside the events."""
@@ -421,6 +454,8 @@ def run_native(args):
                                 "gathered_row_bytes": rows_b, "achieved": round(step_gbs, 1), "peak": hbm,
                                 "unit": "GB/s", "frac": round(step_gbs / hbm, 4)}
         res["kernels"] = kern
+        if not prefill:
+            res["projections"] = time_projections(step, min(args.steps, 20), flush, hbm)
     else:
         units = cfg.B * ws
         unit = "queries/s"

@@ -194,6 +194,25 @@ sa_status sa_dense_mla_decode(const void* q_lat, const void* q_rope,
                               size_t workspace_bytes, sa_stream_t stream);
 
 /*
+ * The per-head projections around sparse MLA ([MLA-S] "“吸收矩阵”是交换线性计算的
+ * 顺序": q^C . (U_K c_j) = (U_K^T q^C) . c_j, so the query is absorbed once and
+ * the output stays in latent space until one up-projection):
+ *   q_lat[r][h][j] = sum_i U_K[h][i][j] * q_c[r][h][i]    (the absorbed query)
+ *   out[r][h][v]   = sum_j U_V[h][v][j] * o_lat[r][h][j]  (value-space output)
+ *   q_c [rows][H][d_C] bf16, U_K [H][d_C][d_c] bf16 (k^C = U_K c), q_lat [rows][H][d_c] bf16 out;
+ *   o_lat [rows][H][d_c] fp32 (the sparse-MLA output), U_V [H][d_v][d_c] bf16, out [rows][H][d_v] fp32.
+ * bf16 operands (o_lat is rounded to bf16), fp32 accumulation on the tensor
+ * cores.  Supported: absorption d_C a multiple of 64 up to 512 and d_c a
+ * multiple of 128 up to 512; up-projection d_c a multiple of 64 up to 512 and
+ * d_v a multiple of 128.  Alignment: q_c, U_K, o_lat, U_V 16 bytes.
+ */
+sa_status sa_mla_absorb_query(const void* q_c, const void* U_K, int rows, int H, int d_C, int d_c, void* q_lat,
+                              sa_stream_t stream);
+
+sa_status sa_mla_up_project(const float* o_lat, const void* U_V, int rows, int H, int d_c, int d_v, float* out,
+                            sa_stream_t stream);
+
+/*
  * Sparse MLA decode for callers that cannot allocate device memory.  The
  * pages have no counterpart of this call: it is a deployment convenience.
  *

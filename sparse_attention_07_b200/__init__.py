@@ -28,7 +28,7 @@ EXPORTS = (
     "sa_sparse_mla_workspace_size", "sa_sparse_mla_prefill_workspace_size", "sa_sparse_mla_decode",
     "sa_sparse_mla_prefill",
     "sa_block_mean_pool", "sa_block_sparse_attn", "sa_sparse_mla_decode_static",
-    "sa_dense_mla_workspace_size", "sa_dense_mla_decode",
+    "sa_dense_mla_workspace_size", "sa_dense_mla_decode", "sa_mla_absorb_query", "sa_mla_up_project",
 )
 
 # Size of the library's static device array behind sparse_mla_decode_static
@@ -66,6 +66,8 @@ def lib():
         L.sa_dense_mla_workspace_size.restype = SZ
         L.sa_dense_mla_workspace_size.argtypes = [I, I, I, I]
         L.sa_dense_mla_decode.argtypes = [P, P, P, I64, P, I64, I64, P, I, P, P, I, I, I, I, I, F, P, P, P, SZ, P]
+        L.sa_mla_absorb_query.argtypes = [P, P, I, I, I, I, P, P]
+        L.sa_mla_up_project.argtypes = [P, P, I, I, I, I, P, P]
         L.sa_sparse_mla_decode_static.argtypes = [P, P, P, I64, P, I64, I64, P, I, P, P, I, I, I, I, I, F, P, P, P]
         L.sa_block_mean_pool.argtypes = [P, I64, I64, I64, I, I, I, I, I, P, I64, P]
         L.sa_block_sparse_attn.argtypes = [P, P, I64, P, P, I64, I64, I64, I, I, I, I, I, I, I, I, F, P, P, P]
@@ -203,6 +205,26 @@ def dense_mla_decode(q_lat, q_rope, c_cache, kr_cache, n_visible, L_max: int, sc
                                    _p(n_visible), rows, H, L_max, d_c, d_R, float(scale), _p(out), _p(lse),
                                    _p(workspace), wbytes, _stream())
     _check("sa_dense_mla_decode", st)
+    return out
+
+
+def mla_absorb_query(q_c, U_K, q_lat=None):
+    """q_lat[r,h,:] = U_K[h]^T q_c[r,h,:]: q_c [rows,H,d_C] bf16, U_K [H,d_C,d_c] bf16 -> [rows,H,d_c] bf16."""
+    rows, H, d_C = q_c.shape
+    d_c = U_K.shape[2]
+    if q_lat is None:
+        q_lat = torch.empty(rows, H, d_c, dtype=torch.bfloat16, device=q_c.device)
+    _check("sa_mla_absorb_query", lib().sa_mla_absorb_query(_p(q_c), _p(U_K), rows, H, d_C, d_c, _p(q_lat), _stream()))
+    return q_lat
+
+
+def mla_up_project(o_lat, U_V, out=None):
+    """out[r,h,:] = U_V[h] o_lat[r,h,:]: o_lat [rows,H,d_c] fp32, U_V [H,d_v,d_c] bf16 -> [rows,H,d_v] fp32."""
+    rows, H, d_c = o_lat.shape
+    d_v = U_V.shape[1]
+    if out is None:
+        out = torch.empty(rows, H, d_v, dtype=torch.float32, device=o_lat.device)
+    _check("sa_mla_up_project", lib().sa_mla_up_project(_p(o_lat), _p(U_V), rows, H, d_c, d_v, _p(out), _stream()))
     return out
 
 

@@ -309,6 +309,28 @@ sa_status sa_sparse_mla_decode_static(const void* q_lat, const void* q_rope, con
     return sparse_mla_launch(a, ns, ws, SA_STATIC_SCRATCH_BYTES, reinterpret_cast<cudaStream_t>(stream));
 }
 
+sa_status sa_mla_absorb_query(const void* q_c, const void* U_K, int rows, int H, int d_C, int d_c, void* q_lat,
+                              sa_stream_t stream) {
+    if (rows < 0 || H < 1 || d_C < 1 || d_c < 1) return SA_EINVAL;
+    if (rows == 0) return SA_OK;
+    if (!q_c || !U_K || !q_lat) return SA_EINVAL;
+    if (d_C % 64 != 0 || d_C > 512 || d_c % 128 != 0 || d_c > 512 || H > 65535) return SA_EUNSUPPORTED;
+    if (!aligned(q_c, 16) || !aligned(U_K, 16) || !aligned(q_lat, 2)) return SA_EINVAL;
+    return mla_absorb_query_launch(q_c, U_K, rows, H, d_C, d_c, q_lat, device_error_word(),
+                                   reinterpret_cast<cudaStream_t>(stream));
+}
+
+sa_status sa_mla_up_project(const float* o_lat, const void* U_V, int rows, int H, int d_c, int d_v, float* out,
+                            sa_stream_t stream) {
+    if (rows < 0 || H < 1 || d_c < 1 || d_v < 1) return SA_EINVAL;
+    if (rows == 0) return SA_OK;
+    if (!o_lat || !U_V || !out) return SA_EINVAL;
+    if (d_c % 64 != 0 || d_c > 512 || d_v % 128 != 0 || H > 65535) return SA_EUNSUPPORTED;
+    if (!aligned(o_lat, 16) || !aligned(U_V, 16) || !aligned(out, 4)) return SA_EINVAL;
+    return mla_up_project_launch(o_lat, U_V, rows, H, d_c, d_v, out, device_error_word(),
+                                 reinterpret_cast<cudaStream_t>(stream));
+}
+
 sa_status sa_block_mean_pool(const void* K, int64_t stride_b, int64_t stride_t, int64_t stride_h, int B, int L,
                              int H, int D, int block, float* pooled, int64_t pooled_ld, sa_stream_t stream) {
     if (B < 0 || L < 0 || H < 0 || block < 1) return SA_EINVAL;

@@ -23,7 +23,8 @@ enum : int {
     kErrIdxWait = 0x100,   // indexer kernel waits (low byte = role/site)
     kErrMlaWait = 0x200,   // sparse-MLA kernel waits
     kErrTopkRow = 0x300,   // top-k: invalid row state
-    kErrMixedGroup = 0x400 // indexer: internal grouping inconsistency
+    kErrMixedGroup = 0x400,  // indexer: internal grouping inconsistency
+    kErrGemmWait = 0x500     // per-head projection GEMM waits
 };
 
 constexpr unsigned long long kWaitLimitNs = 1000ull * 1000ull * 1000ull;  // 1 s

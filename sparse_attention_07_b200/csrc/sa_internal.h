@@ -73,6 +73,11 @@ size_t mla_workspace_bytes(int rows, int H, int k, int d_c, int nsplit);
 int mla_decode_splits(int rows, int k);
 sa_status sparse_mla_launch(const MlaArgs& a, int nsplit, void* ws, size_t ws_bytes, cudaStream_t st);
 
+sa_status mla_absorb_query_launch(const void* q_c, const void* U_K, int rows, int H, int d_C, int d_c, void* q_lat,
+                                  int* err, cudaStream_t st);
+sa_status mla_up_project_launch(const float* o_lat, const void* U_V, int rows, int H, int d_c, int d_v, float* out,
+                                int* err, cudaStream_t st);
+
 sa_status block_mean_pool_launch(const void* K, int64_t sb, int64_t st_, int64_t sh, int B, int L, int H, int D,
                                  int block, float* pooled, int64_t pooled_ld, cudaStream_t st);
 sa_status block_sparse_launch(const void* q, const float* pooled, int64_t pooled_ld, const void* K, const void* V,
