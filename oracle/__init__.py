@@ -222,6 +222,100 @@ def error_bound(v_max: float, Z: float) -> float:
 
 
 # --------------------------------------------------------------------------
+# NSA three-branch decode ([MLA-S] "三条路径，各留住什么？" and "选块和合并输出，
+# 实际算一遍"; [LLMRes] NSA steps 1-3).  Compression is the mean of each
+# complete block of keys and of values (the pages' learned per-block transform
+# has no weights here; [Ch11] §12.6 pools by the mean).
+
+def shared_block_choice(head_probabilities, count: int):
+    """[MLA-S] shared_block_choice: the heads that share a KV head add their
+    block probabilities and keep the `count` best blocks, ties to the lower
+    block index.  Returns the chosen block indices in rank order."""
+    p = _f64(head_probabilities)
+    if p.ndim != 2 or p.shape[1] == 0:
+        raise ValueError("expected nonempty head distributions")
+    if not 1 <= count <= p.shape[1]:
+        raise ValueError("invalid selection count")
+    totals = p.sum(axis=0)
+    return sorted(range(p.shape[1]), key=lambda i: (-totals[i], i))[:count]
+
+
+def nsa_select_scores(p_cmp, l: int, d: int, l_sel: int):
+    """[MLA-S] NSA §3.3 aggregation of compression probabilities into selection
+    block scores: p_sel[j] = sum_{u < l'/d} sum_{v < l/d} p_cmp[(l'/d) j + u + v]
+    for compression blocks of length l and stride d and selection blocks of
+    length l' (d divides both); terms past the end of p_cmp are absent."""
+    p = _f64(p_cmp)
+    if l % d or l_sel % d:
+        raise ValueError("the stride must divide both block lengths")
+    a, b = l_sel // d, l // d
+    n_sel = (len(p) + a - 1) // a if len(p) else 0
+    out = np.zeros(n_sel)
+    for j in range(n_sel):
+        for u in range(a):
+            for v in range(b):
+                i = a * j + u + v
+                if i < len(p):
+                    out[j] += p[i]
+    return out
+
+
+def nsa_combine(o_cmp, o_sel, o_win, gates):
+    """[MLA-S] g_c o_c + g_s o_s + g_w o_w with independent (sigmoid) gates:
+    the gates are not normalised to sum to one."""
+    g = _f64(gates)
+    return g[0] * _f64(o_cmp) + g[1] * _f64(o_sel) + g[2] * _f64(o_win)
+
+
+def _softmax_attend(q, K, V, scale):
+    s = K @ q * scale
+    a = np.exp(s - s.max())
+    a /= a.sum()
+    return a @ V, a
+
+
+def nsa_decode_group(q, K, V, block: int, top_blocks: int, window: int, gates, scale: float, chosen=None):
+    """One decode query per head of a GQA group sharing one KV head.
+
+    q [G, D], K/V [L, D] (the history; the query sees all L positions), gates
+    [G, 3] (compression, selection, window).  Branches, each with its own
+    softmax:
+      compression: the complete blocks n < L // block, key mean(K_block) and
+        value mean(V_block) (no block holding a position >= L is formed);
+      selection: the heads' compression probabilities summed over the group
+        pick min(top_blocks, n_blocks) blocks (ties to the lower index); every
+        head attends to all tokens of those blocks;
+      window: the last `window` positions.
+    A branch with no position (no complete block) contributes zero.
+    `chosen` (block indices) replaces the group's own choice when given: it
+    evaluates the branches on another valid choice among near-tied blocks.
+    Returns (out [G, D], chosen blocks ascending, p_cmp [G, n_blocks])."""
+    q, K, V, g = _f64(q), _f64(K), _f64(V), _f64(gates)
+    G, D = q.shape
+    L = K.shape[0]
+    nb = L // block
+    kbar = K[: nb * block].reshape(nb, block, D).mean(axis=1) if nb else np.zeros((0, D))
+    vbar = V[: nb * block].reshape(nb, block, D).mean(axis=1) if nb else np.zeros((0, D))
+    p_cmp = np.zeros((G, nb))
+    o_cmp = np.zeros((G, D))
+    for h in range(G):
+        if nb:
+            o_cmp[h], p_cmp[h] = _softmax_attend(q[h], kbar, vbar, scale)
+    if chosen is None:
+        chosen = sorted(shared_block_choice(p_cmp, min(top_blocks, nb))) if nb and top_blocks > 0 else []
+    else:
+        chosen = sorted(int(c) for c in chosen)
+    tokens = np.concatenate([np.arange(b * block, (b + 1) * block) for b in chosen]) if chosen else None
+    w0 = max(0, L - window)
+    out = np.zeros((G, D))
+    for h in range(G):
+        o_sel = _softmax_attend(q[h], K[tokens], V[tokens], scale)[0] if tokens is not None else np.zeros(D)
+        o_win = _softmax_attend(q[h], K[w0:], V[w0:], scale)[0] if window > 0 and L > 0 else np.zeros(D)
+        out[h] = nsa_combine(o_cmp[h], o_sel, o_win, g[h])
+    return out, np.asarray(chosen, dtype=np.int64), p_cmp
+
+
+# --------------------------------------------------------------------------
 # Whole-step reference on workload tensors (any device; values copied to host)
 
 def _host64(t):
@@ -301,3 +395,17 @@ def block_step(inp: dict, pairs: Sequence[tuple]) -> dict:
         o, s, bs = block_sparse(q, K, V, cfg.block, cfg.top_blocks, cfg.sink_blocks, cfg.window, cfg.scale)
         outs.append(o); sels.append(s); scores.append(bs)
     return dict(out=np.stack(outs), sel=np.stack(sels), block_scores=np.stack(scores))
+
+
+def nsa_step(inp: dict, pairs: Sequence[tuple]) -> dict:
+    """nsa_decode_group on workload tensors for (sequence b, KV head g) pairs:
+    q [B, H, D], K and V [B, L, H_kv, D], gates [B, H, 3]; query heads
+    g*G .. g*G+G-1 share KV head g (G = H / H_kv)."""
+    cfg = inp["cfg"]
+    G = cfg.H // cfg.H_kv
+    res = {}
+    for b, g in pairs:
+        hs = slice(g * G, (g + 1) * G)
+        res[(b, g)] = nsa_decode_group(_host64(inp["q"][b, hs]), _host64(inp["K"][b, :, g]), _host64(inp["V"][b, :, g]),
+                                       cfg.block, cfg.top_blocks, cfg.window, _host64(inp["gates"][b, hs]), cfg.scale)
+    return res

@@ -326,6 +326,137 @@ def test_block_sink_tokens_always_in():
     np.testing.assert_allclose(out, ref, atol=1e-12)
 
 
+# ------------------------------------------------------------ NSA branches
+
+def _sdpa(q, K, V, scale):
+    """torch's attention routine in fp64, one query per row of q."""
+    t = lambda a: torch.as_tensor(np.asarray(a, dtype=np.float64))
+    o = torch.nn.functional.scaled_dot_product_attention(t(q)[:, None, :], t(K)[None], t(V)[None], scale=scale)
+    return o[:, 0, :].numpy()
+
+
+def test_nsa_shared_choice_example(golden_dir):
+    """MLA-S "选块和合并输出，实际算一遍": alone the heads read blocks 0 and 2,
+    summed over the group they share block 1."""
+    g = _golden(golden_dir, "nsa_shared_choice.json")
+    P = g["head_probabilities"]
+    assert [oracle.shared_block_choice([h], 1)[0] for h in P] == g["each_head_alone"]
+    assert oracle.shared_block_choice(P, g["count"]) == g["shared_choice"]
+    assert oracle.shared_block_choice(P, 3) == [1, 0, 2]
+    assert oracle.shared_block_choice([[0.5, 0.5]], 1) == [0]   # ties to the lower block
+
+
+def test_nsa_gate_example(golden_dir):
+    """MLA-S same section: independent gates, the mix exceeds every branch."""
+    g = _golden(golden_dir, "nsa_gates.json")
+    o = [np.array([x]) for x in g["branch_outputs"]]
+    got = oracle.nsa_combine(*o, g["gates"])
+    assert abs(got[0] - g["output"]) < 1e-12 and got[0] > max(g["branch_outputs"])
+
+
+def test_nsa_select_scores_aggregation():
+    """NSA §3.3 aggregation by hand.  Aligned blocks (l = d = l') leave the
+    scores as they are; l = 4, d = 2, l' = 4 on powers of two (so every term
+    shows in the sum) gives p0+2p1+p2, p2+2p3+p4, p4."""
+    p = np.array([1.0, 2.0, 4.0, 8.0, 16.0])
+    np.testing.assert_array_equal(oracle.nsa_select_scores(p, 4, 4, 4), p)
+    np.testing.assert_array_equal(oracle.nsa_select_scores(p, 4, 2, 4), [9.0, 36.0, 16.0])
+    # l = 2, d = 1, l' = 2: p[2j] + p[2j+1] + p[2j+1] + p[2j+2]
+    np.testing.assert_array_equal(oracle.nsa_select_scores(p[:4], 2, 1, 2), [1 + 2 + 2 + 4, 4 + 8 + 8])
+    with pytest.raises(ValueError):
+        oracle.nsa_select_scores(p, 3, 2, 4)
+
+
+def _nsa_case(seed, G=4, L=300, D=16):
+    rng = np.random.default_rng(seed)
+    return rng.standard_normal((G, D)), rng.standard_normal((L, D)), rng.standard_normal((L, D))
+
+
+def test_nsa_window_branch_is_sliding_window():
+    q, K, V = _nsa_case(11)
+    gates = np.tile([0.0, 0.0, 1.0], (4, 1))
+    out, _, _ = oracle.nsa_decode_group(q, K, V, 32, 2, 45, gates, 0.25)
+    np.testing.assert_allclose(out, _sdpa(q, K[-45:], V[-45:], 0.25), atol=1e-12)
+    out, _, _ = oracle.nsa_decode_group(q, K, V, 32, 2, 10**6, gates, 0.25)   # window past the start
+    np.testing.assert_allclose(out, _sdpa(q, K, V, 0.25), atol=1e-12)
+
+
+def test_nsa_selection_of_every_block_is_dense():
+    q, K, V = _nsa_case(12, L=256)
+    out, chosen, _ = oracle.nsa_decode_group(q, K, V, 32, 8, 0, np.tile([0.0, 1.0, 0.0], (4, 1)), 0.3)
+    assert chosen.tolist() == list(range(8))
+    np.testing.assert_allclose(out, _sdpa(q, K, V, 0.3), atol=1e-12)
+
+
+def test_nsa_compression_equals_dense_on_blockwise_constant_history():
+    """Keys and values constant inside each block: every token of a block has
+    its block's score, so attending to the B copies is attending to the block
+    summary once (the factor B cancels) -- which holds only if the summary is
+    the block mean.  Block 1 compression is plain dense attention."""
+    rng = np.random.default_rng(13)
+    G, B, nb, D = 3, 16, 7, 8
+    Kb, Vb, q = rng.standard_normal((nb, D)), rng.standard_normal((nb, D)), rng.standard_normal((G, D))
+    K, V = np.repeat(Kb, B, axis=0), np.repeat(Vb, B, axis=0)
+    gates = np.tile([1.0, 0.0, 0.0], (G, 1))
+    out, _, p_cmp = oracle.nsa_decode_group(q, K, V, B, 1, 0, gates, 0.4)
+    np.testing.assert_allclose(out, _sdpa(q, K, V, 0.4), atol=1e-12)
+    np.testing.assert_allclose(p_cmp.sum(axis=1), 1.0, atol=1e-14)
+    q, K, V = _nsa_case(14, G=2, L=50)
+    out, _, _ = oracle.nsa_decode_group(q, K, V, 1, 1, 0, np.tile([1.0, 0.0, 0.0], (2, 1)), 0.5)
+    np.testing.assert_allclose(out, _sdpa(q, K, V, 0.5), atol=1e-12)
+
+
+def test_nsa_selection_follows_the_group_not_one_head():
+    """Two heads, one KV head: head 0 alone prefers block 0, head 1 block 2, the
+    group sum block 1 (the shape of the pages' example).  The selected branch
+    reads exactly block 1 for both heads."""
+    D, B = 4, 8
+    K = np.zeros((3 * B, D))
+    K[0:B, 0] = 3.0                    # block 0: head 0's favourite
+    K[B:2 * B, 0] = 2.8                # block 1: good for both
+    K[B:2 * B, 1] = 2.8
+    K[2 * B:, 1] = 3.0                 # block 2: head 1's favourite
+    V = np.random.default_rng(15).standard_normal((3 * B, D))
+    q = np.array([[1.0, 0.0, 0, 0], [0.0, 1.0, 0, 0]])
+    gates = np.tile([0.0, 1.0, 0.0], (2, 1))
+    for h in range(2):
+        _, alone, _ = oracle.nsa_decode_group(q[h:h + 1], K, V, B, 1, 0, gates[:1], 1.0)
+        assert alone.tolist() == [[0], [2]][h]
+    out, chosen, _ = oracle.nsa_decode_group(q, K, V, B, 1, 0, gates, 1.0)
+    assert chosen.tolist() == [1]
+    np.testing.assert_allclose(out, _sdpa(q, K[B:2 * B], V[B:2 * B], 1.0), atol=1e-12)
+
+
+def test_nsa_incomplete_block_stays_out_of_compression_and_selection():
+    """MLA-S causality check: a block that is not complete is never summarised.
+    Changing the keys and values of the tail past the last complete block
+    moves neither the compression scores nor the choice nor (without the
+    window) the output; the window branch does see it."""
+    q, K, V = _nsa_case(16, L=300)
+    gates = np.tile([0.6, 0.8, 0.0], (4, 1))
+    a = oracle.nsa_decode_group(q, K, V, 64, 2, 0, gates, 0.25)
+    K2, V2 = K.copy(), V.copy()
+    K2[256:] = 50.0 * np.random.default_rng(17).standard_normal((44, 16))
+    V2[256:] += 999.0
+    b = oracle.nsa_decode_group(q, K2, V2, 64, 2, 0, gates, 0.25)
+    assert a[2].shape == (4, 4) and a[1].tolist() == b[1].tolist()
+    np.testing.assert_array_equal(a[2], b[2])
+    np.testing.assert_array_equal(a[0], b[0])
+    c = oracle.nsa_decode_group(q, K2, V2, 64, 2, 16, np.tile([0.0, 0.0, 1.0], (4, 1)), 0.25)
+    assert np.all(c[0] > 500.0)
+
+
+def test_nsa_gates_mix_linearly_and_short_history_has_only_the_window():
+    q, K, V = _nsa_case(18, L=200)
+    parts = [oracle.nsa_decode_group(q, K, V, 32, 2, 40, np.tile(e, (4, 1)), 0.25)[0] for e in np.eye(3)]
+    g = np.random.default_rng(19).uniform(0, 1, (4, 3))
+    out, _, _ = oracle.nsa_decode_group(q, K, V, 32, 2, 40, g, 0.25)
+    np.testing.assert_allclose(out, sum(g[:, i:i + 1] * parts[i] for i in range(3)), atol=1e-12)
+    out, chosen, p_cmp = oracle.nsa_decode_group(q, K[:20], V[:20], 32, 2, 8, g, 0.25)
+    assert chosen.size == 0 and p_cmp.shape == (4, 0)
+    np.testing.assert_allclose(out, g[:, 2:3] * _sdpa(q, K[12:20], V[12:20], 0.25), atol=1e-12)
+
+
 # ------------------------------------------------------------ whole step
 
 def test_dsa_step_placement_invariance():

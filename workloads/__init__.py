@@ -104,6 +104,34 @@ class BlockConfig:
         return self.L // self.block
 
 
+@dataclass(frozen=True)
+class NSAConfig:
+    """Shapes of the NSA three-branch decode workload: one decode query per
+    head, H query heads in GQA groups of H / H_kv sharing one KV head."""
+    name: str
+    seed: int
+    B: int
+    L: int
+    H: int
+    H_kv: int
+    D: int = 128
+    block: int = 64
+    top_blocks: int = 16
+    window: int = 512
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.D)
+
+    @property
+    def n_blocks(self) -> int:
+        return self.L // self.block
+
+    @property
+    def G(self) -> int:
+        return self.H // self.H_kv
+
+
 def _ragged_lens(seed: int, n: int, lo: int, hi: int) -> tuple:
     rng = np.random.Generator(np.random.PCG64(seed))
     return tuple(int(x) for x in rng.integers(lo, hi + 1, size=n))
@@ -119,8 +147,11 @@ PREFILL = DSAConfig(name="prefill", seed=1004, n_seqs=1, lens=(65536,), rows=409
                     prefill_start=61440)
 BLOCK = BlockConfig(name="block", seed=1005, B=8, L=131072, H=32)
 
+NSA = NSAConfig(name="nsa", seed=1006, B=8, L=131072, H=32, H_kv=4)
+
 DSA_CONFIGS = {c.name: c for c in (TINY, LONG, RAGGED, PREFILL)}
 BLOCK_CONFIGS = {BLOCK.name: BLOCK}
+NSA_CONFIGS = {NSA.name: NSA}
 
 
 def small_dsa(base: DSAConfig, **kw) -> DSAConfig:
@@ -224,3 +255,16 @@ def block_inputs(cfg: BlockConfig, device="cpu", seed: Optional[int] = None) -> 
     K = _normal_bf16(g, (cfg.B, cfg.L, cfg.H, cfg.D), dev)
     V = _normal_bf16(g, (cfg.B, cfg.L, cfg.H, cfg.D), dev)
     return dict(cfg=cfg, q=q, K=K, V=V)
+
+
+def nsa_inputs(cfg: NSAConfig, device="cpu", seed: Optional[int] = None) -> dict:
+    """Draw q [B,H,D], K and V [B,L,H_kv,D] (all N(0,1) bf16) and the branch
+    gates [B,H,3] (fp32, uniform in (0,1): values a sigmoid can take)."""
+    seed = cfg.seed if seed is None else seed
+    dev = torch.device(device)
+    g = _gen(dev, seed)
+    q = _normal_bf16(g, (cfg.B, cfg.H, cfg.D), dev)
+    K = _normal_bf16(g, (cfg.B, cfg.L, cfg.H_kv, cfg.D), dev)
+    V = _normal_bf16(g, (cfg.B, cfg.L, cfg.H_kv, cfg.D), dev)
+    gates = torch.rand((cfg.B, cfg.H, 3), generator=g, device=dev, dtype=torch.float32)
+    return dict(cfg=cfg, q=q, K=K, V=V, gates=gates)
