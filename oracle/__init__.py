@@ -260,6 +260,26 @@ def nsa_select_scores(p_cmp, l: int, d: int, l_sel: int):
     return out
 
 
+def nsa_compress(X, block: int) -> np.ndarray:
+    """The NSA compressed cache as stored: the mean of each complete block of
+    rows of X [L, D] ([Ch11] §12.6 mean compression), kept in bf16 like the
+    token cache it summarises.  Rounding the mean to bf16 is a quantisation,
+    so it is taken in the precision the stored cache is built in: an fp32 sum
+    over the block's rows in token order, times 1/block, rounded to the
+    nearest bf16 (ties to even).  Returns [L // block, D] float64 holding
+    bf16 values."""
+    import torch
+    X = np.asarray(X, dtype=np.float32)
+    nb = X.shape[0] // block
+    out = np.zeros((nb, X.shape[1]), dtype=np.float32)
+    for n in range(nb):
+        acc = np.zeros(X.shape[1], dtype=np.float32)
+        for i in range(block):
+            acc = acc + X[n * block + i]
+        out[n] = acc * np.float32(1.0 / block)
+    return torch.from_numpy(out).to(torch.bfloat16).to(torch.float64).numpy()
+
+
 def nsa_combine(o_cmp, o_sel, o_win, gates):
     """[MLA-S] g_c o_c + g_s o_s + g_w o_w with independent (sigmoid) gates:
     the gates are not normalised to sum to one."""
@@ -274,7 +294,8 @@ def _softmax_attend(q, K, V, scale):
     return a @ V, a
 
 
-def nsa_decode_group(q, K, V, block: int, top_blocks: int, window: int, gates, scale: float, chosen=None):
+def nsa_decode_group(q, K, V, block: int, top_blocks: int, window: int, gates, scale: float, chosen=None,
+                     compressed=None):
     """One decode query per head of a GQA group sharing one KV head.
 
     q [G, D], K/V [L, D] (the history; the query sees all L positions), gates
@@ -289,13 +310,18 @@ def nsa_decode_group(q, K, V, block: int, top_blocks: int, window: int, gates, s
     A branch with no position (no complete block) contributes zero.
     `chosen` (block indices) replaces the group's own choice when given: it
     evaluates the branches on another valid choice among near-tied blocks.
+    `compressed` = (K_bar, V_bar) replaces the exact block means (e.g. with
+    the stored bf16 cache of nsa_compress).
     Returns (out [G, D], chosen blocks ascending, p_cmp [G, n_blocks])."""
     q, K, V, g = _f64(q), _f64(K), _f64(V), _f64(gates)
     G, D = q.shape
     L = K.shape[0]
     nb = L // block
-    kbar = K[: nb * block].reshape(nb, block, D).mean(axis=1) if nb else np.zeros((0, D))
-    vbar = V[: nb * block].reshape(nb, block, D).mean(axis=1) if nb else np.zeros((0, D))
+    if compressed is not None:
+        kbar, vbar = _f64(compressed[0])[:nb], _f64(compressed[1])[:nb]
+    else:
+        kbar = K[: nb * block].reshape(nb, block, D).mean(axis=1) if nb else np.zeros((0, D))
+        vbar = V[: nb * block].reshape(nb, block, D).mean(axis=1) if nb else np.zeros((0, D))
     p_cmp = np.zeros((G, nb))
     o_cmp = np.zeros((G, D))
     for h in range(G):
@@ -398,14 +424,18 @@ def block_step(inp: dict, pairs: Sequence[tuple]) -> dict:
 
 
 def nsa_step(inp: dict, pairs: Sequence[tuple]) -> dict:
-    """nsa_decode_group on workload tensors for (sequence b, KV head g) pairs:
+    """nsa_decode_group on workload tensors for (sequence b, KV head g) pairs,
+    with the compression branch on the stored bf16 cache (nsa_compress):
     q [B, H, D], K and V [B, L, H_kv, D], gates [B, H, 3]; query heads
-    g*G .. g*G+G-1 share KV head g (G = H / H_kv)."""
+    g*G .. g*G+G-1 share KV head g (G = H / H_kv).  Returns per pair
+    (out [G, D], chosen blocks, p_cmp [G, n_blocks])."""
     cfg = inp["cfg"]
     G = cfg.H // cfg.H_kv
     res = {}
     for b, g in pairs:
         hs = slice(g * G, (g + 1) * G)
-        res[(b, g)] = nsa_decode_group(_host64(inp["q"][b, hs]), _host64(inp["K"][b, :, g]), _host64(inp["V"][b, :, g]),
-                                       cfg.block, cfg.top_blocks, cfg.window, _host64(inp["gates"][b, hs]), cfg.scale)
+        K, V = _host64(inp["K"][b, :, g]), _host64(inp["V"][b, :, g])
+        cache = (nsa_compress(K, cfg.block), nsa_compress(V, cfg.block))
+        res[(b, g)] = nsa_decode_group(_host64(inp["q"][b, hs]), K, V, cfg.block, cfg.top_blocks, cfg.window,
+                                       _host64(inp["gates"][b, hs]), cfg.scale, compressed=cache)
     return res

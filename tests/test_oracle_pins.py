@@ -457,6 +457,26 @@ def test_nsa_gates_mix_linearly_and_short_history_has_only_the_window():
     np.testing.assert_allclose(out, g[:, 2:3] * _sdpa(q, K[12:20], V[12:20], 0.25), atol=1e-12)
 
 
+def test_nsa_compress_stored_cache():
+    """The stored cache is the block mean rounded to bf16: exact on blocks of
+    small integers (their fp32 sums are exact), equal to torch's fp64 mean
+    rounded to bf16 on N(0,1) bf16 data except where that mean sits within an
+    fp32 rounding of a bf16 tie, and never more than half a bf16 ulp (plus
+    the fp32 sum's error) away from the exact mean."""
+    g = torch.Generator().manual_seed(21)
+    Xi = torch.randint(-8, 9, (4 * 64 + 17, 32), generator=g).to(torch.float64)
+    want = Xi[:256].reshape(4, 64, 32).mean(dim=1).to(torch.bfloat16).to(torch.float64).numpy()
+    np.testing.assert_array_equal(oracle.nsa_compress(Xi.numpy(), 64), want)
+    X = torch.randn(64 * 40, 128, generator=g).to(torch.bfloat16).to(torch.float64)
+    exact = X.reshape(40, 64, 128).mean(dim=1)
+    got = oracle.nsa_compress(X.numpy(), 64)
+    ref = exact.to(torch.bfloat16).to(torch.float64).numpy()
+    assert (got == ref).mean() > 0.999
+    ulp = 2.0 ** (np.floor(np.log2(np.maximum(np.abs(exact.numpy()), 1e-30))) - 7)
+    assert np.all(np.abs(got - exact.numpy()) <= 0.5 * ulp + 1e-6)
+    assert oracle.nsa_compress(X.numpy()[:63], 64).shape == (0, 128)
+
+
 # ------------------------------------------------------------ whole step
 
 def test_dsa_step_placement_invariance():
