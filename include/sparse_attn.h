@@ -13,6 +13,9 @@
  *   sa_block_mean_pool   mean-pooled block keys (run when blocks complete)
  *   sa_block_sparse_attn top blocks by q . mean(K_block), plus sink and window; softmax
  *                        over the union of their tokens
+ *   sa_nsa_compress      NSA compressed cache: bf16 block means of K and V
+ *   sa_nsa_decode        NSA three branches (compression, group-shared block
+ *                        selection, window), each its own softmax, gated sum
  *
  * Sources, cited by page title and section:
  *   [Notes]  "Sparse Attention 数学学习笔记" (echobase-5bl.pages.dev, 2026.09.14)
@@ -278,6 +281,48 @@ sa_status sa_block_sparse_attn(const void* q, const float* pooled, int64_t poole
                                int64_t stride_h, int B, int H, int D, int L, int block,
                                int top_blocks, int sink_blocks, int window, float scale,
                                float* out, int32_t* sel_blocks, sa_stream_t stream);
+
+/*
+ * NSA compressed cache ([Ch11] §12.6 mean compression; [MLA-S] NSA: only
+ * complete blocks are summarised):
+ *   Kc[b][h][n][d] = bf16( (sum_{i<block} K[b][n*block+i][h][d]) * (1/block) )
+ * with the sum taken in fp32 in token order and rounded to the nearest bf16;
+ * Vc likewise from V; for every complete block n < L / block.  Run when a
+ * block completes (the decode reads the cache).
+ *   K, V bf16, element (b,t,h,d) at b*stride_b + t*stride_t + h*stride_h + d
+ *   Kc, Vc [B][H_kv][c_ld][D] bf16, c_ld >= L / block
+ * Supported: D = 128.
+ */
+sa_status sa_nsa_compress(const void* K, const void* V, int64_t stride_b, int64_t stride_t, int64_t stride_h,
+                          int B, int L, int H_kv, int D, int block, void* Kc, void* Vc, int64_t c_ld,
+                          sa_stream_t stream);
+
+/*
+ * NSA three-branch decode for the query at position L-1 of every head
+ * ([MLA-S] NSA sections "三条路径，各留住什么？" and "选块和合并输出，实际算一遍";
+ * [LLMRes] NSA steps 1-3).  Query head h uses KV head h / G, G = H / H_kv.
+ * For each (sequence b, KV head g) and its G query heads, three branches,
+ * each with its own softmax over scale * q . k:
+ *   compression: the n_b = L / block complete blocks, keys Kc, values Vc;
+ *   selection:   the min(top_blocks, n_b) blocks with the largest sum over the
+ *                group's heads of the compression probabilities (ties to the
+ *                lower block), all their tokens;
+ *   window:      positions [max(0, L - window), L);
+ *   out[b][h] = gates[b][h][0] o_cmp + gates[b][h][1] o_sel + gates[b][h][2] o_win
+ * A branch with no position contributes zero.  The gates are used as given
+ * (values of a sigmoid; not normalised).
+ *   q [B][H][D] bf16; K, V as in sa_nsa_compress (16-byte aligned rows);
+ *   Kc, Vc from sa_nsa_compress (may be NULL when L < block); gates [B][H][3]
+ *   fp32; out [B][H][D] fp32; sel_blocks [B][H_kv][top_blocks] int32
+ *   (ascending, -1 padded) or NULL.
+ * Supported: D = 128, H / H_kv <= 16, block a multiple of 32 up to 256,
+ * top_blocks <= 64, window <= 4096, L / block <= 4096, and shapes whose
+ * per-CTA shared memory fits (SA_EUNSUPPORTED otherwise).
+ */
+sa_status sa_nsa_decode(const void* q, const void* K, const void* V, int64_t stride_b, int64_t stride_t,
+                        int64_t stride_h, const void* Kc, const void* Vc, int64_t c_ld, const float* gates,
+                        int B, int H, int H_kv, int D, int L, int block, int top_blocks, int window, float scale,
+                        float* out, int32_t* sel_blocks, sa_stream_t stream);
 
 #ifdef __cplusplus
 }

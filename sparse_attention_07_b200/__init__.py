@@ -29,6 +29,7 @@ EXPORTS = (
     "sa_sparse_mla_prefill",
     "sa_block_mean_pool", "sa_block_sparse_attn", "sa_sparse_mla_decode_static",
     "sa_dense_mla_workspace_size", "sa_dense_mla_decode", "sa_mla_absorb_query", "sa_mla_up_project",
+    "sa_nsa_compress", "sa_nsa_decode",
 )
 
 # Size of the library's static device array behind sparse_mla_decode_static
@@ -71,6 +72,8 @@ def lib():
         L.sa_sparse_mla_decode_static.argtypes = [P, P, P, I64, P, I64, I64, P, I, P, P, I, I, I, I, I, F, P, P, P]
         L.sa_block_mean_pool.argtypes = [P, I64, I64, I64, I, I, I, I, I, P, I64, P]
         L.sa_block_sparse_attn.argtypes = [P, P, I64, P, P, I64, I64, I64, I, I, I, I, I, I, I, I, F, P, P, P]
+        L.sa_nsa_compress.argtypes = [P, P, I64, I64, I64, I, I, I, I, I, P, P, I64, P]
+        L.sa_nsa_decode.argtypes = [P, P, P, I64, I64, I64, P, P, I64, P, I, I, I, I, I, I, I, I, F, P, P, P]
         for name in EXPORTS:
             if name not in ("sa_status_string", "sa_version", "sa_sparse_mla_workspace_size",
                             "sa_sparse_mla_prefill_workspace_size", "sa_dense_mla_workspace_size"):
@@ -271,4 +274,39 @@ def block_sparse_attn(q, pooled, K, V, block: int, top_blocks: int, sink_blocks:
                                     K.stride(2), B, H, D, L, block, top_blocks, sink_blocks, window, float(scale),
                                     _p(out), _p(sel_blocks), _stream())
     _check("sa_block_sparse_attn", st)
+    return out
+
+
+def nsa_compress(K, V, block: int = 64, Kc=None, Vc=None):
+    """NSA compressed cache: bf16 block means of K and V [B, L, H_kv, D] ->
+    Kc, Vc [B, H_kv, L//block, D] bf16 (complete blocks only)."""
+    B, L, Hkv, D = K.shape
+    nb = L // block
+    if Kc is None:
+        Kc = torch.empty(B, Hkv, max(nb, 1), D, dtype=torch.bfloat16, device=K.device)
+    if Vc is None:
+        Vc = torch.empty_like(Kc)
+    if V.stride() != K.stride() or not (Kc.is_contiguous() and Vc.is_contiguous()):
+        raise ValueError("K and V must share one layout; Kc and Vc must be contiguous")
+    st = lib().sa_nsa_compress(_p(K), _p(V), K.stride(0), K.stride(1), K.stride(2), B, L, Hkv, D, block, _p(Kc),
+                               _p(Vc), Kc.shape[2], _stream())
+    _check("sa_nsa_compress", st)
+    return Kc, Vc
+
+
+def nsa_decode(q, K, V, Kc, Vc, gates, block: int, top_blocks: int, window: int, scale: float, out=None,
+               sel_blocks=None):
+    """NSA three-branch decode of the query at position L-1 of every head:
+    q [B, H, D] bf16, K and V [B, L, H_kv, D] bf16, Kc and Vc from
+    nsa_compress, gates [B, H, 3] fp32 -> out [B, H, D] fp32."""
+    B, L, Hkv, D = K.shape
+    H = q.shape[1]
+    if V.stride() != K.stride() or not (Kc.is_contiguous() and Vc.is_contiguous()):
+        raise ValueError("K and V must share one layout; Kc and Vc must be contiguous")
+    if out is None:
+        out = torch.empty(B, H, D, dtype=torch.float32, device=q.device)
+    st = lib().sa_nsa_decode(_p(q), _p(K), _p(V), K.stride(0), K.stride(1), K.stride(2), _p(Kc), _p(Vc),
+                             Kc.shape[2], _p(gates), B, H, Hkv, D, L, block,
+                             top_blocks, window, float(scale), _p(out), _p(sel_blocks), _stream())
+    _check("sa_nsa_decode", st)
     return out

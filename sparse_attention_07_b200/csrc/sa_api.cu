@@ -360,4 +360,39 @@ sa_status sa_block_sparse_attn(const void* q, const float* pooled, int64_t poole
                                reinterpret_cast<cudaStream_t>(stream));
 }
 
+sa_status sa_nsa_compress(const void* K, const void* V, int64_t stride_b, int64_t stride_t, int64_t stride_h, int B,
+                          int L, int H_kv, int D, int block, void* Kc, void* Vc, int64_t c_ld, sa_stream_t stream) {
+    if (B < 0 || L < 0 || H_kv < 0 || block < 1) return SA_EINVAL;
+    if (D != 128) return SA_EUNSUPPORTED;
+    if (B == 0 || H_kv == 0 || L / block == 0) return SA_OK;
+    if (!K || !V || !Kc || !Vc || c_ld < L / block) return SA_EINVAL;
+    if (!aligned(K, 8) || !aligned(V, 8) || !aligned(Kc, 8) || !aligned(Vc, 8) || stride_b % 4 || stride_t % 4 ||
+        stride_h % 4)
+        return SA_EINVAL;
+    return nsa_compress_launch(K, V, stride_b, stride_t, stride_h, B, L, H_kv, block, Kc, Vc, c_ld,
+                               reinterpret_cast<cudaStream_t>(stream));
+}
+
+sa_status sa_nsa_decode(const void* q, const void* K, const void* V, int64_t stride_b, int64_t stride_t,
+                        int64_t stride_h, const void* Kc, const void* Vc, int64_t c_ld, const float* gates, int B,
+                        int H, int H_kv, int D, int L, int block, int top_blocks, int window, float scale,
+                        float* out, int32_t* sel_blocks, sa_stream_t stream) {
+    if (B < 0 || H < 1 || H_kv < 1 || H % H_kv != 0 || L < 1 || block < 1 || top_blocks < 0 || window < 0 ||
+        !std::isfinite(scale))
+        return SA_EINVAL;
+    if (D != 128 || H / H_kv > 16 || block % 32 != 0 || block > 256 || top_blocks > 64 || window > 4096 ||
+        L / block > 4096 || static_cast<int64_t>(B) * H_kv * 8 > 0x7fffffff)
+        return SA_EUNSUPPORTED;
+    if (nsa_decode_smem(H / H_kv, L, block, top_blocks, window, nullptr, nullptr) > kNsaMaxSmem)
+        return SA_EUNSUPPORTED;
+    if (B == 0) return SA_OK;
+    if (!q || !K || !V || !gates || !out || (L / block > 0 && (!Kc || !Vc)) || c_ld < L / block) return SA_EINVAL;
+    if (!aligned(q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(out, 4) || !aligned(gates, 4) ||
+        (Kc && !aligned(Kc, 16)) || (Vc && !aligned(Vc, 16)) || stride_b % 8 || stride_t % 8 || stride_h % 8)
+        return SA_EINVAL;
+    return nsa_decode_launch(q, K, V, stride_b, stride_t, stride_h, Kc ? Kc : K, Vc ? Vc : V, c_ld, gates, B, H,
+                             H_kv, L, block, top_blocks, window, scale, out, sel_blocks,
+                             reinterpret_cast<cudaStream_t>(stream));
+}
+
 }  // extern "C"

@@ -135,5 +135,40 @@ def test_block_validation(L):
     assert g(FAKE, 8, 8, 128, 2, 1000, 4, 128, 0, FAKE, 15, None) == sa.SA_EINVAL
 
 
+def test_nsa_validation(L):
+    f = L.sa_nsa_decode
+    args = dict(q=FAKE, K=FAKE, V=FAKE, sb=8 * 131072 * 4 * 128, st=4 * 128, sh=128, Kc=FAKE, Vc=FAKE, cld=2048,
+                gates=FAKE, B=8, H=32, Hkv=4, D=128, L=131072, block=64, top=16, win=512, scale=0.088, out=FAKE,
+                sel=None)
+
+    def call(**kw):
+        a = {**args, **kw}
+        return f(a["q"], a["K"], a["V"], a["sb"], a["st"], a["sh"], a["Kc"], a["Vc"], a["cld"], a["gates"], a["B"],
+                 a["H"], a["Hkv"], a["D"], a["L"], a["block"], a["top"], a["win"], a["scale"], a["out"], a["sel"],
+                 None)
+
+    assert call(B=0) == sa.SA_OK
+    assert call(D=64) == sa.SA_EUNSUPPORTED
+    assert call(H=34, Hkv=2) == sa.SA_EUNSUPPORTED      # groups of 17 heads
+    assert call(block=48) == sa.SA_EUNSUPPORTED
+    assert call(top=65) == sa.SA_EUNSUPPORTED
+    assert call(win=4097) == sa.SA_EUNSUPPORTED
+    assert call(L=64 * 4097) == sa.SA_EUNSUPPORTED
+    assert call(H=30) == sa.SA_EINVAL                   # not a whole number of groups
+    assert call(L=0) == sa.SA_EINVAL
+    assert call(top=-1) == sa.SA_EINVAL
+    assert call(cld=100) == sa.SA_EINVAL
+    assert call(st=4 * 128 + 4) == sa.SA_EINVAL          # rows not 16-byte aligned
+    assert call(q=MISALIGNED) == sa.SA_EINVAL
+    assert call(Kc=None) == sa.SA_EINVAL
+    assert call(gates=None) == sa.SA_EINVAL
+    assert call(scale=float("nan")) == sa.SA_EINVAL
+    g = L.sa_nsa_compress
+    assert g(FAKE, FAKE, 8, 8, 128, 2, 1000, 4, 64, 64, FAKE, FAKE, 15, None) == sa.SA_EUNSUPPORTED
+    assert g(FAKE, FAKE, 8, 8, 128, 2, 1000, 4, 128, 64, FAKE, FAKE, 10, None) == sa.SA_EINVAL   # cache too short
+    assert g(FAKE, None, 8, 8, 128, 2, 1000, 4, 128, 64, FAKE, FAKE, 15, None) == sa.SA_EINVAL
+    assert g(FAKE, FAKE, 8, 8, 128, 2, 63, 4, 128, 64, None, None, 0, None) == sa.SA_OK       # no complete block
+
+
 def test_check_device_error_rejects_null(L):
     assert L.sa_check_device_error(None, None) == sa.SA_EINVAL
