@@ -4,7 +4,7 @@
 One step = the whole decode path over one batch: lightning indexer ->
 exact Top-K -> sparse MLA, i.e. one query per sequence of the workload.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--config long|ragged|tiny|prefill|block]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config long|ragged|tiny|prefill|block|nsa|crossover]
                     [--impl native|reference]
 
 Default workload: long decode, 32 sequences x 32768 tokens, H^I=64 fp8
@@ -73,6 +73,17 @@ def block_bytes(cfg: W.BlockConfig):
     # the union holds at most top*block + sink*block + window tokens
     u_max = min(cfg.L, cfg.top_blocks * cfg.block + cfg.sink_blocks * cfg.block + cfg.window)
     return pooled, u_max
+
+
+def nsa_bytes(cfg: W.NSAConfig):
+    """Algorithmic bytes of one NSA decode step, every (sequence, KV head):
+    the compressed K and V rows of every complete block, the K and V rows of
+    the selected blocks and of the window, the group's queries, gates and
+    outputs."""
+    nb = cfg.n_blocks
+    per_group = (2 * nb * cfg.D * 2 + min(cfg.top_blocks, nb) * cfg.block * 2 * cfg.D * 2
+                 + min(cfg.window, cfg.L) * 2 * cfg.D * 2 + cfg.G * (cfg.D * 2 + 12 + cfg.D * 4))
+    return per_group * cfg.B * cfg.H_kv
 
 
 # ---------------------------------------------------------------- ranks
@@ -226,6 +237,29 @@ class BlockStep:
         pass
 
 
+class NsaStep:
+    def __init__(self, inp, sa):
+        self.sa, self.inp, self.cfg = sa, inp, inp["cfg"]
+        c = self.cfg
+        self.Kc, self.Vc = sa.nsa_compress(inp["K"], inp["V"], c.block)  # once, when the blocks completed
+        self.out = torch.empty(c.B, c.H, c.D, dtype=torch.float32, device=inp["q"].device)
+        self.launches_per_step = 1
+
+    def indexer(self):
+        i, c = self.inp, self.cfg
+        self.sa.nsa_decode(i["q"], i["K"], i["V"], self.Kc, self.Vc, i["gates"], c.block, c.top_blocks, c.window,
+                           c.scale, out=self.out)
+
+    def rest(self):
+        pass
+
+    def topk(self):
+        pass
+
+    def attn(self):
+        pass
+
+
 def time_steps(step, K: int, flush):
     """K steps, each bracketed by CUDA events on the launching stream (torch's
     current stream, which the library calls use); the L2 flush runs between
@@ -285,10 +319,11 @@ def e2e_steps(step, K: int, flush):
     inp = step.inp
     if isinstance(step, DecodeStep):
         names = ["q_idx", "w", "q_lat", "q_rope"]
-        result = step.out
+    elif isinstance(step, NsaStep):
+        names = ["q", "gates"]
     else:
         names = ["q"]
-        result = step.out
+    result = step.out
     host_in = {n: inp[n].cpu().pin_memory() for n in names}
     host_out = torch.empty(result.shape, dtype=result.dtype).pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in host_in.values())
@@ -325,6 +360,18 @@ def cpu_baseline(inp, cfg, budget_s: float = 12.0):
         unit_n = n
         what = "query rows" if cfg.prefill_start < 0 else "query tokens"
         sample = f"{n} of {cfg.rows} {what} of the workload (indexer over every visible key, top-{cfg.topk}, sparse MLA)"
+    elif isinstance(cfg, W.NSAConfig):
+        pairs = [(b, g) for b in range(cfg.B) for g in range(cfg.H_kv)]
+        t0 = time.perf_counter()
+        oracle.nsa_step(inp, pairs[:1])
+        one = time.perf_counter() - t0
+        n = int(max(1, min(len(pairs), budget_s // max(one, 1e-3))))
+        t0 = time.perf_counter()
+        oracle.nsa_step(inp, pairs[:n])
+        dt = time.perf_counter() - t0
+        unit_n = n / cfg.H_kv  # queries = sequences; one query spans every head
+        sample = (f"{n} of {cfg.B * cfg.H_kv} (sequence, KV head) groups ({cfg.G} query heads each; "
+                  f"compressed cache built inside the timed call)")
     else:
         pairs = [(b, h) for b in range(cfg.B) for h in range(cfg.H)]
         t0 = time.perf_counter()
@@ -342,6 +389,8 @@ def cpu_baseline(inp, cfg, budget_s: float = 12.0):
 def workload(name: str):
     if name in W.DSA_CONFIGS:
         return W.DSA_CONFIGS[name]
+    if name in W.NSA_CONFIGS:
+        return W.NSA_CONFIGS[name]
     return W.BLOCK_CONFIGS[name]
 
 
@@ -353,6 +402,11 @@ def describe(cfg, flush_note):
         return {"workload": f"{cfg.name} {kind}: {cfg.rows} queries, {lens}, indexer H^I={cfg.H_I} d^I={cfg.d_I} "
                             f"{cfg.idx_dtype}, top-{cfg.topk}, sparse MLA {cfg.H} heads d_c={cfg.d_c} d_R={cfg.d_R} bf16",
                 "batch": cfg.rows, "seq_len": max(cfg.lens), "topk": cfg.topk, "heads": cfg.H, "l2": flush_note}
+    if isinstance(cfg, W.NSAConfig):
+        return {"workload": f"NSA three-branch decode: B={cfg.B}, L={cfg.L}, {cfg.H} query heads in {cfg.H_kv} GQA "
+                            f"groups, head_dim {cfg.D} bf16, block {cfg.block} (compression = selection blocks), "
+                            f"top-{cfg.top_blocks} blocks chosen per group, {cfg.window}-token window, fp32 gates",
+                "batch": cfg.B, "seq_len": cfg.L, "heads": cfg.H, "kv_heads": cfg.H_kv, "l2": flush_note}
     return {"workload": f"block-sparse decode: B={cfg.B}, L={cfg.L}, {cfg.H} MHA heads, head_dim {cfg.D} bf16, "
                         f"block {cfg.block}, top-{cfg.top_blocks} + {cfg.sink_blocks} sink block + {cfg.window}-token window",
             "batch": cfg.B, "seq_len": cfg.L, "heads": cfg.H, "l2": flush_note}
@@ -372,6 +426,9 @@ def run_native(args):
     if isinstance(cfg, W.DSAConfig):
         inp = W.dsa_inputs(cfg, dev, seed=rank_seed(cfg.seed, rank))
         step = DecodeStep(inp, sa)
+    elif isinstance(cfg, W.NSAConfig):
+        inp = W.nsa_inputs(cfg, dev, seed=rank_seed(cfg.seed, rank))
+        step = NsaStep(inp, sa)
     else:
         inp = W.block_inputs(cfg, dev, seed=rank_seed(cfg.seed, rank))
         step = BlockStep(inp, sa)
@@ -456,6 +513,15 @@ def run_native(args):
         res["kernels"] = kern
         if not prefill:
             res["projections"] = time_projections(step, min(args.steps, 20), flush, hbm)
+    elif isinstance(cfg, W.NSAConfig):
+        units = cfg.B * ws
+        unit = "queries/s"
+        metric = "NSA decode queries/s (compression + group block choice + selection + window, gated)"
+        nbytes = nsa_bytes(cfg)
+        ach = nbytes / (first * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": hbm, "unit": "GB/s", "frac": round(ach / hbm, 4),
+                "traffic": None, "kernel": "nsa_decode_kernel", "bytes_per_launch": nbytes,
+                "peak_source": f"{peak_src} hbm_gbs"}
     else:
         units = cfg.B * ws
         unit = "queries/s"
@@ -591,6 +657,14 @@ def run_reference(args):
         run = lambda: oracle.dsa_step(inp, rows, with_scores=False)  # noqa: E731
         units_per_step = per_step
         sample = f"{per_step} query rows of the workload per step"
+    elif isinstance(cfg, W.NSAConfig):
+        inp = W.nsa_inputs(cfg, dev, seed=cfg.seed)
+        unit = "queries/s"
+        metric = "NSA decode queries/s (compression + group block choice + selection + window, gated)"
+        run = lambda: oracle.nsa_step(inp, [(0, 0)])  # noqa: E731
+        units_per_step = 1.0 / cfg.H_kv  # one of the query's KV-head groups
+        sample = (f"one (sequence, KV head) group ({cfg.G} of the query's {cfg.H} heads) per step, compressed cache "
+                  f"built inside the timed call")
     else:
         inp = W.block_inputs(cfg, dev, seed=cfg.seed)
         unit, metric = "queries/s", "block-sparse decode queries/s (pooled-block scan+top-k+block attention)"
@@ -625,7 +699,7 @@ def main(argv=None):
     p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--impl", choices=["native", "reference"], default="native")
     p.add_argument("--config", default="long",
-                   choices=sorted(list(W.DSA_CONFIGS) + list(W.BLOCK_CONFIGS) + ["crossover"]))
+                   choices=sorted(list(W.DSA_CONFIGS) + list(W.BLOCK_CONFIGS) + list(W.NSA_CONFIGS) + ["crossover"]))
     p.add_argument("--no-cpu-baseline", action="store_true")
     args = p.parse_args(argv)
     if args.warmup < 3 and args.impl == "native":

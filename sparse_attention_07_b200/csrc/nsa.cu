@@ -43,8 +43,9 @@ constexpr int kC = 8;                  // CTAs per (sequence, KV head)
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kRows = 32;              // rows per ring item
-constexpr int kRowB = 2 * kD + 16;     // padded bf16 row: 272 B keeps ldmatrix rows on distinct banks
-constexpr int kItemB = kRows * kRowB;  // 8704 B
+constexpr int kRowB = 2 * kD + 16;     // padded bf16 row of the query tile: 272 B, conflict-free fragment loads
+constexpr int kHalfB = kRows * 128;    // one TMA box: 32 rows x 64 dims, 128-byte swizzle
+constexpr int kItemB = 2 * kHalfB;     // an item: dims 0-63, then dims 64-127
 constexpr int kStages = 8;
 constexpr int kRingB = kStages * kItemB;
 constexpr int kMaxTop = 64;
@@ -86,6 +87,7 @@ __global__ void __launch_bounds__(256) nsa_compress_kernel(const __nv_bfloat16* 
     *reinterpret_cast<uint2*>(dst) = o;
 }
 
+
 // --------------------------------------------------------------- decode
 struct NsaArgs {
     const __nv_bfloat16* q;  // [B][H][D]
@@ -98,6 +100,7 @@ struct NsaArgs {
     const float* gates;      // [B][H][3]: compression, selection, window
     float* out;              // [B][H][D]
     int32_t* sel;            // [B][Hkv][top] or null
+    int* err;
     int H, Hkv, G, L, block, top, window;
     float scale;
     int per;                 // compressed blocks per CTA (multiple of kRows)
@@ -106,16 +109,19 @@ struct NsaArgs {
 
 // Shared-memory plan (bytes from the dynamic base); every region 16-byte aligned.
 struct Smem {
-    int q, sc, pc, sf, pf, keyw, cand, glob, total;
+    int q, sc, pc, sf, pf, part, keyw, cand, glob, recv, recv_ml, total;
     int ld_sc, ld_pc, ld_sf, ld_pf;  // row strides in elements
+    int hpc;                         // heads each CTA finishes
 };
 
-__host__ __device__ inline Smem smem_plan(int gp, int per, int ftok, int top) {
+__host__ __device__ inline Smem smem_plan(int G, int per, int ftok, int top) {
+    const int gp = G <= 8 ? 8 : 16;
     Smem s;
     s.ld_sc = per + 4;   // fp32 rows: stride = 4 mod 32 words spreads the fragment stores over the banks
     s.ld_pc = per + 8;   // bf16 rows: stride = 4 mod 8 words, conflict-free B-fragment loads
     s.ld_sf = ftok + 4;
     s.ld_pf = ftok + 8;
+    s.hpc = (G + kC - 1) / kC;
     int off = kRingB;
     auto take = [&](int bytes) {
         const int at = off;
@@ -127,10 +133,13 @@ __host__ __device__ inline Smem smem_plan(int gp, int per, int ftok, int top) {
     s.pc = take(gp * s.ld_pc * 2);
     s.sf = take(gp * s.ld_sf * 4);
     s.pf = take(gp * s.ld_pf * 2);
+    s.part = take(3 * 2 * (gp / 8) * 32 * 16);   // split-k partial score fragments
     s.keyw = take(per * 8);
     s.cand = take(kWarps * top * 8);
     s.glob = take(kC * top * 8);
-    s.total = off;
+    s.recv = take(kC * 3 * s.hpc * kD * 4);      // partial outputs pushed by the cluster, [rank][branch][head][d]
+    s.recv_ml = take(kC * 3 * s.hpc * 2 * 4);    // their (max, sum)
+    s.total = off + 1024;                        // the ring starts on a 1024-byte boundary (swizzle atoms)
     return s;
 }
 
@@ -156,19 +165,36 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y, int z,
+                                            int w) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5, "
+        "%6}], [%2];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z), "r"(w)
+        : "memory");
+}
 
-// Wait until at most n (0 <= n < kStages) of this thread's cp.async groups are pending.
-__device__ __forceinline__ void cp_async_wait_n(int n) {
-    switch (n) {
-        case 0: asm volatile("cp.async.wait_group 0;" ::: "memory"); break;
-        case 1: asm volatile("cp.async.wait_group 1;" ::: "memory"); break;
-        case 2: asm volatile("cp.async.wait_group 2;" ::: "memory"); break;
-        case 3: asm volatile("cp.async.wait_group 3;" ::: "memory"); break;
-        case 4: asm volatile("cp.async.wait_group 4;" ::: "memory"); break;
-        case 5: asm volatile("cp.async.wait_group 5;" ::: "memory"); break;
-        default: asm volatile("cp.async.wait_group 6;" ::: "memory"); break;
-    }
+// Byte offset of the 16-byte chunk c (0..7) of row r in a 128-byte-swizzled box.
+__device__ __forceinline__ uint32_t swz(int r, int c) {
+    return static_cast<uint32_t>(r * 128 + ((c ^ (r & 7)) << 4));
+}
+
+__device__ __forceinline__ void named_arrive(uint32_t id, uint32_t nthreads) {
+    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ void st_cluster_u64(uint32_t addr, unsigned long long v) {
+    asm volatile("st.shared::cluster.v2.u32 [%0], {%1, %2};" ::"r"(addr), "r"(static_cast<uint32_t>(v)),
+                 "r"(static_cast<uint32_t>(v >> 32))
+                 : "memory");
 }
 
 __device__ __forceinline__ unsigned long long shfl_xor_u64(unsigned long long v, int o) {
@@ -177,30 +203,57 @@ __device__ __forceinline__ unsigned long long shfl_xor_u64(unsigned long long v,
     return (static_cast<unsigned long long>(hi) << 32) | lo;
 }
 
-// One warp: the `count` largest nonzero keys of keys[0, n) into out[0, count)
-// (zero where fewer exist), largest first.  Keys are unique; taken keys are
-// zeroed in place.
-__device__ void warp_top(unsigned long long* keys, int n, int count, unsigned long long* out, int lane) {
-    for (int round = 0; round < count; ++round) {
-        unsigned long long best = 0ull;
-        int bj = -1;
-        for (int j = lane; j < n; j += 32) {
-            const unsigned long long k = keys[j];
-            if (k > best) {
-                best = k;
-                bj = j;
+__device__ __forceinline__ unsigned long long umax64(unsigned long long a, unsigned long long b) { return a > b ? a : b; }
+__device__ __forceinline__ unsigned long long umin64(unsigned long long a, unsigned long long b) { return a > b ? b : a; }
+
+// Bitonic sort, descending, of the warp's 32 (TWO: 64) keys: element e sits in
+// lane e % 32, slot e / 32.  Afterwards element 0 is the largest.
+template <bool TWO>
+__device__ __forceinline__ void warp_sort_desc(unsigned long long& v0, unsigned long long& v1, int lane) {
+#pragma unroll
+    for (int k = 2; k <= (TWO ? 64 : 32); k <<= 1) {
+#pragma unroll
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            if (j == 32) {  // k = 64: the partner is the other slot of this lane; one descending run
+                const unsigned long long hi = umax64(v0, v1), lo = umin64(v0, v1);
+                v0 = hi;
+                v1 = lo;
+                continue;
+            }
+            const bool is_lo = (lane & j) == 0;
+            {
+                const unsigned long long p = shfl_xor_u64(v0, j);
+                const bool desc = (lane & k) == 0;  // k <= 32 here or k = 64 (lane & 64 = 0)
+                v0 = (is_lo == desc) ? umax64(v0, p) : umin64(v0, p);
+            }
+            if (TWO) {
+                const unsigned long long p = shfl_xor_u64(v1, j);
+                const bool desc = ((lane + 32) & k) == 0;
+                v1 = (is_lo == desc) ? umax64(v1, p) : umin64(v1, p);
             }
         }
-        unsigned long long w = best;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const unsigned long long x = shfl_xor_u64(w, o);
-            w = x > w ? x : w;
-        }
-        if (w != 0ull && best == w) keys[bj] = 0ull;
-        if (lane == 0) out[round] = w;
-        __syncwarp();
     }
+}
+
+// Rank of key x (its position in descending order) among 8 descending lists
+// of n keys each (lists[l * n + i]), x being element `pos` of list `self`:
+// pos plus, for every other list, the number of its keys larger than x
+// (binary lifting with p2 > n, the 8 searches independent of one another).
+__device__ int rank_in_lists(const unsigned long long* lists, int n, int p2, int self, int pos,
+                             unsigned long long x) {
+    int c[8];
+#pragma unroll
+    for (int l = 0; l < 8; ++l) c[l] = 0;
+#pragma unroll 1
+    for (int step = p2 >> 1; step > 0; step >>= 1) {
+#pragma unroll
+        for (int l = 0; l < 8; ++l)
+            if (c[l] + step <= n && lists[l * n + c[l] + step - 1] > x) c[l] += step;
+    }
+    int rank = pos;
+#pragma unroll
+    for (int l = 0; l < 8; ++l) rank += l == self ? 0 : c[l];
+    return rank;
 }
 
 // Block key: larger is better; probability bits (nonnegative floats order as
@@ -218,7 +271,7 @@ __device__ __forceinline__ int key_block(unsigned long long k) {
 // for positions that do not exist): per head the max m, P = bf16(2^(s - m))
 // into the bf16 rows p, l = sum of P as rounded (the normaliser of the output
 // the tensor cores form from P).  With `keep`, the fp32 2^(s - m) replaces the
-// scores and its sum goes to Lsel (the compression probabilities that choose
+// scores and its sum goes to lsel (the compression probabilities that choose
 // blocks).  One warp per head; heads G .. GP-1 (padding) get P = 0.
 __device__ void branch_softmax(float* s, int ld_s, __nv_bfloat16* p, int ld_p, int npos, int G, int GP, bool keep,
                                float* m_out, float* l_out, float* lsel_out, int warp, int lane) {
@@ -257,71 +310,105 @@ __device__ void branch_softmax(float* s, int ld_s, __nv_bfloat16* p, int ld_p, i
 
 struct Plan {
     int b, kvh, r;
-    int nwi, nci, nsi, nA, n_items;  // items: window K, compressed K, window V, compressed V, selected K, selected V
+    int nwi, nci, nsi, nA, n_items;  // items: compressed K, window K, window V, compressed V, selected K, selected V
     int w_lo, n_lo, n_hi, ipb;
 };
 
-// cp.async of ring item i (32 rows of 256 B) into its slot; rows that do not
-// exist are zero-filled.  Every thread copies two 16-byte pieces.
-__device__ __forceinline__ void issue_item(const NsaArgs& a, const Plan& p, int i, uint32_t ring_s,
-                                           const int* chosen) {
-    const uint32_t base = ring_s + static_cast<uint32_t>((i % kStages) * kItemB);
-#pragma unroll
-    for (int k = 0; k < 2; ++k) {
-        const int idx = static_cast<int>(threadIdx.x) + k * kThreads;
-        const int row = idx >> 4, ch = idx & 15;
-        const __nv_bfloat16* src = a.Kc;
-        bool ok;
-        int j = i;
-        if (j < p.nwi || (j >= p.nwi + p.nci && j < 2 * p.nwi + p.nci)) {  // window rows
-            const bool isv = j >= p.nwi;
-            if (isv) j -= p.nwi + p.nci;
-            const int t = p.w_lo + kRows * (p.r + kC * j) + row;
-            ok = t < a.L;
-            if (ok) src = (isv ? a.V : a.K) + p.b * a.sb + static_cast<int64_t>(t) * a.st + p.kvh * a.sh;
-        } else if (j < p.nA) {  // compressed rows
-            const bool isv = j >= 2 * p.nwi + p.nci;
-            j -= isv ? 2 * p.nwi + p.nci : p.nwi;
-            const int n = p.n_lo + kRows * j + row;
-            ok = n < p.n_hi;
-            if (ok) src = (isv ? a.Vc : a.Kc) + ((static_cast<int64_t>(p.b) * a.Hkv + p.kvh) * a.c_ld + n) * kD;
-        } else {  // rows of the selected blocks
-            j -= p.nA;
-            const bool isv = j >= p.nsi;
-            if (isv) j -= p.nsi;
-            const int blk = chosen[p.r + kC * (j / p.ipb)];
-            const int t = blk * a.block + kRows * (j % p.ipb) + row;
-            ok = true;
-            src = (isv ? a.V : a.K) + p.b * a.sb + static_cast<int64_t>(t) * a.st + p.kvh * a.sh;
-        }
-        cp_async16(base + static_cast<uint32_t>(row * kRowB + ch * 16), ok ? src + ch * 8 : a.Kc, ok ? 16u : 0u);
+struct Maps {
+    CUtensorMap K, V;    // token cache: dims (D, H_kv, L, B), box 64 x 1 x 32 x 1
+    CUtensorMap Kc, Vc;  // compressed cache: dims (D, n_blocks, H_kv, B), box 64 x 32 x 1 x 1
+};
+
+// One thread: the two TMA boxes (dims 0-63, 64-127) of ring item i into its
+// slot, completing on the slot's mbarrier.  Rows past the end of the history
+// (or of the complete blocks) are zero-filled by the copy.
+__device__ __forceinline__ const CUtensorMap* locate_item(const Maps& m, const Plan& p, int i, const int* chosen,
+                                                         int block, int& y, int& z) {
+    int j = i;
+    const CUtensorMap* map;
+    if (j >= p.nci && j < p.nci + 2 * p.nwi) {  // window rows
+        j -= p.nci;
+        const bool isv = j >= p.nwi;
+        if (isv) j -= p.nwi;
+        map = isv ? &m.V : &m.K;
+        y = p.kvh;
+        z = p.w_lo + kRows * (p.r + kC * j);
+    } else if (j < p.nA) {  // compressed rows
+        const bool isv = j >= p.nci;
+        if (isv) j -= p.nci + 2 * p.nwi;
+        map = isv ? &m.Vc : &m.Kc;
+        y = p.n_lo + kRows * j;
+        z = p.kvh;
+    } else {  // rows of the selected blocks
+        j -= p.nA;
+        const bool isv = j >= p.nsi;
+        if (isv) j -= p.nsi;
+        map = isv ? &m.V : &m.K;
+        y = p.kvh;
+        z = chosen[p.r + kC * (j / p.ipb)] * block + kRows * (j % p.ipb);
     }
+    return map;
 }
 
-// Scores of one item: S^T[32 rows x GP heads] = rows . Q^T on warps
-// (m-tile, n-tile) < (2, NT); results (log2 units) into dst[h][pos0 + row],
+__device__ __forceinline__ void issue_item(const Maps& m, const Plan& p, int i, uint8_t* ring, uint64_t* full,
+                                           const int* chosen, int block) {
+    const int slot = i % kStages;
+    uint8_t* dst = ring + slot * kItemB;
+    mbar_arrive_expect_tx(&full[slot], kItemB);
+    int y, z;
+    const CUtensorMap* map = locate_item(m, p, i, chosen, block, y, z);
+    tma_load_4d(dst, map, &full[slot], 0, y, z, p.b);
+    tma_load_4d(dst + kHalfB, map, &full[slot], 64, y, z, p.b);
+}
+
+// Scores of one item: S^T[32 rows x GP heads] = rows . Q^T, split over the
+// 8 warps as (m-tile = warp & 1) x (quarter of the 128 dims = warp >> 1).
+// The first quarter's warp adds the three other partial fragments in order
+// (deterministic), then writes the scores (log2 units) to dst[h][pos0 + row],
 // -inf where the row does not exist.
 template <int NT>
-__device__ __forceinline__ void item_scores(uint32_t item_s, const uint32_t (&qb)[8][2], float* dst, int ld,
-                                            int pos0, int nvalid_rows, float c2, int warp, int lane) {
-    if (warp >= 2 * NT) return;
-    const int mt = warp & 1, nt = warp >> 1;
-    const int g = lane >> 2, c4 = lane & 3;
-    const uint32_t abase =
-        item_s + static_cast<uint32_t>((16 * mt + (lane & 7) + ((lane >> 3) & 1) * 8) * kRowB + (lane >> 4) * 16);
-    float d[4] = {0.f, 0.f, 0.f, 0.f};
+__device__ __forceinline__ void item_scores(uint32_t item_s, const uint32_t (&qb)[2][NT][2], float4* part, float* dst,
+                                            int ld, int pos0, int nvalid_rows, float c2, int warp, int lane) {
+    const int mt = warp & 1, kq = warp >> 1;
+    const int R = 16 * mt + (lane & 7) + ((lane >> 3) & 1) * 8;
+    const uint32_t hbase = item_s + static_cast<uint32_t>((kq >> 1) * kHalfB);
+    const int c0 = (kq & 1) * 4 + (lane >> 4);
+    float d[NT][4];
 #pragma unroll
-    for (int kk = 0; kk < 8; ++kk) {
+    for (int nt = 0; nt < NT; ++nt) d[nt][0] = d[nt][1] = d[nt][2] = d[nt][3] = 0.f;
+#pragma unroll
+    for (int s = 0; s < 2; ++s) {
         uint32_t af[4];
-        ldsm_x4(abase + kk * 32, af);
-        mma_bf16_16816(d, af, qb[kk][0], qb[kk][1]);
+        ldsm_x4(hbase + swz(R, c0 + 2 * s), af);
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(d[nt], af, qb[s][nt][0], qb[s][nt][1]);
     }
+    if (kq != 0) {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+            part[(((kq - 1) * 2 + mt) * NT + nt) * 32 + lane] = make_float4(d[nt][0], d[nt][1], d[nt][2], d[nt][3]);
+        named_arrive(1 + mt, 128);
+        return;
+    }
+    named_sync(1 + mt, 128);
+    const int g = lane >> 2, c4 = lane & 3;
     const int r0 = 16 * mt + g, r1 = r0 + 8;
-    const int h0 = 8 * nt + 2 * c4;
-    dst[h0 * ld + pos0 + r0] = r0 < nvalid_rows ? d[0] * c2 : -INFINITY;
-    dst[(h0 + 1) * ld + pos0 + r0] = r0 < nvalid_rows ? d[1] * c2 : -INFINITY;
-    dst[h0 * ld + pos0 + r1] = r1 < nvalid_rows ? d[2] * c2 : -INFINITY;
-    dst[(h0 + 1) * ld + pos0 + r1] = r1 < nvalid_rows ? d[3] * c2 : -INFINITY;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+        for (int q = 1; q < 4; ++q) {
+            const float4 v = part[(((q - 1) * 2 + mt) * NT + nt) * 32 + lane];
+            d[nt][0] += v.x;
+            d[nt][1] += v.y;
+            d[nt][2] += v.z;
+            d[nt][3] += v.w;
+        }
+        const int h0 = 8 * nt + 2 * c4;
+        dst[h0 * ld + pos0 + r0] = r0 < nvalid_rows ? d[nt][0] * c2 : -INFINITY;
+        dst[(h0 + 1) * ld + pos0 + r0] = r0 < nvalid_rows ? d[nt][1] * c2 : -INFINITY;
+        dst[h0 * ld + pos0 + r1] = r1 < nvalid_rows ? d[nt][2] * c2 : -INFINITY;
+        dst[(h0 + 1) * ld + pos0 + r1] = r1 < nvalid_rows ? d[nt][3] * c2 : -INFINITY;
+    }
 }
 
 // O^T[16 dims of this warp x GP heads] += rows^T . P^T over one item's 32 rows.
@@ -329,12 +416,12 @@ template <int NT>
 __device__ __forceinline__ void item_pv(uint32_t item_s, const __nv_bfloat16* P, int ldp, int pos0, float (&acc)[NT][4],
                                         int warp, int lane) {
     const int g = lane >> 2, c4 = lane & 3;
-    const uint32_t vbase = item_s + static_cast<uint32_t>(((lane & 7) + ((lane >> 4) & 1) * 8) * kRowB +
-                                                          (16 * warp + ((lane >> 3) & 1) * 8) * 2);
+    const uint32_t hbase = item_s + static_cast<uint32_t>((warp >> 2) * kHalfB);
+    const int c = 2 * (warp & 3) + ((lane >> 3) & 1);
 #pragma unroll
     for (int ks = 0; ks < 2; ++ks) {
         uint32_t af[4];
-        ldsm_x4_trans(vbase + ks * 16 * kRowB, af);
+        ldsm_x4_trans(hbase + swz(16 * ks + (lane & 7) + ((lane >> 4) & 1) * 8, c), af);
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
             const __nv_bfloat16* pr = P + (8 * nt + g) * ldp + pos0 + 16 * ks + 2 * c4;
@@ -344,30 +431,38 @@ __device__ __forceinline__ void item_pv(uint32_t item_s, const __nv_bfloat16* P,
     }
 }
 
-__device__ __forceinline__ float ld_cluster_f32(uint32_t addr) { return __uint_as_float(ld_cluster_u32(addr)); }
-
 template <int NT>
-__global__ void __cluster_dims__(kC, 1, 1) __launch_bounds__(kThreads, 2) nsa_decode_kernel(const NsaArgs a) {
+__global__ void __cluster_dims__(kC, 1, 1) __launch_bounds__(kThreads, 2)
+    nsa_decode_kernel(const __grid_constant__ Maps maps, const NsaArgs a) {
     constexpr int GP = 8 * NT;
-    extern __shared__ __align__(128) uint8_t smem[];
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    __shared__ __align__(8) uint64_t s_full[kStages];
     __shared__ float s_m[3][kMaxG], s_l[3][kMaxG];  // per branch (compression, selection, window) and head
     __shared__ float s_lsel[kMaxG], s_fac[kMaxG];
-    __shared__ float s_pub_m[kMaxG], s_pub_L[kMaxG];  // read by the other CTAs of the cluster
-    __shared__ unsigned long long s_pub_top[kMaxTop];
+    __shared__ float s_allm[kC][kMaxG], s_allL[kC][kMaxG];  // compression statistics pushed by the cluster
+    __shared__ unsigned long long s_ctop[kMaxTop], s_gtop[kMaxTop];
     __shared__ int s_chosen[kMaxTop];
-    __shared__ int s_nch;
+    __shared__ float s_gate[kMaxG][3];
+    __shared__ int s_abort;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int G = a.G;
-    const Smem sp = smem_plan(GP, a.per, a.ftok, a.top);
-    const uint32_t ring_s = smem_u32(smem);
+    const Smem sp = smem_plan(G, a.per, a.ftok, a.top);
+    uint8_t* ring = smem;
+    const uint32_t ring_s = smem_u32(ring);
     float* s_sc = reinterpret_cast<float*>(smem + sp.sc);
     __nv_bfloat16* s_pc = reinterpret_cast<__nv_bfloat16*>(smem + sp.pc);
     float* s_sf = reinterpret_cast<float*>(smem + sp.sf);
     __nv_bfloat16* s_pf = reinterpret_cast<__nv_bfloat16*>(smem + sp.pf);
+    float4* part = reinterpret_cast<float4*>(smem + sp.part);
     unsigned long long* keyw = reinterpret_cast<unsigned long long*>(smem + sp.keyw);
     unsigned long long* cand = reinterpret_cast<unsigned long long*>(smem + sp.cand);
     unsigned long long* glob = reinterpret_cast<unsigned long long*>(smem + sp.glob);
+    float* recv = reinterpret_cast<float*>(smem + sp.recv);
+    float* recv_ml = reinterpret_cast<float*>(smem + sp.recv_ml);
+
+    cluster_arrive_relaxed();  // this CTA has started; the matching wait precedes the first push into another CTA
 
     Plan p;
     p.r = static_cast<int>(cluster_rank());
@@ -404,17 +499,31 @@ __global__ void __cluster_dims__(kC, 1, 1) __launch_bounds__(kThreads, 2) nsa_de
         s_m[tid / kMaxG][tid % kMaxG] = -INFINITY;
         s_l[tid / kMaxG][tid % kMaxG] = 0.f;
     }
-    __syncthreads();
-    uint32_t qb[8][2];
-    {
-        const int nt = (warp >> 1) < NT ? (warp >> 1) : 0;
-        const uint8_t* qr = smem + sp.q + (8 * nt + (lane >> 2)) * kRowB + (lane & 3) * 4;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-            qb[kk][0] = *reinterpret_cast<const uint32_t*>(qr + kk * 32);
-            qb[kk][1] = *reinterpret_cast<const uint32_t*>(qr + kk * 32 + 16);
-        }
+    if (tid < kMaxTop) s_ctop[tid] = 0ull;
+    if (tid < 3 * G) s_gate[tid / 3][tid % 3] = a.gates[qrow0 * 3 + tid];
+    if (tid == 0) {
+        tma_prefetch_desc(&maps.K);
+        tma_prefetch_desc(&maps.V);
+        tma_prefetch_desc(&maps.Kc);
+        tma_prefetch_desc(&maps.Vc);
+        for (int i = 0; i < kStages; ++i) mbar_init(&s_full[i], 1);
+        fence_mbar_init();
+        s_abort = 0;
     }
+    __syncthreads();
+    uint32_t qb[2][NT][2];
+    {
+        const int kq = warp >> 1;
+#pragma unroll
+        for (int s = 0; s < 2; ++s)
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                const uint8_t* qr = smem + sp.q + (8 * nt + (lane >> 2)) * kRowB + (16 * (2 * kq + s) + 2 * (lane & 3)) * 2;
+                qb[s][nt][0] = *reinterpret_cast<const uint32_t*>(qr);
+                qb[s][nt][1] = *reinterpret_cast<const uint32_t*>(qr + 16);
+            }
+    }
+    const WaitCtx wc{a.err, &s_abort};
 
     float acc_c[NT][4], acc_s[NT][4], acc_w[NT][4];
 #pragma unroll
@@ -423,145 +532,156 @@ __global__ void __cluster_dims__(kC, 1, 1) __launch_bounds__(kThreads, 2) nsa_de
         for (int e = 0; e < 4; ++e) acc_c[nt][e] = acc_s[nt][e] = acc_w[nt][e] = 0.f;
 
     bool ready = false;  // the selected blocks are known
-    int issued = 0;
+    int issued = 0;      // the same count in every thread; warp 0 issues
     auto top_up = [&](int limit) {
         while (issued < limit && issued < p.n_items && (issued < p.nA || ready)) {
-            issue_item(a, p, issued, ring_s, s_chosen);
-            cp_async_commit();
+            if (tid == 0) issue_item(maps, p, issued, ring, s_full, s_chosen, a.block);
             ++issued;
         }
     };
 
-    // Compression softmax, the cluster's exchange of its statistics, the
-    // group's block probabilities and the shared choice of blocks; also the
-    // window softmax (its scores are complete by then).
-    auto choose = [&]() {
-        __syncthreads();
-        branch_softmax(s_sf, sp.ld_sf, s_pf, sp.ld_pf, kRows * p.nwi, G, GP, false, s_m[2], s_l[2], nullptr, warp,
-                       lane);
-        branch_softmax(s_sc, sp.ld_sc, s_pc, sp.ld_pc, kRows * p.nci, G, GP, true, s_m[0], s_l[0], s_lsel, warp,
-                       lane);
-        __syncthreads();
-        if (tid < kMaxG) {
-            s_pub_m[tid] = tid < G ? s_m[0][tid] : -INFINITY;
-            s_pub_L[tid] = tid < G ? s_lsel[tid] : 0.f;
-        }
-        cluster_sync_all();
-        if (tid < G) {
-            float mr[kC], Lr[kC];
-            float M = -INFINITY;
-#pragma unroll
-            for (int rr = 0; rr < kC; ++rr) {
-                mr[rr] = ld_cluster_f32(mapa_u32(smem_u32(&s_pub_m[tid]), rr));
-                Lr[rr] = ld_cluster_f32(mapa_u32(smem_u32(&s_pub_L[tid]), rr));
-                M = fmaxf(M, mr[rr]);
+    // The group's choice of blocks, in three steps placed between ring items
+    // so that the cluster's exchanges overlap the streaming of window and
+    // compressed-value rows:
+    //  E1 (after the compressed keys): compression softmax; every CTA's
+    //     per-head (max, sum) pushed to every CTA of the cluster; arrive.
+    //  E2 (after the window keys): window softmax; wait; the group's block
+    //     probabilities of this chunk; its top blocks (warp sorts, then a
+    //     merge of the warps' lists) pushed to every CTA; arrive.
+    //  E3 (after the window values): wait; merge of the CTAs' lists into the
+    //     group's top blocks, ascending -> the selected-block rows may load.
+    const int e1 = p.nci, e2 = p.nci + p.nwi, e3 = p.nci + 2 * p.nwi;
+    int p2 = 1;
+    while (p2 <= ntop) p2 <<= 1;
+    auto events = [&](int done) {
+        if (done == e1) {
+            __syncthreads();
+            branch_softmax(s_sc, sp.ld_sc, s_pc, sp.ld_pc, kRows * p.nci, G, GP, true, s_m[0], s_l[0], s_lsel, warp,
+                           lane);
+            __syncthreads();
+            cluster_wait();  // every CTA of the cluster has started
+            for (int t = tid; t < kC * G; t += kThreads) {
+                const uint32_t dst = static_cast<uint32_t>(t / G), h = static_cast<uint32_t>(t % G);
+                st_cluster_u32(mapa_u32(smem_u32(&s_allm[p.r][h]), dst), __float_as_uint(s_m[0][h]));
+                st_cluster_u32(mapa_u32(smem_u32(&s_allL[p.r][h]), dst), __float_as_uint(s_lsel[h]));
             }
-            float Lt = 0.f;
+            cluster_arrive();
+        }
+        if (done == e2) {
+            __syncthreads();
+            branch_softmax(s_sf, sp.ld_sf, s_pf, sp.ld_pf, kRows * p.nwi, G, GP, false, s_m[2], s_l[2], nullptr,
+                           warp, lane);
+            cluster_wait();
+            if (tid < G) {
+                float M = -INFINITY;
 #pragma unroll
-            for (int rr = 0; rr < kC; ++rr)
-                if (mr[rr] != -INFINITY) Lt += Lr[rr] * exp2f(mr[rr] - M);
-            const float mine = s_m[0][tid];
-            s_fac[tid] = (mine != -INFINITY && Lt > 0.f) ? exp2f(mine - M) / Lt : 0.f;
-        }
-        __syncthreads();
-        // the group's probability of each block of this chunk, as a key
-        for (int n = tid; n < kRows * p.nci; n += kThreads) {
-            unsigned long long k = 0ull;
-            if (n < nvc) {
-                float pg = 0.f;
-                for (int h = 0; h < G; ++h) pg += s_sc[h * sp.ld_sc + n] * s_fac[h];
-                k = block_key(pg, p.n_lo + n);
+                for (int rr = 0; rr < kC; ++rr) M = fmaxf(M, s_allm[rr][tid]);
+                float Lt = 0.f;
+#pragma unroll
+                for (int rr = 0; rr < kC; ++rr)
+                    Lt += s_allm[rr][tid] == -INFINITY ? 0.f : s_allL[rr][tid] * fast_exp2(s_allm[rr][tid] - M);
+                const float mine = s_m[0][tid];
+                s_fac[tid] = (mine != -INFINITY && Lt > 0.f) ? fast_exp2(mine - M) / Lt : 0.f;
             }
-            keyw[n] = k;
-        }
-        __syncthreads();
-        if (ntop > 0) {
-            const int span = kRows * p.nci;
-            const int sl = (span + kWarps - 1) / kWarps;
-            const int lo = min(span, warp * sl);
-            warp_top(keyw + lo, min(span, lo + sl) - lo, ntop, cand + warp * ntop, lane);
-        }
-        __syncthreads();
-        if (warp == 0 && ntop > 0) warp_top(cand, kWarps * ntop, ntop, s_pub_top, lane);
-        cluster_sync_all();
-        if (warp == 0) {
+            __syncthreads();
+            // the group's probability of each block of this chunk, as a key (0: no block)
+            for (int n = tid; n < a.per; n += kThreads) {
+                unsigned long long k = 0ull;
+                if (n < nvc) {
+                    float pg = 0.f;
+                    for (int h = 0; h < G; ++h) pg += s_sc[h * sp.ld_sc + n] * s_fac[h];
+                    k = block_key(pg, p.n_lo + n);
+                }
+                keyw[n] = k;
+            }
+            __syncthreads();
             if (ntop > 0) {
-                for (int j = lane; j < kC * ntop; j += 32) {
-                    const uint32_t ra = mapa_u32(smem_u32(&s_pub_top[j % ntop]), static_cast<uint32_t>(j / ntop));
-                    const uint32_t lo = ld_cluster_u32(ra), hi = ld_cluster_u32(ra + 4);
-                    glob[j] = (static_cast<unsigned long long>(hi) << 32) | lo;
+                const int kw = a.per / kWarps;  // 4 .. 64 keys per warp
+                const unsigned long long* src = keyw + warp * kw;
+                unsigned long long v0 = lane < kw ? src[lane] : 0ull;
+                unsigned long long v1 = lane + 32 < kw ? src[lane + 32] : 0ull;
+                if (kw > 32) warp_sort_desc<true>(v0, v1, lane);
+                else warp_sort_desc<false>(v0, v1, lane);
+                if (lane < ntop) cand[warp * ntop + lane] = v0;
+                if (lane + 32 < ntop) cand[warp * ntop + lane + 32] = kw > 32 ? v1 : 0ull;
+                __syncthreads();
+                for (int c = tid; c < kWarps * ntop; c += kThreads) {
+                    const unsigned long long x = cand[c];
+                    if (x == 0ull) continue;
+                    const int rank = rank_in_lists(cand, ntop, p2, c / ntop, c % ntop, x);
+                    if (rank < ntop) s_ctop[rank] = x;
                 }
-                __syncwarp();
-                warp_top(glob, kC * ntop, ntop, cand, lane);
-                __syncwarp();
-                if (lane == 0) {
-                    int nch = 0;
-                    for (int j = 0; j < ntop; ++j) {
-                        if (cand[j] == 0ull) continue;
-                        const int v = key_block(cand[j]);
-                        int t = nch++;
-                        while (t > 0 && s_chosen[t - 1] > v) {
-                            s_chosen[t] = s_chosen[t - 1];
-                            --t;
-                        }
-                        s_chosen[t] = v;
-                    }
-                    s_nch = nch;
+                __syncthreads();
+                for (int t = tid; t < kC * ntop; t += kThreads) {
+                    const uint32_t dst = static_cast<uint32_t>(t / ntop);
+                    const int j = t % ntop;
+                    st_cluster_u64(mapa_u32(smem_u32(glob + p.r * ntop + j), dst), s_ctop[j]);
                 }
-            } else if (lane == 0) {
-                s_nch = 0;
             }
+            cluster_arrive();
         }
-        __syncthreads();
-        if (p.r == 0 && a.sel != nullptr && tid < a.top)
-            a.sel[(static_cast<int64_t>(p.b) * a.Hkv + p.kvh) * a.top + tid] = tid < s_nch ? s_chosen[tid] : -1;
-        ready = true;
-    };
-
-    top_up(kStages - 1);
-    if (p.nwi + p.nci == 0) {
-        choose();
-        top_up(kStages - 1);
-    }
-    for (int i = 0; i < p.n_items; ++i) {
-        cp_async_wait_n(issued - i - 1);
-        __syncthreads();
-        top_up(i + kStages);  // into the slot of item i - 1
-        const uint32_t item_s = ring_s + static_cast<uint32_t>((i % kStages) * kItemB);
-        if (i < p.nwi) {
-            const int t0 = p.w_lo + kRows * (p.r + kC * i);
-            item_scores<NT>(item_s, qb, s_sf, sp.ld_sf, kRows * i, a.L - t0, c2, warp, lane);
-        } else if (i < p.nwi + p.nci) {
-            const int j = i - p.nwi;
-            item_scores<NT>(item_s, qb, s_sc, sp.ld_sc, kRows * j, nvc - kRows * j, c2, warp, lane);
-        } else if (i < 2 * p.nwi + p.nci) {
-            item_pv<NT>(item_s, s_pf, sp.ld_pf, kRows * (i - p.nwi - p.nci), acc_w, warp, lane);
-        } else if (i < p.nA) {
-            item_pv<NT>(item_s, s_pc, sp.ld_pc, kRows * (i - 2 * p.nwi - p.nci), acc_c, warp, lane);
-        } else if (i < p.nA + p.nsi) {
-            item_scores<NT>(item_s, qb, s_sf, sp.ld_sf, kRows * (i - p.nA), kRows, c2, warp, lane);
-        } else {
-            item_pv<NT>(item_s, s_pf, sp.ld_pf, kRows * (i - p.nA - p.nsi), acc_s, warp, lane);
+        if (done == e3) {
+            cluster_wait();
+            if (ntop > 0) {
+                for (int c = tid; c < kC * ntop; c += kThreads) {
+                    const unsigned long long x = glob[c];
+                    if (x == 0ull) continue;
+                    const int rank = rank_in_lists(glob, ntop, p2, c / ntop, c % ntop, x);
+                    if (rank < ntop) s_gtop[rank] = x;
+                }
+                __syncthreads();
+                if (tid < ntop) {
+                    const int blk = key_block(s_gtop[tid]);
+                    int at = 0;
+                    for (int u = 0; u < ntop; ++u) at += key_block(s_gtop[u]) < blk;
+                    s_chosen[at] = blk;
+                }
+            }
+            __syncthreads();
+            if (p.r == 0 && a.sel != nullptr && tid < a.top)
+                a.sel[(static_cast<int64_t>(p.b) * a.Hkv + p.kvh) * a.top + tid] = tid < ntop ? s_chosen[tid] : -1;
+            ready = true;
         }
-        if (i + 1 == p.nwi + p.nci) {
-            choose();
-            top_up(i + kStages);
-        }
-        if (p.nsi > 0 && i + 1 == p.nA + p.nsi) {
+        if (p.nsi > 0 && done == p.nA + p.nsi) {
             __syncthreads();
             branch_softmax(s_sf, sp.ld_sf, s_pf, sp.ld_pf, kRows * p.nsi, G, GP, false, s_m[1], s_l[1], nullptr, warp,
                            lane);
         }
-    }
-    __syncthreads();  // every item consumed: the ring holds the partial states now
+    };
 
-    float* pm = reinterpret_cast<float*>(smem);  // [3][kMaxG]
-    float* pl = pm + 3 * kMaxG;                  // [3][kMaxG]
-    float* po = pl + 3 * kMaxG;                  // [3][GP][kD]
-    if (tid < 3 * kMaxG) {
-        pm[tid] = s_m[tid / kMaxG][tid % kMaxG];
-        pl[tid] = s_l[tid / kMaxG][tid % kMaxG];
+    top_up(kStages - 1);
+    events(0);
+    top_up(kStages - 1);
+    for (int i = 0; i < p.n_items; ++i) {
+        const int slot = i % kStages;
+        const bool got = warp_wait(&s_full[slot], static_cast<uint32_t>((i / kStages) & 1), wc, kErrNsaWait | slot);
+        const bool ok = __syncthreads_and(got) != 0;  // also: every warp is done with item i - 1
+        top_up(i + kStages);                           // into the slot of item i - 1
+        const uint32_t item_s = ring_s + static_cast<uint32_t>(slot * kItemB);
+        if (ok) {
+            if (i < e1) {
+                item_scores<NT>(item_s, qb, part, s_sc, sp.ld_sc, kRows * i, nvc - kRows * i, c2, warp, lane);
+            } else if (i < e2) {
+                const int j = i - e1;
+                const int t0 = p.w_lo + kRows * (p.r + kC * j);
+                item_scores<NT>(item_s, qb, part, s_sf, sp.ld_sf, kRows * j, a.L - t0, c2, warp, lane);
+            } else if (i < e3) {
+                item_pv<NT>(item_s, s_pf, sp.ld_pf, kRows * (i - e2), acc_w, warp, lane);
+            } else if (i < p.nA) {
+                item_pv<NT>(item_s, s_pc, sp.ld_pc, kRows * (i - e3), acc_c, warp, lane);
+            } else if (i < p.nA + p.nsi) {
+                item_scores<NT>(item_s, qb, part, s_sf, sp.ld_sf, kRows * (i - p.nA), kRows, c2, warp, lane);
+            } else {
+                item_pv<NT>(item_s, s_pf, sp.ld_pf, kRows * (i - p.nA - p.nsi), acc_s, warp, lane);
+            }
+        }
+        events(i + 1);
+        if (i + 1 == e3) top_up(i + kStages);
     }
+    __syncthreads();  // every item consumed: the ring is free for the partial outputs
+
+    // partial outputs to this CTA's shared memory, then pushed to the CTA that finishes each head
+    float* po = reinterpret_cast<float*>(ring);  // [3][GP][kD]
     {
         const int g = lane >> 2, c4 = lane & 3;
         const int d0 = 16 * warp + g;
@@ -578,35 +698,50 @@ __global__ void __cluster_dims__(kC, 1, 1) __launch_bounds__(kThreads, 2) nsa_de
             }
         }
     }
+    __syncthreads();
+    const int hpc = sp.hpc;
+    for (int t = tid; t < 3 * G * 32; t += kThreads) {
+        const int br = t / (G * 32), h = (t / 32) % G, c16 = t % 32;
+        const float4 v = *reinterpret_cast<const float4*>(po + (br * GP + h) * kD + 4 * c16);
+        const uint32_t at = smem_u32(recv + (((p.r * 3 + br) * hpc + h / kC) * kD + 4 * c16));
+        st_cluster_v4(mapa_u32(at, static_cast<uint32_t>(h % kC)), __float_as_uint(v.x), __float_as_uint(v.y),
+                      __float_as_uint(v.z), __float_as_uint(v.w));
+    }
+    for (int t = tid; t < 3 * G; t += kThreads) {
+        const int br = t / G, h = t % G;
+        const uint32_t at = smem_u32(recv_ml + ((p.r * 3 + br) * hpc + h / kC) * 2);
+        const uint32_t dst = static_cast<uint32_t>(h % kC);
+        st_cluster_u32(mapa_u32(at, dst), __float_as_uint(s_m[br][h]));
+        st_cluster_u32(mapa_u32(at + 4, dst), __float_as_uint(s_l[br][h]));
+    }
     cluster_sync_all();
     {
-        const int h = p.r + kC * (tid >> 7), d = tid & (kD - 1);
-        if (h < G) {
+        const int sl = tid >> 7, d = tid & (kD - 1);
+        const int h = p.r + kC * sl;
+        if (sl < hpc && h < G) {
             float res = 0.f;
 #pragma unroll
             for (int br = 0; br < 3; ++br) {
-                float mr[kC];
                 float M = -INFINITY;
 #pragma unroll
-                for (int rr = 0; rr < kC; ++rr) {
-                    mr[rr] = ld_cluster_f32(mapa_u32(smem_u32(pm + br * kMaxG + h), rr));
-                    M = fmaxf(M, mr[rr]);
-                }
+                for (int rr = 0; rr < kC; ++rr) M = fmaxf(M, recv_ml[((rr * 3 + br) * hpc + sl) * 2]);
                 float num = 0.f, den = 0.f;
+                if (M != -INFINITY) {
 #pragma unroll
-                for (int rr = 0; rr < kC; ++rr) {
-                    if (mr[rr] == -INFINITY) continue;
-                    const float w = exp2f(mr[rr] - M);
-                    den += w * ld_cluster_f32(mapa_u32(smem_u32(pl + br * kMaxG + h), rr));
-                    num += w * ld_cluster_f32(mapa_u32(smem_u32(po + (br * GP + h) * kD + d), rr));
+                    for (int rr = 0; rr < kC; ++rr) {
+                        const float mr = recv_ml[((rr * 3 + br) * hpc + sl) * 2];
+                        if (mr == -INFINITY) continue;
+                        const float w = exp2f(mr - M);
+                        den += w * recv_ml[((rr * 3 + br) * hpc + sl) * 2 + 1];
+                        num += w * recv[((rr * 3 + br) * hpc + sl) * kD + d];
+                    }
                 }
                 const float o = den > 0.f ? num / den : 0.f;
-                res += a.gates[(qrow0 + h) * 3 + br] * o;
+                res += s_gate[h][br] * o;
             }
             a.out[(qrow0 + h) * kD + d] = res;
         }
     }
-    cluster_sync_all();  // the other CTAs have read this CTA's partial states
 }
 
 }  // namespace
@@ -633,12 +768,12 @@ int nsa_decode_smem(int G, int L, int block, int top, int window, int* per_out, 
     const int ftok = std::max(1, fitems) * kRows;
     if (per_out) *per_out = per;
     if (ftok_out) *ftok_out = ftok;
-    return smem_plan(G <= 8 ? 8 : 16, per, ftok, top).total;
+    return smem_plan(G, per, ftok, top).total;
 }
 
 sa_status nsa_decode_launch(const void* q, const void* K, const void* V, int64_t sb, int64_t st_, int64_t sh,
                             const void* Kc, const void* Vc, int64_t c_ld, const float* gates, int B, int H, int Hkv,
-                            int L, int block, int top, int window, float scale, float* out, int32_t* sel,
+                            int L, int block, int top, int window, float scale, float* out, int32_t* sel, int* err,
                             cudaStream_t st) {
     NsaArgs a;
     a.q = static_cast<const __nv_bfloat16*>(q);
@@ -653,6 +788,7 @@ sa_status nsa_decode_launch(const void* q, const void* K, const void* V, int64_t
     a.gates = gates;
     a.out = out;
     a.sel = sel;
+    a.err = err;
     a.H = H;
     a.Hkv = Hkv;
     a.G = H / Hkv;
@@ -663,14 +799,33 @@ sa_status nsa_decode_launch(const void* q, const void* K, const void* V, int64_t
     a.scale = scale;
     const int smem = nsa_decode_smem(a.G, L, block, top, window, &a.per, &a.ftok);
     if (smem > kNsaMaxSmem) return SA_EUNSUPPORTED;
+    Maps m;
+    {
+        const uint64_t tdims[4] = {static_cast<uint64_t>(kD), static_cast<uint64_t>(Hkv), static_cast<uint64_t>(L),
+                                   static_cast<uint64_t>(B)};
+        const uint64_t tstr[3] = {static_cast<uint64_t>(sh) * 2, static_cast<uint64_t>(st_) * 2,
+                                  static_cast<uint64_t>(sb) * 2};
+        const uint32_t tbox[4] = {64, 1, kRows, 1};
+        const uint64_t cdims[4] = {static_cast<uint64_t>(kD), static_cast<uint64_t>(std::max(1, L / block)),
+                                   static_cast<uint64_t>(Hkv), static_cast<uint64_t>(B)};
+        const uint64_t cstr[3] = {static_cast<uint64_t>(kD) * 2, static_cast<uint64_t>(c_ld) * kD * 2,
+                                  static_cast<uint64_t>(c_ld) * kD * 2 * Hkv};
+        const uint32_t cbox[4] = {64, kRows, 1, 1};
+        const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+        const CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B;
+        if (!encode_tiled(&m.K, bf, 4, K, tdims, tstr, tbox, sw) || !encode_tiled(&m.V, bf, 4, V, tdims, tstr, tbox, sw) ||
+            !encode_tiled(&m.Kc, bf, 4, Kc, cdims, cstr, cbox, sw) ||
+            !encode_tiled(&m.Vc, bf, 4, Vc, cdims, cstr, cbox, sw))
+            return SA_ECUDA;
+    }
     const unsigned grid = static_cast<unsigned>(B) * Hkv * kC;
     cudaError_t e;
     if (a.G <= 8) {
         e = cudaFuncSetAttribute(nsa_decode_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e == cudaSuccess) nsa_decode_kernel<1><<<grid, kThreads, smem, st>>>(a);
+        if (e == cudaSuccess) nsa_decode_kernel<1><<<grid, kThreads, smem, st>>>(m, a);
     } else {
         e = cudaFuncSetAttribute(nsa_decode_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e == cudaSuccess) nsa_decode_kernel<2><<<grid, kThreads, smem, st>>>(a);
+        if (e == cudaSuccess) nsa_decode_kernel<2><<<grid, kThreads, smem, st>>>(m, a);
     }
     if (e != cudaSuccess) return launch_status(e);
     return launch_status(cudaGetLastError());

@@ -391,7 +391,7 @@ sa_status sa_nsa_decode(const void* q, const void* K, const void* V, int64_t str
         (Kc && !aligned(Kc, 16)) || (Vc && !aligned(Vc, 16)) || stride_b % 8 || stride_t % 8 || stride_h % 8)
         return SA_EINVAL;
     return nsa_decode_launch(q, K, V, stride_b, stride_t, stride_h, Kc ? Kc : K, Vc ? Vc : V, c_ld, gates, B, H,
-                             H_kv, L, block, top_blocks, window, scale, out, sel_blocks,
+                             H_kv, L, block, top_blocks, window, scale, out, sel_blocks, device_error_word(),
                              reinterpret_cast<cudaStream_t>(stream));
 }
 

@@ -24,7 +24,8 @@ enum : int {
     kErrMlaWait = 0x200,   // sparse-MLA kernel waits
     kErrTopkRow = 0x300,   // top-k: invalid row state
     kErrMixedGroup = 0x400,  // indexer: internal grouping inconsistency
-    kErrGemmWait = 0x500     // per-head projection GEMM waits
+    kErrGemmWait = 0x500,    // per-head projection GEMM waits
+    kErrNsaWait = 0x600      // NSA decode waits (low byte = ring slot)
 };
 
 constexpr unsigned long long kWaitLimitNs = 1000ull * 1000ull * 1000ull;  // 1 s

@@ -86,13 +86,13 @@ sa_status block_sparse_launch(const void* q, const float* pooled, int64_t pooled
                               int32_t* sel_blocks, cudaStream_t st);
 
 // NSA three-branch decode (nsa.cu).
-constexpr int kNsaMaxSmem = 227 * 1024;
+constexpr int kNsaMaxSmem = 227 * 1024 - 4096;  // dynamic part; the kernel also has ~3 KB of static shared memory
 sa_status nsa_compress_launch(const void* K, const void* V, int64_t sb, int64_t st_, int64_t sh, int B, int L,
                               int Hkv, int block, void* Kc, void* Vc, int64_t c_ld, cudaStream_t st);
 int nsa_decode_smem(int G, int L, int block, int top, int window, int* per_out, int* ftok_out);
 sa_status nsa_decode_launch(const void* q, const void* K, const void* V, int64_t sb, int64_t st_, int64_t sh,
                             const void* Kc, const void* Vc, int64_t c_ld, const float* gates, int B, int H, int Hkv,
-                            int L, int block, int top, int window, float scale, float* out, int32_t* sel,
+                            int L, int block, int top, int window, float scale, float* out, int32_t* sel, int* err,
                             cudaStream_t st);
 
 }  // namespace sa
