@@ -342,6 +342,55 @@ def nsa_decode_group(q, K, V, block: int, top_blocks: int, window: int, gates, s
 
 
 # --------------------------------------------------------------------------
+# CSA: DSA over m-token compressed entries ([LLMRes] "DeepSeek CSA & HCA";
+# [MLA-S] on DeepSeek-V4's two kinds of attention layer).
+
+def csa_compress(Ca, Cb, Za, Zb, Ba, Bb, m: int) -> np.ndarray:
+    """Compressed entries of one sequence, [LLMRes] CSA.  Ca, Cb, Za, Zb
+    [n, c] (the two streams of entries and their compression weights), Ba, Bb
+    [m, c] (position biases).  Entry i (0 <= i < n // m, complete groups only)
+    merges group i of stream a with group i - 1 of stream b: the 2m weight
+    rows Za[mi : m(i+1)] + Ba and Zb[m(i-1) : mi] + Bb, stacked along the
+    sequence, are normalised by a softmax along the sequence separately for
+    every channel, and weight the matching 2m entry rows, summed.  For i = 0
+    stream b contributes nothing (its weights are -inf, its entries 0).
+    Returns [n // m, c] float64."""
+    Ca, Cb, Za, Zb, Ba, Bb = (_f64(x) for x in (Ca, Cb, Za, Zb, Ba, Bb))
+    n, c = Ca.shape
+    nc = n // m
+    out = np.zeros((nc, c))
+    for i in range(nc):
+        za = Za[m * i: m * (i + 1)] + Ba
+        ca = Ca[m * i: m * (i + 1)]
+        if i == 0:
+            zb, cb = np.full((m, c), -np.inf), np.zeros((m, c))
+        else:
+            zb, cb = Zb[m * (i - 1): m * i] + Bb, Cb[m * (i - 1): m * i]
+        z = np.concatenate([za, zb], axis=0)
+        e = np.exp(z - z.max(axis=0, keepdims=True))
+        wgt = e / e.sum(axis=0, keepdims=True)
+        out[i] = (wgt[:m] * ca).sum(axis=0) + (wgt[m:] * cb).sum(axis=0)
+    return out
+
+
+def csa_attend(q, C_comp, C_raw, chosen, window: int, scale: float):
+    """CSA core attention of one query, [LLMRes] CSA: every head of q [H, c]
+    attends (one softmax, keys = values = the entries) to the chosen
+    compressed entries C_comp[chosen] together with the raw entries of the
+    last `window` positions of C_raw [L, c].  Returns [H, c]."""
+    q, C_comp, C_raw = _f64(q), _f64(C_comp), _f64(C_raw)
+    L = C_raw.shape[0]
+    rows = [C_comp[int(j)] for j in chosen if j >= 0] + [C_raw[t] for t in range(max(0, L - window), L)]
+    if not rows:
+        return np.zeros_like(q)
+    E = np.stack(rows)
+    s = q @ E.T * scale
+    a = np.exp(s - s.max(axis=1, keepdims=True))
+    a /= a.sum(axis=1, keepdims=True)
+    return a @ E
+
+
+# --------------------------------------------------------------------------
 # Whole-step reference on workload tensors (any device; values copied to host)
 
 def _host64(t):
@@ -439,3 +488,29 @@ def nsa_step(inp: dict, pairs: Sequence[tuple]) -> dict:
         res[(b, g)] = nsa_decode_group(_host64(inp["q"][b, hs]), K, V, cfg.block, cfg.top_blocks, cfg.window,
                                        _host64(inp["gates"][b, hs]), cfg.scale, compressed=cache)
     return res
+
+
+def csa_step(inp: dict, rows: Sequence[int]) -> dict:
+    """The CSA decode of the given sequences from the workload's streams:
+    compressed entries (csa_compress; stored as bf16, the indexer keys as
+    e4m3), index scores over the n_c compressed keys, Top-K, then csa_attend
+    over the chosen entries and the raw window.  Returns out [rows, H, c],
+    idx [rows, k], scores [rows, n_c], kv_comp / ki_comp (lists of [n_c, .])."""
+    import torch
+    cfg = inp["cfg"]
+    outs, idxs, scs, kvs, kis = [], [], [], [], []
+    for r in rows:
+        kv = csa_compress(*(_host64(inp[n][r]) for n in ("Ca", "Cb", "Za", "Zb")), _host64(inp["Ba"]),
+                          _host64(inp["Bb"]), cfg.m)
+        kv = torch.from_numpy(kv).to(torch.bfloat16).to(torch.float64).numpy()
+        ki = csa_compress(*(_host64(inp[n][r]) for n in ("CIa", "CIb", "ZIa", "ZIb")), _host64(inp["BIa"]),
+                          _host64(inp["BIb"]), cfg.m)
+        ki = torch.from_numpy(ki).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+        sc = index_scores(_host64(inp["q_idx"][r: r + 1]), _host64(inp["w"][r: r + 1]), ki, [0], [cfg.n_c])
+        sel = topk(sc, [cfg.n_c], cfg.topk)[0]
+        outs.append(csa_attend(_host64(inp["q"][r]), kv, _host64(inp["Ca"][r]), sel, cfg.window, cfg.scale))
+        idxs.append(sel)
+        scs.append(sc[0])
+        kvs.append(kv)
+        kis.append(ki)
+    return dict(out=np.stack(outs), idx=np.stack(idxs), scores=np.stack(scs), kv_comp=kvs, ki_comp=kis)

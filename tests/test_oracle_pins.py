@@ -477,6 +477,112 @@ def test_nsa_compress_stored_cache():
     assert oracle.nsa_compress(X.numpy()[:63], 64).shape == (0, 128)
 
 
+# ------------------------------------------------------------ CSA compression
+
+def _csa_streams(seed, n, c, m):
+    rng = np.random.default_rng(seed)
+    return (rng.standard_normal((n, c)), rng.standard_normal((n, c)), rng.standard_normal((n, c)),
+            rng.standard_normal((n, c)), rng.standard_normal((m, c)), rng.standard_normal((m, c)))
+
+
+def test_csa_uniform_weights_give_the_mean_of_both_groups():
+    """[LLMRes] CSA: equal weights -> entry i is the mean of the 2m rows (group
+    i of stream a, group i-1 of stream b); entry 0 has stream a only."""
+    m, c = 4, 6
+    Ca, Cb, _, _, _, _ = _csa_streams(1, 4 * m + 3, c, m)
+    Z, B = np.zeros_like(Ca), np.zeros((m, c))
+    out = oracle.csa_compress(Ca, Cb, Z, Z, B, B, m)
+    assert out.shape == (4, c)                               # the ragged tail forms no entry
+    np.testing.assert_allclose(out[0], Ca[:m].mean(axis=0), atol=1e-14)
+    for i in range(1, 4):
+        want = np.concatenate([Ca[m * i: m * (i + 1)], Cb[m * (i - 1): m * i]]).mean(axis=0)
+        np.testing.assert_allclose(out[i], want, atol=1e-14)
+
+
+def test_csa_weights_follow_the_logits_and_the_biases():
+    """Weight logits log(1..2m) (through Z or through the position biases)
+    give weights proportional to 1..2m: a closed form per channel."""
+    m, c = 4, 3
+    Ca, Cb, _, _, _, _ = _csa_streams(2, 3 * m, c, m)
+    lw = np.log(np.arange(1, 2 * m + 1, dtype=np.float64))
+    wts = np.arange(1, 2 * m + 1) / np.arange(1, 2 * m + 1).sum()
+    Za = np.tile(lw[:m, None], (3, c))
+    Zb = np.tile(lw[m:, None], (3, c))
+    zero = np.zeros((m, c))
+    via_z = oracle.csa_compress(Ca, Cb, Za, Zb, zero, zero, m)
+    via_b = oracle.csa_compress(Ca, Cb, np.zeros_like(Ca), np.zeros_like(Cb), np.tile(lw[:m, None], (1, c)),
+                                np.tile(lw[m:, None], (1, c)), m)
+    for i in (1, 2):
+        want = wts[:m] @ Ca[m * i: m * (i + 1)] + wts[m:] @ Cb[m * (i - 1): m * i]
+        np.testing.assert_allclose(via_z[i], want, atol=1e-13)
+        np.testing.assert_allclose(via_b[i], want, atol=1e-13)
+    w0 = np.arange(1, m + 1) / np.arange(1, m + 1).sum()     # entry 0: the softmax over stream a alone
+    np.testing.assert_allclose(via_z[0], w0 @ Ca[:m], atol=1e-13)
+
+
+def test_csa_softmax_is_per_channel_along_the_sequence():
+    """Channel 0 puts all weight on row 0 of stream a, channel 1 on row 1 of
+    stream b: a softmax over channels, or over both axes, fails this."""
+    m, c = 4, 2
+    Ca, Cb, _, _, _, _ = _csa_streams(3, 2 * m, c, m)
+    Za, Zb = np.zeros_like(Ca), np.zeros_like(Cb)
+    Za[m + 0, 0] = 60.0
+    Zb[1, 1] = 60.0
+    zero = np.zeros((m, c))
+    out = oracle.csa_compress(Ca, Cb, Za, Zb, zero, zero, m)
+    assert abs(out[1, 0] - Ca[m, 0]) < 1e-20 + 1e-12 * abs(Ca[m, 0])
+    assert abs(out[1, 1] - Cb[1, 1]) < 1e-20 + 1e-12 * abs(Cb[1, 1])
+
+
+def test_csa_entries_see_only_their_own_groups():
+    """Entry i reads stream a's group i and stream b's group i-1 only: moving
+    any later row (or stream b's group i) leaves entries 0..i unchanged."""
+    m, c = 4, 5
+    Ca, Cb, Za, Zb, Ba, Bb = _csa_streams(4, 6 * m, c, m)
+    ref = oracle.csa_compress(Ca, Cb, Za, Zb, Ba, Bb, m)
+    Ca2, Cb2, Za2, Zb2 = Ca.copy(), Cb.copy(), Za.copy(), Zb.copy()
+    Ca2[3 * m:] += 7.0
+    Za2[3 * m:] -= 3.0
+    Cb2[2 * m:] += 5.0
+    Zb2[2 * m:] += 2.0
+    got = oracle.csa_compress(Ca2, Cb2, Za2, Zb2, Ba, Bb, m)
+    np.testing.assert_array_equal(got[:3], ref[:3])
+    assert np.abs(got[3:] - ref[3:]).min() > 0
+
+
+def test_csa_attention_reduces_to_plain_attention():
+    """Keys = values = the entries: only compressed entries (no window), or
+    only the window, is attention over those rows; both is one softmax over
+    their union."""
+    rng = np.random.default_rng(5)
+    H, c, nc, L = 3, 8, 20, 50
+    q, Cc, Cr = rng.standard_normal((H, c)), rng.standard_normal((nc, c)), rng.standard_normal((L, c))
+    chosen = np.array([1, 4, 7, 19, -1])
+    got = oracle.csa_attend(q, Cc, Cr, chosen, 0, 0.3)
+    E = Cc[[1, 4, 7, 19]]
+    np.testing.assert_allclose(got, _sdpa(q, E, E, 0.3), atol=1e-12)
+    got = oracle.csa_attend(q, Cc, Cr, np.array([-1, -1]), 6, 0.3)
+    np.testing.assert_allclose(got, _sdpa(q, Cr[-6:], Cr[-6:], 0.3), atol=1e-12)
+    got = oracle.csa_attend(q, Cc, Cr, chosen, 6, 0.3)
+    E = np.concatenate([Cc[[1, 4, 7, 19]], Cr[-6:]])
+    np.testing.assert_allclose(got, _sdpa(q, E, E, 0.3), atol=1e-12)
+
+
+def test_csa_workload_indexer_keys_compress_to_their_integers():
+    """The CSA workload's indexer-key streams repeat one integer vector over
+    the 2m rows each entry merges, so compression (weights summing to one)
+    returns exactly that vector and its e4m3 copy is exact."""
+    import workloads
+    cfg = workloads.CSAConfig(name="t", seed=0, n_seqs=2, L=203, H=4, topk=8, window=8)
+    inp = workloads.csa_inputs(cfg, seed=3)
+    res = oracle.csa_step(inp, [0, 1])
+    for r in range(2):
+        want = inp["CIa"][r, :: cfg.m].double().numpy()[: cfg.n_c]
+        np.testing.assert_array_equal(res["ki_comp"][r], want)
+        assert np.abs(want).max() <= 8 and (want == np.round(want)).all()
+    assert res["idx"].shape == (2, 8) and (np.diff(res["idx"], axis=1) > 0).all()
+
+
 # ------------------------------------------------------------ whole step
 
 def test_dsa_step_placement_invariance():

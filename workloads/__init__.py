@@ -132,6 +132,46 @@ class NSAConfig:
         return self.H // self.H_kv
 
 
+@dataclass(frozen=True)
+class CSAConfig:
+    """Shapes of the CSA workload: DSA over m-token compressed entries plus a
+    window of raw entries, one decode query per sequence."""
+    name: str
+    seed: int
+    n_seqs: int
+    L: int                      # raw tokens per sequence
+    m: int = 4                  # tokens per compressed entry
+    c: int = 512                # entry width (keys = values)
+    H: int = 128                # query heads of the core attention
+    H_I: int = 64
+    d_I: int = 128
+    topk: int = 2048
+    window: int = 128
+    int_lo: int = -8
+    int_hi: int = 8
+    w_values: tuple = tuple(2.0 ** e for e in range(-4, 2))
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.c)
+
+    @property
+    def n_c(self) -> int:
+        return self.L // self.m
+
+    @property
+    def idx_pages(self) -> int:       # indexer pool pages per sequence (compressed keys)
+        return max(1, (self.n_c + PAGE - 1) // PAGE)
+
+    @property
+    def n_cap(self) -> int:           # latent positions before the window slots
+        return self.idx_pages * PAGE
+
+    @property
+    def lat_pages(self) -> int:       # latent pool pages per sequence (compressed entries, then window slots)
+        return (self.n_cap + self.window + PAGE - 1) // PAGE
+
+
 def _ragged_lens(seed: int, n: int, lo: int, hi: int) -> tuple:
     rng = np.random.Generator(np.random.PCG64(seed))
     return tuple(int(x) for x in rng.integers(lo, hi + 1, size=n))
@@ -152,6 +192,8 @@ NSA = NSAConfig(name="nsa", seed=1006, B=8, L=131072, H=32, H_kv=4)
 DSA_CONFIGS = {c.name: c for c in (TINY, LONG, RAGGED, PREFILL)}
 BLOCK_CONFIGS = {BLOCK.name: BLOCK}
 NSA_CONFIGS = {NSA.name: NSA}
+CSA = CSAConfig(name="csa", seed=1007, n_seqs=32, L=131072)
+CSA_CONFIGS = {CSA.name: CSA}
 
 
 def small_dsa(base: DSAConfig, **kw) -> DSAConfig:
@@ -255,6 +297,51 @@ def block_inputs(cfg: BlockConfig, device="cpu", seed: Optional[int] = None) -> 
     K = _normal_bf16(g, (cfg.B, cfg.L, cfg.H, cfg.D), dev)
     V = _normal_bf16(g, (cfg.B, cfg.L, cfg.H, cfg.D), dev)
     return dict(cfg=cfg, q=q, K=K, V=V)
+
+
+def csa_inputs(cfg: CSAConfig, device="cpu", seed: Optional[int] = None) -> dict:
+    """Draw every input of the CSA step.
+
+    Entry streams (the two per-token projections the compression merges) and
+    their compression weights, [n_seqs, L, width] bf16, N(0,1): Ca, Cb, Za, Zb
+    (width c) and the indexer-key streams CIa, CIb, ZIa, ZIb (width d_I);
+    position biases Ba, Bb [m, c], BIa, BIb [m, d_I] fp32.  The indexer-key
+    entry streams are integers in [int_lo, int_hi] that repeat over the 2m rows
+    each compressed entry merges (group g of stream a and group g-1 of stream
+    b carry the same integers), so every compressed indexer key is that
+    integer vector exactly and the index scores are exact in fp32.
+    Query side: q_idx [n_seqs, H_I, d_I] e4m3 integers, w powers of two, q
+    [n_seqs, H, c] bf16, q_rope zeros [n_seqs, H, 64].
+    Caches the compression fills: idx_pool [n_seqs * idx_pages * 64, d_I] e4m3
+    and lat_pool [n_seqs * lat_pages * 64, c] bf16, whose window slots
+    (latent positions n_cap .. n_cap + window - 1 of each sequence) hold the
+    raw entries Ca of the last `window` tokens, oldest first."""
+    seed = cfg.seed if seed is None else seed
+    dev = torch.device(device)
+    g = _gen(dev, seed)
+    S, L, m, c, dI = cfg.n_seqs, cfg.L, cfg.m, cfg.c, cfg.d_I
+    Ca, Cb, Za, Zb = (_normal_bf16(g, (S, L, c), dev) for _ in range(4))
+    Ba, Bb = (torch.randn((m, c), generator=g, device=dev) for _ in range(2))
+    n_groups = (L + m - 1) // m
+    V = _ints(g, (S, n_groups + 1, dI), cfg.int_lo, cfg.int_hi, dev)
+    CIa = V[:, :n_groups].repeat_interleave(m, dim=1)[:, :L].to(torch.bfloat16).contiguous()
+    CIb = V[:, 1:n_groups + 1].repeat_interleave(m, dim=1)[:, :L].to(torch.bfloat16).contiguous()
+    ZIa, ZIb = (_normal_bf16(g, (S, L, dI), dev) for _ in range(2))
+    BIa, BIb = (torch.randn((m, dI), generator=g, device=dev) for _ in range(2))
+    q_idx = _ints(g, (S, cfg.H_I, dI), cfg.int_lo, cfg.int_hi, dev).to(torch.float8_e4m3fn)
+    wv = torch.tensor(cfg.w_values, dtype=torch.float32, device=dev)
+    w = wv[torch.randint(0, len(cfg.w_values), (S, cfg.H_I), generator=g, device=dev)].contiguous()
+    q = _normal_bf16(g, (S, cfg.H, c), dev)
+    q_rope = torch.zeros((S, cfg.H, 64), dtype=torch.bfloat16, device=dev)
+    idx_pool = torch.zeros((S * cfg.idx_pages * PAGE, dI), dtype=torch.float8_e4m3fn, device=dev)
+    lat_pool = torch.zeros((S * cfg.lat_pages * PAGE, c), dtype=torch.bfloat16, device=dev)
+    wl = min(cfg.window, L)
+    lat3 = lat_pool.view(S, cfg.lat_pages * PAGE, c)
+    lat3[:, cfg.n_cap: cfg.n_cap + wl] = Ca[:, L - wl:]
+    return dict(cfg=cfg, Ca=Ca, Cb=Cb, Za=Za, Zb=Zb, Ba=Ba, Bb=Bb, CIa=CIa, CIb=CIb, ZIa=ZIa, ZIb=ZIb, BIa=BIa,
+                BIb=BIb, q_idx=q_idx, w=w, q=q, q_rope=q_rope, idx_pool=idx_pool, lat_pool=lat_pool,
+                n_visible=torch.full((S,), cfg.n_c, dtype=torch.int32, device=dev),
+                seq_lens=torch.full((S,), L, dtype=torch.int32, device=dev))
 
 
 def nsa_inputs(cfg: NSAConfig, device="cpu", seed: Optional[int] = None) -> dict:
