@@ -16,6 +16,9 @@
  *   sa_nsa_compress      NSA compressed cache: bf16 block means of K and V
  *   sa_nsa_decode        NSA three branches (compression, group-shared block
  *                        selection, window), each its own softmax, gated sum
+ *   sa_csa_compress      CSA: m-token entries merged by a per-channel softmax
+ *   sa_csa_window_index  CSA: selected compressed entries plus the raw window,
+ *                        as the index list of sa_sparse_mla_decode
  *
  * Sources, cited by page title and section:
  *   [Notes]  "Sparse Attention 数学学习笔记" (echobase-5bl.pages.dev, 2026.09.14)
@@ -323,6 +326,39 @@ sa_status sa_nsa_decode(const void* q, const void* K, const void* V, int64_t str
                         int64_t stride_h, const void* Kc, const void* Vc, int64_t c_ld, const float* gates,
                         int B, int H, int H_kv, int D, int L, int block, int top_blocks, int window, float scale,
                         float* out, int32_t* sel_blocks, sa_stream_t stream);
+
+/*
+ * CSA compressed entries ([LLMRes] "DeepSeek CSA & HCA", CSA): for every
+ * sequence s and entry g in [g0, g1) (g1 <= L / m: complete groups only),
+ *   out[s][g][ch] = sum_{r<m} w_a[r][ch] Ca[s][m g + r][ch]
+ *                 + sum_{r<m} w_b[r][ch] Cb[s][m (g-1) + r][ch]
+ * where, per channel ch, (w_a, w_b) = softmax over the 2m values
+ * (Za[s][m g + r][ch] + Ba[r][ch], Zb[s][m (g-1) + r][ch] + Bb[r][ch]);
+ * for g = 0 the stream-b terms are absent (weight 0).  Sums and softmax in
+ * fp32, the result rounded to nearest bf16, or to e4m3 with saturation.
+ *   Ca, Cb, Za, Zb bf16, element (s, t, ch) at s*seq_stride + t*row_stride + ch
+ *   Ba, Bb [m][c] fp32
+ *   out: element (s, g, ch) at s*out_seq_stride + g*out_row_stride + ch, in
+ *   elements of out_dtype (SA_BF16 or SA_E4M3)
+ * Run for the groups that complete (decode: one group every m tokens).
+ * Supported: c a multiple of 4 up to 8192, m <= 256.
+ */
+sa_status sa_csa_compress(const void* Ca, const void* Cb, const void* Za, const void* Zb, int64_t seq_stride,
+                          int64_t row_stride, const float* Ba, const float* Bb, int n_seqs, int L, int m, int c,
+                          int g0, int g1, void* out, sa_dtype out_dtype, int64_t out_seq_stride,
+                          int64_t out_row_stride, sa_stream_t stream);
+
+/*
+ * CSA core-attention slot list ([LLMRes] CSA: the selected compressed entries
+ * plus the raw entries of a recent window, attended together):
+ *   idx_out[r][j]     = topk_idx[r][j]                          j < k
+ *   idx_out[r][k + j] = j < min(window, raw_len[r]) ? win_base + j : -1   j < window
+ * idx_out [rows][k + window] int32, the index list of sa_sparse_mla_decode
+ * over a latent pool whose positions win_base .. win_base + window - 1 hold
+ * the raw entries of each sequence's last tokens (oldest first).
+ */
+sa_status sa_csa_window_index(const int32_t* topk_idx, int rows, int k, const int32_t* raw_len, int window,
+                              int win_base, int32_t* idx_out, sa_stream_t stream);
 
 #ifdef __cplusplus
 }

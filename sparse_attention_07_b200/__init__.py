@@ -29,7 +29,7 @@ EXPORTS = (
     "sa_sparse_mla_prefill",
     "sa_block_mean_pool", "sa_block_sparse_attn", "sa_sparse_mla_decode_static",
     "sa_dense_mla_workspace_size", "sa_dense_mla_decode", "sa_mla_absorb_query", "sa_mla_up_project",
-    "sa_nsa_compress", "sa_nsa_decode",
+    "sa_nsa_compress", "sa_nsa_decode", "sa_csa_compress", "sa_csa_window_index",
 )
 
 # Size of the library's static device array behind sparse_mla_decode_static
@@ -74,6 +74,8 @@ def lib():
         L.sa_block_sparse_attn.argtypes = [P, P, I64, P, P, I64, I64, I64, I, I, I, I, I, I, I, I, F, P, P, P]
         L.sa_nsa_compress.argtypes = [P, P, I64, I64, I64, I, I, I, I, I, P, P, I64, P]
         L.sa_nsa_decode.argtypes = [P, P, P, I64, I64, I64, P, P, I64, P, I, I, I, I, I, I, I, I, F, P, P, P]
+        L.sa_csa_compress.argtypes = [P, P, P, P, I64, I64, P, P, I, I, I, I, I, I, P, I, I64, I64, P]
+        L.sa_csa_window_index.argtypes = [P, I, I, P, I, I, P, P]
         for name in EXPORTS:
             if name not in ("sa_status_string", "sa_version", "sa_sparse_mla_workspace_size",
                             "sa_sparse_mla_prefill_workspace_size", "sa_dense_mla_workspace_size"):
@@ -310,3 +312,29 @@ def nsa_decode(q, K, V, Kc, Vc, gates, block: int, top_blocks: int, window: int,
                              top_blocks, window, float(scale), _p(out), _p(sel_blocks), _stream())
     _check("sa_nsa_decode", st)
     return out
+
+
+def csa_compress(Ca, Cb, Za, Zb, Ba, Bb, m: int, out, out_seq_stride: int, out_row_stride: int, g0: int = 0,
+                 g1: Optional[int] = None):
+    """CSA compressed entries g0 .. g1-1 of every sequence: streams [S, L, c]
+    bf16 (one layout for all four), biases [m, c] fp32; written into `out`
+    (bf16 or e4m3) at s*out_seq_stride + g*out_row_stride (elements)."""
+    S, L, c = Ca.shape
+    if not (Cb.stride() == Za.stride() == Zb.stride() == Ca.stride()):
+        raise ValueError("the four streams must share one layout")
+    g1 = L // m if g1 is None else g1
+    code = 1 if out.dtype == torch.float8_e4m3fn else (2 if out.dtype == torch.bfloat16 else -1)
+    st = lib().sa_csa_compress(_p(Ca), _p(Cb), _p(Za), _p(Zb), Ca.stride(0), Ca.stride(1), _p(Ba), _p(Bb), S, L, m,
+                               c, g0, g1, _p(out), code, out_seq_stride, out_row_stride, _stream())
+    _check("sa_csa_compress", st)
+    return out
+
+
+def csa_window_index(topk_idx, raw_len, window: int, win_base: int, idx_out=None):
+    """[rows, k + window] int32: the selected entries, then the window slots."""
+    rows, k = topk_idx.shape
+    if idx_out is None:
+        idx_out = torch.empty(rows, k + window, dtype=torch.int32, device=topk_idx.device)
+    st = lib().sa_csa_window_index(_p(topk_idx), rows, k, _p(raw_len), window, win_base, _p(idx_out), _stream())
+    _check("sa_csa_window_index", st)
+    return idx_out

@@ -395,4 +395,33 @@ sa_status sa_nsa_decode(const void* q, const void* K, const void* V, int64_t str
                              reinterpret_cast<cudaStream_t>(stream));
 }
 
+sa_status sa_csa_compress(const void* Ca, const void* Cb, const void* Za, const void* Zb, int64_t seq_stride,
+                          int64_t row_stride, const float* Ba, const float* Bb, int n_seqs, int L, int m, int c,
+                          int g0, int g1, void* out, sa_dtype out_dtype, int64_t out_seq_stride,
+                          int64_t out_row_stride, sa_stream_t stream) {
+    if (n_seqs < 0 || L < 0 || m < 1 || c < 1 || g0 < 0 || g1 < g0 || g1 > L / m) return SA_EINVAL;
+    if (c % 4 != 0 || c > 8192 || m > 256 || (out_dtype != SA_BF16 && out_dtype != SA_E4M3)) return SA_EUNSUPPORTED;
+    if (n_seqs == 0 || g1 == g0) return SA_OK;
+    if (!Ca || !Cb || !Za || !Zb || !Ba || !Bb || !out) return SA_EINVAL;
+    if (row_stride < c || out_row_stride < c) return SA_EINVAL;
+    const size_t oa = out_dtype == SA_E4M3 ? 4 : 8;
+    if (!aligned(Ca, 8) || !aligned(Cb, 8) || !aligned(Za, 8) || !aligned(Zb, 8) || !aligned(Ba, 16) ||
+        !aligned(Bb, 16) || !aligned(out, oa) || seq_stride % 4 || row_stride % 4 || out_seq_stride % 4 ||
+        out_row_stride % 4)
+        return SA_EINVAL;
+    return csa_compress_launch(Ca, Cb, Za, Zb, seq_stride, row_stride, Ba, Bb, n_seqs, m, c, g0, g1, out,
+                               out_dtype == SA_E4M3 ? 1 : 0, out_seq_stride, out_row_stride,
+                               reinterpret_cast<cudaStream_t>(stream));
+}
+
+sa_status sa_csa_window_index(const int32_t* topk_idx, int rows, int k, const int32_t* raw_len, int window,
+                              int win_base, int32_t* idx_out, sa_stream_t stream) {
+    if (rows < 0 || k < 0 || window < 0 || win_base < 0 || k + window < 1) return SA_EINVAL;
+    if (rows == 0) return SA_OK;
+    if ((k > 0 && !topk_idx) || !raw_len || !idx_out) return SA_EINVAL;
+    if ((topk_idx && !aligned(topk_idx, 4)) || !aligned(raw_len, 4) || !aligned(idx_out, 4)) return SA_EINVAL;
+    return csa_window_index_launch(topk_idx, rows, k, raw_len, window, win_base, idx_out,
+                                   reinterpret_cast<cudaStream_t>(stream));
+}
+
 }  // extern "C"

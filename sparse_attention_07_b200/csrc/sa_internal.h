@@ -95,4 +95,12 @@ sa_status nsa_decode_launch(const void* q, const void* K, const void* V, int64_t
                             int L, int block, int top, int window, float scale, float* out, int32_t* sel, int* err,
                             cudaStream_t st);
 
+// CSA compression and window slots (csa.cu).
+sa_status csa_compress_launch(const void* Ca, const void* Cb, const void* Za, const void* Zb, int64_t seq_stride,
+                              int64_t row_stride, const float* Ba, const float* Bb, int n_seqs, int m, int c, int g0,
+                              int g1, void* out, int out_e4m3, int64_t out_seq_stride, int64_t out_row_stride,
+                              cudaStream_t st);
+sa_status csa_window_index_launch(const int32_t* topk_idx, int rows, int k, const int32_t* raw_len, int window,
+                                  int win_base, int32_t* idx_out, cudaStream_t st);
+
 }  // namespace sa

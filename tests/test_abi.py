@@ -170,5 +170,34 @@ def test_nsa_validation(L):
     assert g(FAKE, FAKE, 8, 8, 128, 2, 63, 4, 128, 64, None, None, 0, None) == sa.SA_OK       # no complete block
 
 
+def test_csa_validation(L):
+    f = L.sa_csa_compress
+    args = dict(Ca=FAKE, Cb=FAKE, Za=FAKE, Zb=FAKE, ss=1024 * 512, rs=512, Ba=FAKE, Bb=FAKE, S=2, L=1024, m=4, c=512,
+                g0=0, g1=256, out=FAKE, dt=sa.SA_BF16, oss=256 * 512, ors=512)
+
+    def call(**kw):
+        a = {**args, **kw}
+        return f(a["Ca"], a["Cb"], a["Za"], a["Zb"], a["ss"], a["rs"], a["Ba"], a["Bb"], a["S"], a["L"], a["m"],
+                 a["c"], a["g0"], a["g1"], a["out"], a["dt"], a["oss"], a["ors"], None)
+
+    assert call(S=0) == sa.SA_OK
+    assert call(g0=5, g1=5) == sa.SA_OK
+    assert call(g1=257) == sa.SA_EINVAL                 # past the complete groups
+    assert call(g0=-1) == sa.SA_EINVAL
+    assert call(m=0) == sa.SA_EINVAL
+    assert call(c=510) == sa.SA_EUNSUPPORTED
+    assert call(dt=sa.SA_F32) == sa.SA_EUNSUPPORTED
+    assert call(rs=256) == sa.SA_EINVAL                 # rows overlap
+    assert call(Za=None) == sa.SA_EINVAL
+    assert call(Ba=MISALIGNED) == sa.SA_EINVAL
+    assert call(ors=514) == sa.SA_EINVAL
+    g = L.sa_csa_window_index
+    assert g(FAKE, 0, 16, FAKE, 8, 64, FAKE, None) == sa.SA_OK
+    assert g(FAKE, 2, 0, FAKE, 0, 64, FAKE, None) == sa.SA_EINVAL     # no slot at all
+    assert g(None, 2, 16, FAKE, 8, 64, FAKE, None) == sa.SA_EINVAL
+    assert g(FAKE, 2, 16, FAKE, -1, 64, FAKE, None) == sa.SA_EINVAL
+    assert g(FAKE, 2, 16, None, 8, 64, FAKE, None) == sa.SA_EINVAL
+
+
 def test_check_device_error_rejects_null(L):
     assert L.sa_check_device_error(None, None) == sa.SA_EINVAL
