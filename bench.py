@@ -4,7 +4,7 @@
 One step = the whole decode path over one batch: lightning indexer ->
 exact Top-K -> sparse MLA, i.e. one query per sequence of the workload.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--config long|ragged|tiny|prefill|block|nsa|crossover]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config long|ragged|tiny|prefill|block|nsa|csa|crossover]
                     [--impl native|reference]
 
 Default workload: long decode, 32 sequences x 32768 tokens, H^I=64 fp8
@@ -84,6 +84,16 @@ def nsa_bytes(cfg: W.NSAConfig):
     per_group = (2 * nb * cfg.D * 2 + min(cfg.top_blocks, nb) * cfg.block * 2 * cfg.D * 2
                  + min(cfg.window, cfg.L) * 2 * cfg.D * 2 + cfg.G * (cfg.D * 2 + 12 + cfg.D * 4))
     return per_group * cfg.B * cfg.H_kv
+
+
+def csa_bytes(cfg: W.CSAConfig):
+    """Algorithmic bytes of one CSA decode step: every compressed indexer key
+    once (e4m3, d_I bytes), then every selected entry and window slot once
+    (a 512-wide bf16 latent row plus the 64 dims the attention kernel reads
+    as its RoPE key), per sequence."""
+    keys = cfg.n_seqs * cfg.n_c * cfg.d_I
+    rows = cfg.n_seqs * (min(cfg.topk, cfg.n_c) + min(cfg.window, cfg.L)) * (cfg.c + 64) * 2
+    return keys, rows
 
 
 # ---------------------------------------------------------------- ranks
@@ -260,6 +270,70 @@ class NsaStep:
         pass
 
 
+class CsaStep:
+    """indexer over the compressed keys -> Top-K -> window slots + sparse
+    attention over the selected entries and the window."""
+
+    def __init__(self, inp, sa):
+        self.sa, self.inp, self.cfg = sa, inp, inp["cfg"]
+        c, dev = self.cfg, inp["q"].device
+        S = c.n_seqs
+        lat = inp["lat_pool"].view(S, c.lat_pages * 64, c.c)
+        idx = inp["idx_pool"].view(S, c.idx_pages * 64, c.d_I)
+        self.compress = lambda: (  # noqa: E731  (run as groups complete; timed on its own)
+            sa.csa_compress(inp["Ca"], inp["Cb"], inp["Za"], inp["Zb"], inp["Ba"], inp["Bb"], c.m, inp["lat_pool"],
+                            lat.stride(0), lat.stride(1)),
+            sa.csa_compress(inp["CIa"], inp["CIb"], inp["ZIa"], inp["ZIb"], inp["BIa"], inp["BIb"], c.m,
+                            inp["idx_pool"], idx.stride(0), idx.stride(1)))
+        self.compress()
+        self.scores = torch.empty(S, c.idx_pages * 64, dtype=torch.float32, device=dev)
+        self.idx = torch.empty(S, c.topk, dtype=torch.int32, device=dev)
+        self.slots = torch.empty(S, c.topk + c.window, dtype=torch.int32, device=dev)
+        self.out = torch.empty(S, c.H, c.c, dtype=torch.float32, device=dev)
+        self.ws = torch.empty(max(1, sa.sparse_mla_workspace_size(S, c.H, c.topk + c.window, c.c)),
+                              dtype=torch.uint8, device=dev)
+        combine = sa.sparse_mla_workspace_size(S, c.H, c.topk + c.window, c.c) > \
+            sa.sparse_mla_prefill_workspace_size(S, c.H, c.topk + c.window, c.c)
+        self.launches_per_step = 4 + (1 if combine else 0)
+
+    def indexer(self):
+        i, c = self.inp, self.cfg
+        self.sa.index_scores(i["q_idx"], i["w"], i["idx_pool"], i["n_visible"], c.idx_pages, scores=self.scores)
+
+    def rest(self):
+        self.topk()
+        self.attn()
+
+    def topk(self):
+        self.sa.topk_select(self.scores, self.inp["n_visible"], self.cfg.topk, idx_out=self.idx)
+
+    def attn(self):
+        i, c = self.inp, self.cfg
+        self.sa.csa_window_index(self.idx, i["seq_lens"], c.window, c.n_cap, idx_out=self.slots)
+        self.sa.sparse_mla_decode(i["q"], i["q_rope"], i["lat_pool"], i["lat_pool"], self.slots, c.scale,
+                                  c.lat_pages, out=self.out, workspace=self.ws)
+
+
+def time_compress(step, K: int, flush, hbm: float):
+    """The CSA compression of the whole history (both entry kinds), timed on
+    its own: in decode it runs once per m tokens, outside the step."""
+    c = step.cfg
+    for _ in range(2):
+        step.compress()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    for a, b in ev:
+        flush.zero_()
+        a.record()
+        step.compress()
+        b.record()
+    torch.cuda.synchronize()
+    us = statistics.mean(a.elapsed_time(b) for a, b in ev) * 1e3
+    nbytes = c.n_seqs * c.L * 4 * 2 * (c.c + c.d_I) + c.n_seqs * c.n_c * (c.c * 2 + c.d_I)
+    return {"kernel": "csa_compress_kernel x2", "us": round(us, 1), "tokens_per_s": round(c.n_seqs * c.L / (us * 1e-6), 1),
+            "bytes": nbytes, "hbm_gbs": round(nbytes / (us * 1e-6) / 1e9, 1),
+            "hbm_frac": round(nbytes / (us * 1e-6) / 1e9 / hbm, 4)}
+
+
 def time_steps(step, K: int, flush):
     """K steps, each bracketed by CUDA events on the launching stream (torch's
     current stream, which the library calls use); the L2 flush runs between
@@ -319,6 +393,8 @@ def e2e_steps(step, K: int, flush):
     inp = step.inp
     if isinstance(step, DecodeStep):
         names = ["q_idx", "w", "q_lat", "q_rope"]
+    elif isinstance(step, CsaStep):
+        names = ["q_idx", "w", "q", "q_rope"]
     elif isinstance(step, NsaStep):
         names = ["q", "gates"]
     else:
@@ -360,6 +436,18 @@ def cpu_baseline(inp, cfg, budget_s: float = 12.0):
         unit_n = n
         what = "query rows" if cfg.prefill_start < 0 else "query tokens"
         sample = f"{n} of {cfg.rows} {what} of the workload (indexer over every visible key, top-{cfg.topk}, sparse MLA)"
+    elif isinstance(cfg, W.CSAConfig):
+        t0 = time.perf_counter()
+        oracle.csa_step(inp, [0])
+        one = time.perf_counter() - t0
+        n = int(max(1, min(cfg.n_seqs, budget_s // max(one, 1e-3))))
+        t0 = time.perf_counter()
+        oracle.csa_step(inp, list(range(n)))
+        dt = time.perf_counter() - t0
+        unit_n = n
+        sample = (f"{n} of {cfg.n_seqs} query rows (compression of the whole history inside the timed call, "
+                  f"indexer over every compressed key, top-{cfg.topk}, attention)")
+        threads = 1
     elif isinstance(cfg, W.NSAConfig):
         pairs = [(b, g) for b in range(cfg.B) for g in range(cfg.H_kv)]
         t0 = time.perf_counter()
@@ -391,6 +479,8 @@ def workload(name: str):
         return W.DSA_CONFIGS[name]
     if name in W.NSA_CONFIGS:
         return W.NSA_CONFIGS[name]
+    if name in W.CSA_CONFIGS:
+        return W.CSA_CONFIGS[name]
     return W.BLOCK_CONFIGS[name]
 
 
@@ -402,6 +492,12 @@ def describe(cfg, flush_note):
         return {"workload": f"{cfg.name} {kind}: {cfg.rows} queries, {lens}, indexer H^I={cfg.H_I} d^I={cfg.d_I} "
                             f"{cfg.idx_dtype}, top-{cfg.topk}, sparse MLA {cfg.H} heads d_c={cfg.d_c} d_R={cfg.d_R} bf16",
                 "batch": cfg.rows, "seq_len": max(cfg.lens), "topk": cfg.topk, "heads": cfg.H, "l2": flush_note}
+    if isinstance(cfg, W.CSAConfig):
+        return {"workload": f"CSA decode: {cfg.n_seqs} queries, L={cfg.L} raw tokens compressed {cfg.m}:1 "
+                            f"({cfg.n_c} entries), indexer H^I={cfg.H_I} d^I={cfg.d_I} e4m3 over the entries, "
+                            f"top-{cfg.topk} + {cfg.window}-token raw window, attention {cfg.H} heads over "
+                            f"{cfg.c}-wide bf16 entries (keys = values)",
+                "batch": cfg.n_seqs, "seq_len": cfg.L, "topk": cfg.topk, "heads": cfg.H, "l2": flush_note}
     if isinstance(cfg, W.NSAConfig):
         return {"workload": f"NSA three-branch decode: B={cfg.B}, L={cfg.L}, {cfg.H} query heads in {cfg.H_kv} GQA "
                             f"groups, head_dim {cfg.D} bf16, block {cfg.block} (compression = selection blocks), "
@@ -429,6 +525,9 @@ def run_native(args):
     elif isinstance(cfg, W.NSAConfig):
         inp = W.nsa_inputs(cfg, dev, seed=rank_seed(cfg.seed, rank))
         step = NsaStep(inp, sa)
+    elif isinstance(cfg, W.CSAConfig):
+        inp = W.csa_inputs(cfg, dev, seed=rank_seed(cfg.seed, rank))
+        step = CsaStep(inp, sa)
     else:
         inp = W.block_inputs(cfg, dev, seed=rank_seed(cfg.seed, rank))
         step = BlockStep(inp, sa)
@@ -513,6 +612,27 @@ def run_native(args):
         res["kernels"] = kern
         if not prefill:
             res["projections"] = time_projections(step, min(args.steps, 20), flush, hbm)
+    elif isinstance(cfg, W.CSAConfig):
+        units = cfg.n_seqs * ws
+        unit = "queries/s"
+        metric = "CSA decode queries/s (indexer over compressed entries + topk + window + attention)"
+        keys_b, rows_b = csa_bytes(cfg)
+        kern = {"indexer": {"kernel": "idx_tc_kernel", "us": t_idx * 1e3, "bytes": keys_b},
+                "topk": {"kernel": "topk_kernel", "us": t_topk * 1e3, "bytes": cfg.n_seqs * cfg.n_c * 4},
+                "attn": {"kernel": "csa_window_index_kernel + mla_kernel (+ combine)", "us": t_attn * 1e3,
+                         "bytes": rows_b}}
+        for v in kern.values():
+            v["hbm_gbs"] = round(v["bytes"] / (v["us"] * 1e-6) / 1e9, 1)
+            v["hbm_frac"] = round(v["hbm_gbs"] / hbm, 4)
+            v["us"] = round(v["us"], 2)
+        dom = kern[max(kern, key=lambda n: kern[n]["us"])]
+        roof = {"bound": "hbm", "achieved": dom["hbm_gbs"], "peak": hbm, "unit": "GB/s", "frac": dom["hbm_frac"],
+                "traffic": None, "kernel": dom["kernel"], "peak_source": f"{peak_src} hbm_gbs"}
+        step_gbs = (keys_b + rows_b) / (ms * 1e-3) / 1e9
+        res["step_roofline"] = {"bytes_per_step": keys_b + rows_b, "achieved": round(step_gbs, 1), "peak": hbm,
+                                "unit": "GB/s", "frac": round(step_gbs / hbm, 4)}
+        res["kernels"] = kern
+        res["compression"] = time_compress(step, min(args.steps, 10), flush, hbm)
     elif isinstance(cfg, W.NSAConfig):
         units = cfg.B * ws
         unit = "queries/s"
@@ -535,7 +655,7 @@ def run_native(args):
     res.update({
         "metric": metric, "value": round(value, 1), "unit": unit, "n_gpus": ws, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "e4m3 indexer / bf16 MLA, fp32 accumulate" if isinstance(cfg, W.DSAConfig)
+        "vs_baseline": None, "dtype": "e4m3 indexer / bf16 MLA, fp32 accumulate" if isinstance(cfg, (W.DSAConfig, W.CSAConfig))
         else "bf16, fp32 accumulate",
         "data": "synthetic (seeded, shapes and value distributions of the workload)",
         "config": describe(cfg, f"flushed between steps ({L2_FLUSH_BYTES >> 20} MiB write, outside the events)"),
@@ -657,6 +777,13 @@ def run_reference(args):
         run = lambda: oracle.dsa_step(inp, rows, with_scores=False)  # noqa: E731
         units_per_step = per_step
         sample = f"{per_step} query rows of the workload per step"
+    elif isinstance(cfg, W.CSAConfig):
+        inp = W.csa_inputs(cfg, dev, seed=cfg.seed)
+        unit = "queries/s"
+        metric = "CSA decode queries/s (indexer over compressed entries + topk + window + attention)"
+        run = lambda: oracle.csa_step(inp, [0])  # noqa: E731
+        units_per_step = 1
+        sample = "one query row per step (compression of its whole history inside the timed call)"
     elif isinstance(cfg, W.NSAConfig):
         inp = W.nsa_inputs(cfg, dev, seed=cfg.seed)
         unit = "queries/s"
@@ -699,7 +826,8 @@ def main(argv=None):
     p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--impl", choices=["native", "reference"], default="native")
     p.add_argument("--config", default="long",
-                   choices=sorted(list(W.DSA_CONFIGS) + list(W.BLOCK_CONFIGS) + list(W.NSA_CONFIGS) + ["crossover"]))
+                   choices=sorted(list(W.DSA_CONFIGS) + list(W.BLOCK_CONFIGS) + list(W.NSA_CONFIGS) +
+                                  list(W.CSA_CONFIGS) + ["crossover"]))
     p.add_argument("--no-cpu-baseline", action="store_true")
     args = p.parse_args(argv)
     if args.warmup < 3 and args.impl == "native":
