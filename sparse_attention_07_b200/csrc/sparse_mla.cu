@@ -154,7 +154,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1) mla_ker
     const int t0 = static_cast<int>(static_cast<int64_t>(split) * T / ka.nsplit);
     const int t1 = static_cast<int>(static_cast<int64_t>(split + 1) * T / ka.nsplit);
     const int nt = t1 - t0;  // at most kMaxTilesPerCta (the host picks the splits)
-    const int seq = a.seq_of_row ? a.seq_of_row[r] : r;
     WaitCtx wc{a.err, &s_abort};
 
     if (tid == 0) {
@@ -187,41 +186,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1) mla_ker
         tmem_alloc(&s_tmem, kTmemCols);
         tmem_relinquish();
     }
-    // pool rows of every slot of this CTA's tiles (-1: padded slot)
-    for (int i = tid; i < nt * kNK && nt <= kMaxTilesPerCta; i += kThreads) {
-        const int p = idx_at(a, r, t0 * kNK + i);
-        sRows[i] = p >= 0 ? static_cast<int>(pool_row(a, seq, p)) : -1;
-    }
     tc_fence_before();
-    cluster_sync_all();  // barriers, row table and slot are in place, and the partner has started
+    __syncthreads();  // the TMEM address is published
     tc_fence_after();
     const uint32_t tmem = s_tmem;
-    const uint32_t my_slot = s_slot;
-    const uint32_t peer_slot = ld_cluster_u32(mapa_u32(smem_u32(&s_slot), partner));
-    // both CTAs skip the work alike when either has no scratch slot (recorded above)
-    const bool run = my_slot < static_cast<uint32_t>(kMlaScratchSlots) &&
-                     peer_slot < static_cast<uint32_t>(kMlaScratchSlots) && nt <= kMaxTilesPerCta;
+    const int seq = a.seq_of_row ? a.seq_of_row[r] : r;
 
     if (warp < 4) {
         // The query slice of head `tid` into its TMEM lane: column c holds
         // elements 2c, 2c+1 (rows beyond H are zero and never written out).
+        // Sixteen 16-byte loads in flight per round.
         const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
         const bool live = tid < a.H;
         const uint4* ql = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.q_lat) +
                                                          (static_cast<int64_t>(r) * a.H + (live ? tid : 0)) * 512 +
                                                          rank * 256);
 #pragma unroll 1
-        for (int c = 0; c < 128; c += 32) {
-            uint32_t v[32];
+        for (int c = 0; c < 128; c += 64) {
+            uint32_t v[64];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
+            for (int j = 0; j < 16; ++j) {
                 const uint4 u = live ? ql[c / 4 + j] : make_uint4(0u, 0u, 0u, 0u);
                 v[4 * j] = u.x;
                 v[4 * j + 1] = u.y;
                 v[4 * j + 2] = u.z;
                 v[4 * j + 3] = u.w;
             }
-            tmem_st32(tmem + lane_base + kColQ + c, v);
+            tmem_st32(tmem + lane_base + kColQ + c, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+            tmem_st32(tmem + lane_base + kColQ + c + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
         }
         if (rank == 1) {
             const uint4* qr = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.q_rope) +
@@ -238,10 +230,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1) mla_ker
             tmem_st32(tmem + lane_base + kColQ + 128, v);
         }
         tmem_st_wait();
+    } else if (nt <= kMaxTilesPerCta) {
+        // pool rows of every slot of this CTA's tiles (-1: padded slot), four
+        // selection reads in flight per thread
+        const int n = nt * kNK, nthr = kThreads - 128;
+        for (int i0 = tid - 128; i0 < n; i0 += 4 * nthr) {
+            int pos[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int i = i0 + u * nthr;
+                pos[u] = i < n ? idx_at(a, r, t0 * kNK + i) : -1;
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int i = i0 + u * nthr;
+                if (i < n) sRows[i] = pos[u] >= 0 ? static_cast<int>(pool_row(a, seq, pos[u])) : -1;
+            }
+        }
     }
     tc_fence_before();
-    __syncthreads();
+    cluster_sync_all();  // query, row table and slot are in place, and the partner has started
     tc_fence_after();
+    const uint32_t my_slot = s_slot;
+    const uint32_t peer_slot = ld_cluster_u32(mapa_u32(smem_u32(&s_slot), partner));
+    // both CTAs skip the work alike when either has no scratch slot (recorded above)
+    const bool run = my_slot < static_cast<uint32_t>(kMlaScratchSlots) &&
+                     peer_slot < static_cast<uint32_t>(kMlaScratchSlots) && nt <= kMaxTilesPerCta;
 
     if (!run) {
         // nothing to do: fall through to the teardown
