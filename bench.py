@@ -41,6 +41,7 @@ L2_FLUSH_BYTES = 256 << 20  # > 126 MB L2
 # kernel source it was taken on (the figure is reported only while they match).
 TRAFFIC = {
     "long": {"kernel": "sparse_mla.cu", "bytes_per_launch": 84673792, "src_sha": "abf9ef8dff4ed76b"},
+    "nsa": {"kernel": "nsa.cu", "bytes_per_launch": 59266560, "src_sha": "32750ff2eacb326c"},
 }
 
 
@@ -639,8 +640,11 @@ def run_native(args):
         metric = "NSA decode queries/s (compression + group block choice + selection + window, gated)"
         nbytes = nsa_bytes(cfg)
         ach = nbytes / (first * 1e-3) / 1e9
+        tr = TRAFFIC.get(args.config, {})
+        traffic = tr.get("bytes_per_launch") if tr.get("src_sha") == src_sha(
+            "sparse_attention_07_b200/csrc/" + tr.get("kernel", "nsa.cu")) else None
         roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": hbm, "unit": "GB/s", "frac": round(ach / hbm, 4),
-                "traffic": None, "kernel": "nsa_decode_kernel", "bytes_per_launch": nbytes,
+                "traffic": traffic, "kernel": "nsa_decode_kernel", "bytes_per_launch": nbytes,
                 "peak_source": f"{peak_src} hbm_gbs"}
     else:
         units = cfg.B * ws
