@@ -120,3 +120,14 @@ def test_topk_many_candidates():
     more keys than a CTA lists as candidates, so the refinement scans the slice."""
     _topk_case(3, [131072, 100000, 65536], 2048, 11, lo=0, hi=1)
     _topk_case(2, [131072, 70001], 60000, 12, lo=0, hi=1)
+
+
+def test_topk_edge_rows():
+    """Ragged tails (n not a multiple of 4), two-valued rows whose boundary
+    class holds half the row, k = 1 and k = n - 1, wide integer ranges,
+    against the oracle bit for bit."""
+    _topk_case(3, [49152, 49151, 30001], 2048, 21, lo=-50, hi=50, ld=49152)
+    _topk_case(3, [32768, 32767, 20000], 2048, 22, lo=0, hi=1, ld=32768)
+    _topk_case(2, [1000, 999], 1, 23)
+    _topk_case(2, [1000, 1001], 999, 24, lo=-2, hi=2)
+    _topk_case(4, [32768] * 4, 2048, 25, lo=-100000, hi=100000, ld=32768)
