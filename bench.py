@@ -193,6 +193,8 @@ class DecodeStep:
         self.idx = torch.empty(cfg.rows, cfg.topk, dtype=torch.int32, device=dev)
         self.out = torch.empty(cfg.rows, cfg.H, cfg.d_c, dtype=torch.float32, device=dev)
         self.lse = torch.empty(cfg.rows, cfg.H, dtype=torch.float32, device=dev)
+        # the indexer counts each row's first Top-K digit; the Top-K starts from it and clears it
+        self.hist = sa.topk_histogram(cfg.rows, dev)
         self.prefill = cfg.prefill_start >= 0
         size = sa.sparse_mla_prefill_workspace_size if self.prefill else sa.sparse_mla_workspace_size
         self.ws = torch.empty(size(cfg.rows, cfg.H, cfg.topk, cfg.d_c), dtype=torch.uint8, device=dev)
@@ -204,14 +206,15 @@ class DecodeStep:
     def indexer(self):
         i, c = self.inp, self.cfg
         self.sa.index_scores(i["q_idx"], i["w"], i["k_idx_cache"], i["n_visible"], c.pages_per_seq,
-                             page_table=i["page_table"], seq_of_row=i["seq_of_row"], scores=self.scores)
+                             page_table=i["page_table"], seq_of_row=i["seq_of_row"], scores=self.scores,
+                             hist=self.hist)
 
     def rest(self):
         self.topk()
         self.attn()
 
     def topk(self):
-        self.sa.topk_select(self.scores, self.inp["n_visible"], self.cfg.topk, idx_out=self.idx)
+        self.sa.topk_select(self.scores, self.inp["n_visible"], self.cfg.topk, idx_out=self.idx, hist=self.hist)
 
     def attn(self):
         i, c = self.inp, self.cfg

@@ -7,6 +7,9 @@
  *
  *   sa_index_scores      lightning indexer  I_{t,s} = sum_j w_{t,j} ReLU(q^I_{t,j} . k^I_s)
  *   sa_topk_select       exact Top-K of I_{t,:} (ties to the lower position)
+ *   sa_index_scores_hist / sa_topk_select_hist
+ *                        the same two steps, the indexer also counting each row's
+ *                        first-digit histogram for the Top-K
  *   sa_sparse_mla_decode / sa_sparse_mla_prefill
  *                        softmax over the selected set of the absorbed content score
  *                        plus the RoPE score, scaled; output sum_j a_j c_j in latent space
@@ -116,6 +119,19 @@ sa_status sa_index_scores(const void* q, const float* w, const void* k_cache, in
                           const int32_t* seq_of_row, const int32_t* n_visible,
                           int rows, int H_I, int d_I, int64_t scores_ld, float* scores,
                           sa_stream_t stream);
+
+/*
+ * sa_index_scores, and with it the first step of the Top-K selection: every
+ * score written also counts in hist[r][key >> 20], where key is the score's
+ * order-preserving 32-bit pattern (sign, exponent and three mantissa bits
+ * select one of 4096 bins; -0.0 counts as +0.0).  hist [rows][4096] int32
+ * must hold zeros on entry (sa_topk_select_hist leaves it zeroed again, so
+ * one buffer serves every step).  The scores are those of sa_index_scores.
+ */
+sa_status sa_index_scores_hist(const void* q, const float* w, const void* k_cache, int64_t pool_pages,
+                               sa_dtype dtype, const int32_t* page_table, int pages_per_seq,
+                               const int32_t* seq_of_row, const int32_t* n_visible, int rows, int H_I, int d_I,
+                               int64_t scores_ld, float* scores, int32_t* hist, sa_stream_t stream);
 
 /*
  * Exact Top-K ([Notes] §9, S_t = {s | I_{t,s} in TopK(I_{t,:}, k)}; [MLA-S]
@@ -359,6 +375,16 @@ sa_status sa_csa_compress(const void* Ca, const void* Cb, const void* Za, const 
  */
 sa_status sa_csa_window_index(const int32_t* topk_idx, int rows, int k, const int32_t* raw_len, int window,
                               int win_base, int32_t* idx_out, sa_stream_t stream);
+
+/*
+ * sa_topk_select with the row histograms sa_index_scores_hist counted: the
+ * selection starts from them instead of histogramming the scores again, and
+ * clears them (zeros on return).  Same output as sa_topk_select.  A row whose
+ * counts do not add up to its visible length (a buffer already cleared, say)
+ * is selected from its scores alone, as sa_topk_select does.
+ */
+sa_status sa_topk_select_hist(const float* scores, int64_t scores_ld, const int32_t* n_valid, int rows, int k,
+                              int32_t* hist, int32_t* idx_out, sa_stream_t stream);
 
 #ifdef __cplusplus
 }

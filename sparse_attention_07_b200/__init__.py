@@ -30,6 +30,7 @@ EXPORTS = (
     "sa_block_mean_pool", "sa_block_sparse_attn", "sa_sparse_mla_decode_static",
     "sa_dense_mla_workspace_size", "sa_dense_mla_decode", "sa_mla_absorb_query", "sa_mla_up_project",
     "sa_nsa_compress", "sa_nsa_decode", "sa_csa_compress", "sa_csa_window_index",
+    "sa_index_scores_hist", "sa_topk_select_hist",
 )
 
 # Size of the library's static device array behind sparse_mla_decode_static
@@ -58,6 +59,8 @@ def lib():
         L.sa_check_device_error.argtypes = [ctypes.POINTER(I), P]
         L.sa_index_scores.argtypes = [P, P, P, I64, I, P, I, P, P, I, I, I, I64, P, P]
         L.sa_topk_select.argtypes = [P, I64, P, I, I, P, P]
+        L.sa_index_scores_hist.argtypes = [P, P, P, I64, I, P, I, P, P, I, I, I, I64, P, P, P]
+        L.sa_topk_select_hist.argtypes = [P, I64, P, I, I, P, P, P]
         L.sa_sparse_mla_workspace_size.restype = SZ
         L.sa_sparse_mla_workspace_size.argtypes = [I, I, I, I]
         L.sa_sparse_mla_decode.argtypes = [P, P, P, I64, P, I64, I64, P, I, P, P, I, I, I, I, I, F, P, P, P, SZ, P]
@@ -114,28 +117,50 @@ def check_device_error() -> int:
     return code.value
 
 
+HIST_BINS = 4096
+
+
+def topk_histogram(rows: int, device) -> torch.Tensor:
+    """A zeroed [rows, 4096] int32 buffer for index_scores(hist=...) and
+    topk_select(hist=...): the Top-K leaves it zeroed, so one serves every step."""
+    return torch.zeros(rows, HIST_BINS, dtype=torch.int32, device=device)
+
+
 def index_scores(q_idx, w, k_idx_cache, n_visible, pages_per_seq: int, page_table=None, seq_of_row=None,
-                 scores=None, scores_ld: Optional[int] = None):
-    """Lightning-indexer scores [rows, scores_ld] fp32 (entries past n_visible untouched)."""
+                 scores=None, scores_ld: Optional[int] = None, hist=None):
+    """Lightning-indexer scores [rows, scores_ld] fp32 (entries past n_visible untouched).
+    With `hist` (zeroed [rows, 4096] int32) it also counts each row's first
+    Top-K digit, for topk_select(hist=...)."""
     rows, H_I, d_I = q_idx.shape
     ld = scores_ld or pages_per_seq * 64
     if scores is None:
         scores = torch.empty(rows, ld, dtype=torch.float32, device=q_idx.device)
     pool_pages = k_idx_cache.shape[0] // 64
-    st = lib().sa_index_scores(_p(q_idx), _p(w), _p(k_idx_cache), pool_pages, _dtype_code(q_idx), _p(page_table),
-                               pages_per_seq, _p(seq_of_row), _p(n_visible), rows, H_I, d_I, scores.stride(0),
-                               _p(scores), _stream())
-    _check("sa_index_scores", st)
+    args = (_p(q_idx), _p(w), _p(k_idx_cache), pool_pages, _dtype_code(q_idx), _p(page_table), pages_per_seq,
+            _p(seq_of_row), _p(n_visible), rows, H_I, d_I, scores.stride(0), _p(scores))
+    if hist is None:
+        st = lib().sa_index_scores(*args, _stream())
+        _check("sa_index_scores", st)
+    else:
+        st = lib().sa_index_scores_hist(*args, _p(hist), _stream())
+        _check("sa_index_scores_hist", st)
     return scores
 
 
-def topk_select(scores, n_valid, k: int, idx_out=None):
-    """Exact Top-K positions [rows, k] int32, ascending, -1 padded."""
+def topk_select(scores, n_valid, k: int, idx_out=None, hist=None):
+    """Exact Top-K positions [rows, k] int32, ascending, -1 padded.  With
+    `hist` (as filled by index_scores(hist=...)) the selection starts from it
+    and clears it."""
     rows = scores.shape[0]
     if idx_out is None:
         idx_out = torch.empty(rows, k, dtype=torch.int32, device=scores.device)
-    st = lib().sa_topk_select(_p(scores), scores.stride(0), _p(n_valid), rows, k, _p(idx_out), _stream())
-    _check("sa_topk_select", st)
+    if hist is None:
+        st = lib().sa_topk_select(_p(scores), scores.stride(0), _p(n_valid), rows, k, _p(idx_out), _stream())
+        _check("sa_topk_select", st)
+    else:
+        st = lib().sa_topk_select_hist(_p(scores), scores.stride(0), _p(n_valid), rows, k, _p(hist), _p(idx_out),
+                                       _stream())
+        _check("sa_topk_select_hist", st)
     return idx_out
 
 

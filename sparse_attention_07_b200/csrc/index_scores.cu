@@ -26,6 +26,16 @@
 namespace sa {
 namespace {
 
+// First-digit histogram of the scores a warp writes: lanes with equal digits
+// add once (global atomics, one per distinct digit of the warp).
+__device__ __forceinline__ void hist_add_global(int32_t* hist, bool active, uint32_t digit, int lane) {
+    const unsigned am = __ballot_sync(0xffffffffu, active);
+    if (active) {
+        const unsigned peers = __match_any_sync(am, digit);
+        if (lane == __ffs(peers) - 1) atomicAdd(&hist[digit], __popc(peers));
+    }
+}
+
 constexpr int kPage = 64;
 constexpr int kTileKeys = 128;
 constexpr int kStages = 6;
@@ -423,8 +433,11 @@ __global__ void __launch_bounds__(TcCfg<NH, R, NEPI>::kThreads, 1)
                             }
                         }
                     }
-                    if (s < nvis[0] && g_cnt > 0)
-                        a.scores[static_cast<int64_t>(g_r0) * a.scores_ld + s] = (acc4[0] + acc4[1]) + (acc4[2] + acc4[3]);
+                    const float sc = (acc4[0] + acc4[1]) + (acc4[2] + acc4[3]);
+                    const bool live = s < nvis[0] && g_cnt > 0;
+                    if (live) a.scores[static_cast<int64_t>(g_r0) * a.scores_ld + s] = sc;
+                    if (a.hist) hist_add_global(a.hist + static_cast<int64_t>(g_r0) * kHistBins, live,
+                                                score_order_key(sc) >> 20, lane);
                 } else {
 #pragma unroll
                 for (int j = 0; j < kRowsPerHalf; ++j) {
@@ -449,7 +462,10 @@ __global__ void __launch_bounds__(TcCfg<NH, R, NEPI>::kThreads, 1)
                                     sum += w_own[gi * NH + c + x] * fmaxf(__uint_as_float(v[x]), 0.f);
                             }
                         }
-                        if (s < nvis[j]) a.scores[static_cast<int64_t>(g_r0 + gi) * a.scores_ld + s] = sum;
+                        const bool live = s < nvis[j];
+                        if (live) a.scores[static_cast<int64_t>(g_r0 + gi) * a.scores_ld + s] = sum;
+                        if (a.hist) hist_add_global(a.hist + static_cast<int64_t>(g_r0 + gi) * kHistBins, live,
+                                                    score_order_key(sum) >> 20, lane);
                     }
                 }
                 }
@@ -501,6 +517,7 @@ __global__ void __launch_bounds__(128) idx_cc_kernel(const T* __restrict__ q, co
     const int page = page_of(a, seq, s / kPage);
     if (page < 0 || page >= a.pool_pages) {  // precondition broken: no read outside the pool
         a.scores[static_cast<int64_t>(r) * a.scores_ld + s] = 0.f;
+        if (a.hist) atomicAdd(&a.hist[static_cast<int64_t>(r) * kHistBins + (score_order_key(0.f) >> 20)], 1);
         return;
     }
     const int64_t row = static_cast<int64_t>(page) * kPage + (s % kPage);
@@ -520,6 +537,7 @@ __global__ void __launch_bounds__(128) idx_cc_kernel(const T* __restrict__ q, co
 #pragma unroll
     for (int j = 0; j < NH; ++j) sum += s_w[j] * fmaxf(dot[j], 0.f);
     a.scores[static_cast<int64_t>(r) * a.scores_ld + s] = sum;
+    if (a.hist) atomicAdd(&a.hist[static_cast<int64_t>(r) * kHistBins + (score_order_key(sum) >> 20)], 1);
 }
 
 template <typename T, int NH>

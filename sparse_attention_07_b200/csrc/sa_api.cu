@@ -118,13 +118,14 @@ sa_status sa_check_device_error(int* code_out, sa_stream_t stream) {
     return v ? SA_ETIMEOUT : SA_OK;
 }
 
-sa_status sa_index_scores(const void* q, const float* w, const void* k_cache, int64_t pool_pages, sa_dtype dtype,
-                          const int32_t* page_table, int pages_per_seq, const int32_t* seq_of_row,
-                          const int32_t* n_visible, int rows, int H_I, int d_I, int64_t scores_ld, float* scores,
-                          sa_stream_t stream) {
+static sa_status index_scores_impl(const void* q, const float* w, const void* k_cache, int64_t pool_pages,
+                                   sa_dtype dtype, const int32_t* page_table, int pages_per_seq,
+                                   const int32_t* seq_of_row, const int32_t* n_visible, int rows, int H_I, int d_I,
+                                   int64_t scores_ld, float* scores, int32_t* hist, sa_stream_t stream) {
     if (rows < 0 || H_I < 1 || d_I < 1 || pages_per_seq < 1 || pool_pages < 1 || scores_ld < 1) return SA_EINVAL;
     if (rows == 0) return SA_OK;
     if (!q || !w || !k_cache || !n_visible || !scores) return SA_EINVAL;
+    if (hist && !aligned(hist, 4)) return SA_EINVAL;
     if (dtype != SA_F32 && dtype != SA_E4M3) return SA_EUNSUPPORTED;
     if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(w, 4) || !aligned(scores, 4)) return SA_EINVAL;
     if (pool_pages * 64 > (int64_t(1) << 31)) return SA_EUNSUPPORTED;
@@ -140,6 +141,7 @@ sa_status sa_index_scores(const void* q, const float* w, const void* k_cache, in
     a.d_I = d_I;
     a.scores = scores;
     a.scores_ld = scores_ld;
+    a.hist = hist;
     a.err = device_error_word();
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const bool tc_shape = dtype == SA_E4M3 && d_I == 128 && (H_I == 16 || H_I == 32 || H_I == 64 || H_I == 128) &&
@@ -149,14 +151,44 @@ sa_status sa_index_scores(const void* q, const float* w, const void* k_cache, in
     return index_scores_cc(q, k_cache, dtype, a, st);
 }
 
-sa_status sa_topk_select(const float* scores, int64_t scores_ld, const int32_t* n_valid, int rows, int k,
-                         int32_t* idx_out, sa_stream_t stream) {
+sa_status sa_index_scores(const void* q, const float* w, const void* k_cache, int64_t pool_pages, sa_dtype dtype,
+                          const int32_t* page_table, int pages_per_seq, const int32_t* seq_of_row,
+                          const int32_t* n_visible, int rows, int H_I, int d_I, int64_t scores_ld, float* scores,
+                          sa_stream_t stream) {
+    return index_scores_impl(q, w, k_cache, pool_pages, dtype, page_table, pages_per_seq, seq_of_row, n_visible,
+                             rows, H_I, d_I, scores_ld, scores, nullptr, stream);
+}
+
+sa_status sa_index_scores_hist(const void* q, const float* w, const void* k_cache, int64_t pool_pages,
+                               sa_dtype dtype, const int32_t* page_table, int pages_per_seq,
+                               const int32_t* seq_of_row, const int32_t* n_visible, int rows, int H_I, int d_I,
+                               int64_t scores_ld, float* scores, int32_t* hist, sa_stream_t stream) {
+    if (!hist) return SA_EINVAL;
+    return index_scores_impl(q, w, k_cache, pool_pages, dtype, page_table, pages_per_seq, seq_of_row, n_visible,
+                             rows, H_I, d_I, scores_ld, scores, hist, stream);
+}
+
+static sa_status topk_impl(const float* scores, int64_t scores_ld, const int32_t* n_valid, int rows, int k,
+                           int32_t* hist, int32_t* idx_out, sa_stream_t stream) {
     if (rows < 0 || k < 1 || scores_ld < 1) return SA_EINVAL;
     if (rows == 0) return SA_OK;
     if (!scores || !n_valid || !idx_out) return SA_EINVAL;
-    if (!aligned(scores, 16) || scores_ld % 4 != 0 || !aligned(idx_out, 4)) return SA_EINVAL;
+    if (!aligned(scores, 16) || scores_ld % 4 != 0 || !aligned(idx_out, 4) || (hist && !aligned(hist, 4)))
+        return SA_EINVAL;
     if (scores_ld > 262144) return SA_EUNSUPPORTED;
-    return topk_select_launch(scores, scores_ld, n_valid, rows, k, idx_out, reinterpret_cast<cudaStream_t>(stream));
+    return topk_select_launch(scores, scores_ld, n_valid, rows, k, hist, idx_out,
+                              reinterpret_cast<cudaStream_t>(stream));
+}
+
+sa_status sa_topk_select(const float* scores, int64_t scores_ld, const int32_t* n_valid, int rows, int k,
+                         int32_t* idx_out, sa_stream_t stream) {
+    return topk_impl(scores, scores_ld, n_valid, rows, k, nullptr, idx_out, stream);
+}
+
+sa_status sa_topk_select_hist(const float* scores, int64_t scores_ld, const int32_t* n_valid, int rows, int k,
+                              int32_t* hist, int32_t* idx_out, sa_stream_t stream) {
+    if (!hist) return SA_EINVAL;
+    return topk_impl(scores, scores_ld, n_valid, rows, k, hist, idx_out, stream);
 }
 
 size_t sa_sparse_mla_workspace_size(int rows, int H, int k, int d_c) {

@@ -44,6 +44,18 @@ __device__ __forceinline__ void record_error(int* err, int code) {
     if (err) atomicCAS(err, 0, code);
 }
 
+// ---------------------------------------------------------------- score keys
+// fp32 -> uint32 whose unsigned order is the float order; -0 and +0 map alike.
+__device__ __forceinline__ uint32_t score_order_key(float f) {
+    uint32_t u = __float_as_uint(f);
+    if (u == 0x80000000u) u = 0u;
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// The first radix digit of a score key: bits 31..20 (sign, exponent, three
+// mantissa bits), 4096 bins per row.
+constexpr int kHistBins = 4096;
+
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t* b, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(b)), "r"(count) : "memory");

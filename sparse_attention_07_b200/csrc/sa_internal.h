@@ -31,6 +31,7 @@ struct IdxArgs {
     int d_I;
     float* scores;
     int64_t scores_ld;
+    int32_t* hist;  // [rows][kHistBins] first-digit counts of the scores written, or null
     int* err;
 };
 
@@ -38,7 +39,7 @@ sa_status index_scores_tc(const void* q, const void* k_cache, const IdxArgs& a, 
 sa_status index_scores_cc(const void* q, const void* k_cache, sa_dtype dt, const IdxArgs& a, cudaStream_t st);
 
 sa_status topk_select_launch(const float* scores, int64_t ld, const int32_t* n_valid, int rows, int k,
-                             int32_t* idx_out, cudaStream_t st);
+                             int32_t* hist, int32_t* idx_out, cudaStream_t st);
 
 struct MlaArgs {
     const void* q_lat;

@@ -35,12 +35,7 @@ constexpr int kOwn = kBins0 / kCluster;      // first-digit bins reduced by each
 constexpr int kCandCap = 4096;               // candidate slots per CTA
 static_assert(kOwn == kThreads, "one owned bin per thread");
 
-// fp32 -> uint32 whose unsigned order is the float order; -0 and +0 map alike.
-__device__ __forceinline__ uint32_t order_key(float f) {
-    uint32_t u = __float_as_uint(f);
-    if (u == 0x80000000u) u = 0u;
-    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
+__device__ __forceinline__ uint32_t order_key(float f) { return score_order_key(f); }
 
 // Histogram increment by a whole warp: lanes with equal digits add once.
 __device__ __forceinline__ void hist_add(int* hist, bool active, uint32_t digit, int lane) {
@@ -63,7 +58,7 @@ __device__ __forceinline__ int warp_suffix(int v, int lane) {
 
 __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
     topk_kernel(const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ n_valid, int k, int chunk,
-                int32_t* __restrict__ out) {
+                int32_t* __restrict__ hist, int32_t* __restrict__ out) {
     extern __shared__ __align__(16) uint32_t s_keys[];  // [chunk] keys of this CTA's slice
     __shared__ int s_hist0[kBins0];
     __shared__ int s_hist[2][256];
@@ -84,8 +79,10 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
     n = n < 0 ? 0 : (n > ld ? static_cast<int>(ld) : n);
     int32_t* orow = out + static_cast<int64_t>(row) * k;
 
+    int32_t* hrow = hist ? hist + static_cast<int64_t>(row) * kHistBins : nullptr;
     if (n <= k) {  // every position is selected; the rest is padding
         for (int s = static_cast<int>(rank) * kThreads + tid; s < k; s += kCluster * kThreads) orow[s] = s < n ? s : -1;
+        if (hrow) hrow[static_cast<int>(rank) * kOwn + tid] = 0;  // leave the row's histogram cleared
         return;
     }
 
@@ -117,10 +114,12 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
                 kk = make_uint4(order_key(v[u].x), order_key(v[u].y), order_key(v[u].z), order_key(v[u].w));
                 reinterpret_cast<uint4*>(s_keys)[i] = kk;
             }
-            hist_add(s_hist0, ok, kk.x >> 20, lane);
-            hist_add(s_hist0, ok, kk.y >> 20, lane);
-            hist_add(s_hist0, ok, kk.z >> 20, lane);
-            hist_add(s_hist0, ok, kk.w >> 20, lane);
+            if (!hrow) {
+                hist_add(s_hist0, ok, kk.x >> 20, lane);
+                hist_add(s_hist0, ok, kk.y >> 20, lane);
+                hist_add(s_hist0, ok, kk.z >> 20, lane);
+                hist_add(s_hist0, ok, kk.w >> 20, lane);
+            }
         }
     }
     if (warp == 0) {  // up to three keys after the last full vector
@@ -131,8 +130,66 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
             key = order_key(src[i]);
             s_keys[i] = key;
         }
-        hist_add(s_hist0, ok, key >> 20, lane);
+        if (!hrow) hist_add(s_hist0, ok, key >> 20, lane);
     }
+    // The row's first-digit histogram may come with the scores (the indexer
+    // counted them).  It is used only if its total is the row's length: every
+    // CTA of the cluster reads the same counts, so all take the same branch and
+    // the same cluster barriers; otherwise the counts are built here.
+    bool from_global = false;
+    if (hrow) {
+        constexpr int kPer = kBins0 / kThreads;  // bins per thread, highest first
+        const int b_hi = kBins0 - 1 - tid * kPer;
+        int v[kPer];
+        int mine = 0;
+#pragma unroll
+        for (int j = 0; j < kPer; ++j) {
+            v[j] = hrow[b_hi - j];
+            mine += v[j];
+        }
+        int incl = mine;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int t = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += t;
+        }
+        if (lane == 31) s_wsum[warp] = incl;
+        if (tid == 0) {  // defined values should no bin qualify
+            s_sel0[0] = 0;
+            s_sel0[1] = 0;
+            s_sel0[2] = 0;
+        }
+        __syncthreads();
+        int above = incl - mine;  // keys in bins above this thread's bins
+        int total = 0;
+        for (int w = 0; w < kWarps; ++w) {
+            if (w < warp) above += s_wsum[w];
+            total += s_wsum[w];
+        }
+        from_global = total == n;
+        if (from_global && above < k && k <= above + mine) {
+#pragma unroll
+            for (int j = 0; j < kPer; ++j) {
+                if (k <= above + v[j]) {
+                    s_sel0[0] = b_hi - j;
+                    s_sel0[1] = above;
+                    s_sel0[2] = v[j];
+                    break;
+                }
+                above += v[j];
+            }
+        }
+        __syncthreads();
+        if (!from_global) {  // counts of the keys loaded above (s_hist0 is still zero)
+            const int cnt_round = ((cnt + kThreads - 1) / kThreads) * kThreads;
+            for (int base = 0; base < cnt_round; base += kThreads) {
+                const int i = base + tid;
+                const bool ok = i < cnt;
+                hist_add(s_hist0, ok, ok ? s_keys[i] >> 20 : 0u, lane);
+            }
+        }
+    }
+    if (!from_global) {
     cluster_sync_all();
 
     // CTA `rank` reduces bins rank*512 .. rank*512+511 over the cluster
@@ -169,6 +226,7 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
         }
     }
     cluster_sync_all();
+    }
 
     uint32_t prefix = static_cast<uint32_t>(s_sel0[0]) << 20, mask = 0xFFF00000u;
     int remaining = k - s_sel0[1];
@@ -227,7 +285,12 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
                 int add = 0;
                 for (int w = warp + 1; w < 8; ++w) add += s_wsum[w];
                 s_suf[tid] += add;
-                if (tid == 0) s_suf[256] = 0;
+                if (tid == 0) {
+                    s_suf[256] = 0;
+                    s_sel[0] = 0;  // defined values should no bin qualify
+                    s_sel[1] = 0;
+                    s_sel[2] = -1;
+                }
             }
             __syncthreads();
             if (tid < 256) {
@@ -276,6 +339,7 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
         s_counts[1] = esum;
     }
     cluster_sync_all();
+    if (hrow) hrow[static_cast<int>(rank) * kOwn + tid] = 0;  // every CTA has read it: clear for the next step
     // offsets of this CTA: ranks below take their "above" keys and their share of the class
     int off = 0, eq_before = 0;
     for (uint32_t r = 0; r < rank; ++r) {
@@ -316,13 +380,13 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
 }  // namespace
 
 sa_status topk_select_launch(const float* scores, int64_t ld, const int32_t* n_valid, int rows, int k,
-                             int32_t* idx_out, cudaStream_t st) {
+                             int32_t* hist, int32_t* idx_out, cudaStream_t st) {
     const int chunk = static_cast<int>((((ld + kCluster - 1) / kCluster) + 3) & ~int64_t(3));
     const size_t smem = static_cast<size_t>(chunk) * 4;
     cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return launch_status(e);
-    topk_kernel<<<rows * kCluster, kThreads, smem, st>>>(scores, ld, n_valid, k, chunk, idx_out);
+    topk_kernel<<<rows * kCluster, kThreads, smem, st>>>(scores, ld, n_valid, k, chunk, hist, idx_out);
     return launch_status(cudaGetLastError());
 }
 

@@ -131,3 +131,55 @@ def test_topk_edge_rows():
     _topk_case(2, [1000, 999], 1, 23)
     _topk_case(2, [1000, 1001], 999, 24, lo=-2, hi=2)
     _topk_case(4, [32768] * 4, 2048, 25, lo=-100000, hi=100000, ld=32768)
+
+
+def _order_key_np(x):
+    u = np.asarray(x, dtype=np.float32).view(np.uint32).copy()
+    u[u == 0x80000000] = 0
+    return np.where(u & 0x80000000, ~u, u | 0x80000000).astype(np.uint32)
+
+
+@pytest.mark.parametrize("base,kw", [
+    (W.LONG, dict(n_seqs=3, rows=3, lens=(5000, 2100, 4097), topk=2048)),
+    (W.RAGGED, dict(n_seqs=4, rows=4, lens=(9000, 700, 3000, 64), topk=512)),
+    (W.PREFILL, dict(n_seqs=1, rows=40, lens=(6000,), prefill_start=5000, topk=256)),
+    (W.TINY, dict()),
+])
+def test_indexer_histogram_feeds_topk(base, kw):
+    """The indexer's first-digit counts equal the histogram of the oracle's
+    scores (bit-exact scores, so bit-exact counts); the Top-K started from
+    them matches the oracle and leaves the buffer zeroed for the next step."""
+    cfg = W.small_dsa(base, **kw) if kw else base
+    inp = W.dsa_inputs(cfg, DEV, seed=17)
+    hist = sa.topk_histogram(cfg.rows, DEV)
+    scores = sa.index_scores(inp["q_idx"], inp["w"], inp["k_idx_cache"], inp["n_visible"], cfg.pages_per_seq,
+                             page_table=inp["page_table"], seq_of_row=inp["seq_of_row"], hist=hist)
+    torch.cuda.synchronize()
+    got_h = hist.cpu().numpy()
+    ref = oracle.dsa_step(inp, list(range(cfg.rows)))
+    for i in range(cfg.rows):
+        n = int(ref["n_visible"][i])
+        want = np.bincount(_order_key_np(ref["scores"][i, :n]) >> 20, minlength=4096)
+        assert np.array_equal(got_h[i], want), f"row {i}: histogram"
+    idx = sa.topk_select(scores, inp["n_visible"], cfg.topk, hist=hist)
+    torch.cuda.synchronize()
+    assert np.array_equal(idx.cpu().numpy(), ref["idx"])
+    assert int(hist.abs().sum()) == 0
+    assert sa.check_device_error() == 0
+
+
+def test_topk_histogram_already_cleared():
+    """A second Top-K on the same (now cleared) histogram: the counts no longer
+    add up to the row, so the selection counts the scores itself — same sets."""
+    cfg = W.small_dsa(W.LONG, n_seqs=3, rows=3, lens=(5000, 2100, 4097), topk=2048)
+    inp = W.dsa_inputs(cfg, DEV, seed=19)
+    hist = sa.topk_histogram(cfg.rows, DEV)
+    scores = sa.index_scores(inp["q_idx"], inp["w"], inp["k_idx_cache"], inp["n_visible"], cfg.pages_per_seq,
+                             hist=hist)
+    first = sa.topk_select(scores, inp["n_visible"], cfg.topk, hist=hist)
+    again = sa.topk_select(scores, inp["n_visible"], cfg.topk, hist=hist)
+    plain = sa.topk_select(scores, inp["n_visible"], cfg.topk)
+    torch.cuda.synchronize()
+    assert torch.equal(first, plain) and torch.equal(again, plain)
+    assert int(hist.abs().sum()) == 0
+    assert sa.check_device_error() == 0
