@@ -291,6 +291,7 @@ class CsaStep:
                             inp["idx_pool"], idx.stride(0), idx.stride(1)))
         self.compress()
         self.scores = torch.empty(S, c.idx_pages * 64, dtype=torch.float32, device=dev)
+        self.hist = sa.topk_histogram(S, dev)
         self.idx = torch.empty(S, c.topk, dtype=torch.int32, device=dev)
         self.slots = torch.empty(S, c.topk + c.window, dtype=torch.int32, device=dev)
         self.out = torch.empty(S, c.H, c.c, dtype=torch.float32, device=dev)
@@ -302,14 +303,15 @@ class CsaStep:
 
     def indexer(self):
         i, c = self.inp, self.cfg
-        self.sa.index_scores(i["q_idx"], i["w"], i["idx_pool"], i["n_visible"], c.idx_pages, scores=self.scores)
+        self.sa.index_scores(i["q_idx"], i["w"], i["idx_pool"], i["n_visible"], c.idx_pages, scores=self.scores,
+                             hist=self.hist)
 
     def rest(self):
         self.topk()
         self.attn()
 
     def topk(self):
-        self.sa.topk_select(self.scores, self.inp["n_visible"], self.cfg.topk, idx_out=self.idx)
+        self.sa.topk_select(self.scores, self.inp["n_visible"], self.cfg.topk, idx_out=self.idx, hist=self.hist)
 
     def attn(self):
         i, c = self.inp, self.cfg

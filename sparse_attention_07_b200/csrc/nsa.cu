@@ -18,9 +18,10 @@
 // cache, built when a block completes).
 //
 // nsa_decode: a cluster of kC CTAs per (sequence, KV head).  Every CTA streams
-// its share of the data through one ring of 32-row items (cp.async, padded
-// rows): window K rows, compressed K rows (its chunk of blocks), window V,
-// compressed V, then selected-block K and V.  Contractions run on mma.sync
+// its share of the data through one ring of 32-row items (two TMA boxes of 64
+// dims each, 128-byte swizzle, one mbarrier per slot): compressed K rows (its
+// chunk of blocks), window K rows, window V, compressed V, then selected-block
+// K and V.  Contractions run on mma.sync
 // m16n8k16 bf16 with the group's heads as N = 8 (scores as S^T = K Q^T,
 // outputs as O^T = V^T P^T): with at most 16 query rows per KV head, tcgen05's
 // smallest tile (M = 64) would be mostly padding, and the kernel is bound by
