@@ -166,12 +166,12 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-__device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y, int z,
-                                            int w) {
+__device__ __forceinline__ void tma_load_5d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y, int z,
+                                            int w, int v) {
     asm volatile(
-        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5, "
-        "%6}], [%2];" ::"r"(smem_u32(dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z), "r"(w)
+        "cp.async.bulk.tensor.5d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5, "
+        "%6, %7}], [%2];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(v)
         : "memory");
 }
 
@@ -316,8 +316,10 @@ struct Plan {
 };
 
 struct Maps {
-    CUtensorMap K, V;    // token cache: dims (D, H_kv, L, B), box 64 x 1 x 32 x 1
-    CUtensorMap Kc, Vc;  // compressed cache: dims (D, n_blocks, H_kv, B), box 64 x 32 x 1 x 1
+    // Dims (64 dims, row, dim half, KV head, sequence): one box of 64 x 32 x 2 x 1 x 1
+    // lands as [half][row][64 dims], 128-byte swizzled.
+    CUtensorMap K, V;    // token cache: rows = positions
+    CUtensorMap Kc, Vc;  // compressed cache: rows = complete blocks
 };
 
 // One thread: the two TMA boxes (dims 0-63, 64-127) of ring item i into its
@@ -332,8 +334,8 @@ __device__ __forceinline__ const CUtensorMap* locate_item(const Maps& m, const P
         const bool isv = j >= p.nwi;
         if (isv) j -= p.nwi;
         map = isv ? &m.V : &m.K;
-        y = p.kvh;
-        z = p.w_lo + kRows * (p.r + kC * j);
+        y = p.w_lo + kRows * (p.r + kC * j);
+        z = p.kvh;
     } else if (j < p.nA) {  // compressed rows
         const bool isv = j >= p.nci;
         if (isv) j -= p.nci + 2 * p.nwi;
@@ -345,8 +347,8 @@ __device__ __forceinline__ const CUtensorMap* locate_item(const Maps& m, const P
         const bool isv = j >= p.nsi;
         if (isv) j -= p.nsi;
         map = isv ? &m.V : &m.K;
-        y = p.kvh;
-        z = chosen[p.r + kC * (j / p.ipb)] * block + kRows * (j % p.ipb);
+        y = chosen[p.r + kC * (j / p.ipb)] * block + kRows * (j % p.ipb);
+        z = p.kvh;
     }
     return map;
 }
@@ -358,8 +360,7 @@ __device__ __forceinline__ void issue_item(const Maps& m, const Plan& p, int i, 
     mbar_arrive_expect_tx(&full[slot], kItemB);
     int y, z;
     const CUtensorMap* map = locate_item(m, p, i, chosen, block, y, z);
-    tma_load_4d(dst, map, &full[slot], 0, y, z, p.b);
-    tma_load_4d(dst + kHalfB, map, &full[slot], 64, y, z, p.b);
+    tma_load_5d(dst, map, &full[slot], 0, y, 0, z, p.b);  // y = first row, z = KV head
 }
 
 // Scores of one item: S^T[32 rows x GP heads] = rows . Q^T, split over the
@@ -802,21 +803,20 @@ sa_status nsa_decode_launch(const void* q, const void* K, const void* V, int64_t
     if (smem > kNsaMaxSmem) return SA_EUNSUPPORTED;
     Maps m;
     {
-        const uint64_t tdims[4] = {static_cast<uint64_t>(kD), static_cast<uint64_t>(Hkv), static_cast<uint64_t>(L),
+        const uint64_t tdims[5] = {64, static_cast<uint64_t>(L), 2, static_cast<uint64_t>(Hkv),
                                    static_cast<uint64_t>(B)};
-        const uint64_t tstr[3] = {static_cast<uint64_t>(sh) * 2, static_cast<uint64_t>(st_) * 2,
+        const uint64_t tstr[4] = {static_cast<uint64_t>(st_) * 2, 128, static_cast<uint64_t>(sh) * 2,
                                   static_cast<uint64_t>(sb) * 2};
-        const uint32_t tbox[4] = {64, 1, kRows, 1};
-        const uint64_t cdims[4] = {static_cast<uint64_t>(kD), static_cast<uint64_t>(std::max(1, L / block)),
-                                   static_cast<uint64_t>(Hkv), static_cast<uint64_t>(B)};
-        const uint64_t cstr[3] = {static_cast<uint64_t>(kD) * 2, static_cast<uint64_t>(c_ld) * kD * 2,
+        const uint64_t cdims[5] = {64, static_cast<uint64_t>(std::max(1, L / block)), 2, static_cast<uint64_t>(Hkv),
+                                   static_cast<uint64_t>(B)};
+        const uint64_t cstr[4] = {static_cast<uint64_t>(kD) * 2, 128, static_cast<uint64_t>(c_ld) * kD * 2,
                                   static_cast<uint64_t>(c_ld) * kD * 2 * Hkv};
-        const uint32_t cbox[4] = {64, kRows, 1, 1};
+        const uint32_t box[5] = {64, kRows, 2, 1, 1};
         const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
         const CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B;
-        if (!encode_tiled(&m.K, bf, 4, K, tdims, tstr, tbox, sw) || !encode_tiled(&m.V, bf, 4, V, tdims, tstr, tbox, sw) ||
-            !encode_tiled(&m.Kc, bf, 4, Kc, cdims, cstr, cbox, sw) ||
-            !encode_tiled(&m.Vc, bf, 4, Vc, cdims, cstr, cbox, sw))
+        if (!encode_tiled(&m.K, bf, 5, K, tdims, tstr, box, sw) || !encode_tiled(&m.V, bf, 5, V, tdims, tstr, box, sw) ||
+            !encode_tiled(&m.Kc, bf, 5, Kc, cdims, cstr, box, sw) ||
+            !encode_tiled(&m.Vc, bf, 5, Vc, cdims, cstr, box, sw))
             return SA_ECUDA;
     }
     const unsigned grid = static_cast<unsigned>(B) * Hkv * kC;
