@@ -18,8 +18,8 @@
 // cache, built when a block completes).
 //
 // nsa_decode: a cluster of kC CTAs per (sequence, KV head).  Every CTA streams
-// its share of the data through one ring of 32-row items (two TMA boxes of 64
-// dims each, 128-byte swizzle, one mbarrier per slot): compressed K rows (its
+// its share of the data through one ring of 32-row items (one TMA box each,
+// both 64-dim halves of the rows, 128-byte swizzle, one mbarrier per slot): compressed K rows (its
 // chunk of blocks), window K rows, window V, compressed V, then selected-block
 // K and V.  Contractions run on mma.sync
 // m16n8k16 bf16 with the group's heads as N = 8 (scores as S^T = K Q^T,
@@ -322,9 +322,8 @@ struct Maps {
     CUtensorMap Kc, Vc;  // compressed cache: rows = complete blocks
 };
 
-// One thread: the two TMA boxes (dims 0-63, 64-127) of ring item i into its
-// slot, completing on the slot's mbarrier.  Rows past the end of the history
-// (or of the complete blocks) are zero-filled by the copy.
+// The tensor map and first row (y) of ring item i: compressed K rows, window K,
+// window V, compressed V, then the rows of the selected blocks, K and V.
 __device__ __forceinline__ const CUtensorMap* locate_item(const Maps& m, const Plan& p, int i, const int* chosen,
                                                          int block, int& y, int& z) {
     int j = i;
@@ -353,6 +352,9 @@ __device__ __forceinline__ const CUtensorMap* locate_item(const Maps& m, const P
     return map;
 }
 
+// One thread: the TMA box of ring item i (both halves, dims 0-63 and 64-127)
+// into its slot, completing on the slot's mbarrier.  Rows past the end of the
+// history (or of the complete blocks) are zero-filled by the copy.
 __device__ __forceinline__ void issue_item(const Maps& m, const Plan& p, int i, uint8_t* ring, uint64_t* full,
                                            const int* chosen, int block) {
     const int slot = i % kStages;
