@@ -115,3 +115,31 @@ def test_sparse_mla_leading_empty_tiles(fn_name):
     assert_attention_close(out, ref_out, "leading empty tiles")
     assert_lse_close(lse, ref_lse, "lse")
     assert sa.check_device_error() == 0
+
+
+def test_sparse_mla_split_merge_repeatable():
+    """Split keys (three rows: sixteen key splits each): the merged output is
+    the same on every call, whatever the workspace held before, and one
+    workspace serves calls back to back."""
+    cfg, inp, idx = _case(3, 128, 2048, 5000, seed=77)
+    need = sa.sparse_mla_workspace_size(cfg.rows, cfg.H, cfg.topk, cfg.d_c)
+
+    def call(ws):
+        lse = torch.empty(cfg.rows, cfg.H, dtype=torch.float32, device=DEV)
+        out = sa.sparse_mla_decode(inp["q_lat"], inp["q_rope"], inp["c_cache"], inp["kr_cache"], idx, cfg.scale,
+                                   cfg.pages_per_seq, page_table=inp["page_table"], lse=lse, workspace=ws)
+        torch.cuda.synchronize()
+        return out, lse
+
+    out0, lse0 = call(torch.zeros(need, dtype=torch.uint8, device=DEV))
+    for fill in (255, 0x5A):
+        out, lse = call(torch.full((need,), fill, dtype=torch.uint8, device=DEV))
+        assert torch.equal(out, out0) and torch.equal(lse, lse0)
+    ws = torch.full((need,), 255, dtype=torch.uint8, device=DEV)
+    for _ in range(3):
+        out, lse = call(ws)
+        assert torch.equal(out, out0) and torch.equal(lse, lse0)
+    ref_out, ref_lse = _oracle(cfg, inp, idx)
+    assert_attention_close(out0.cpu().numpy(), ref_out, "split merge")
+    assert_lse_close(lse0.cpu().numpy(), ref_lse, "lse")
+    assert sa.check_device_error() == 0
