@@ -565,36 +565,86 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1) mla_ker
     if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
 }
 
-// Merge the split partial states of every (row, head).
-__global__ void __launch_bounds__(128) mla_combine_kernel(const MlaKernelArgs ka) {
+// Merge the split partial states of every (row, head).  Thread = (row, head,
+// four 16-byte pieces d, d + 128, d + 256, d + 384 of the 512 latent dims):
+// 32 threads per head, eight heads per CTA, three CTAs per SM; the loads of
+// two splits (their states and outputs) are in flight together.
+constexpr int kCombThreads = 256;
+constexpr int kCombHeads = kCombThreads / 32;
+constexpr int kCombChunk = 2;  // splits whose loads are issued together
+
+__global__ void __launch_bounds__(kCombThreads, 3) mla_combine_kernel(const MlaKernelArgs ka) {
     const MlaArgs& a = ka.a;
-    const int r = blockIdx.x / a.H, h = blockIdx.x % a.H;
+    const int64_t rh = static_cast<int64_t>(blockIdx.x) * kCombHeads + (threadIdx.x >> 5);
+    if (rh >= static_cast<int64_t>(a.rows) * a.H) return;
+    const int r = static_cast<int>(rh / a.H), h = static_cast<int>(rh % a.H);
     const int ns = ka.nsplit;
+    const int d = (threadIdx.x & 31) * 4;
+    const int64_t base0 = static_cast<int64_t>(r) * ns * a.H + h;  // (row, split 0, head)
     float M = -INFINITY;
-    for (int s = 0; s < ns; ++s) {
-        const float* ml = ka.ws_ml + ((static_cast<int64_t>(r) * ns + s) * a.H + h) * 4;
-        if (ml[1] > 0.f) M = fmaxf(M, ml[0]);
+    for (int s0 = 0; s0 < ns; s0 += kCombChunk) {
+        float mv[kCombChunk], lv[kCombChunk];
+#pragma unroll
+        for (int j = 0; j < kCombChunk; ++j) {
+            mv[j] = -INFINITY;
+            lv[j] = 0.f;
+            if (s0 + j < ns) {
+                const float* ml = ka.ws_ml + (base0 + static_cast<int64_t>(s0 + j) * a.H) * 4;
+                mv[j] = ml[0];
+                lv[j] = ml[1];
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < kCombChunk; ++j)
+            if (lv[j] > 0.f) M = fmaxf(M, mv[j]);
     }
     float L = 0.f, LX = 0.f;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    const int d = threadIdx.x * 4;
-    for (int s = 0; s < ns; ++s) {
-        const int64_t base = (static_cast<int64_t>(r) * ns + s) * a.H + h;
-        const float* ml = ka.ws_ml + base * 4;
-        if (!(ml[1] > 0.f)) continue;
-        const float wgt = exp2f(ml[0] - M);
-        L += ml[1] * wgt;
-        LX += ml[2] * wgt;
-        const float4 o = *reinterpret_cast<const float4*>(ka.ws_o + base * 512 + d);
-        acc.x += o.x * wgt;
-        acc.y += o.y * wgt;
-        acc.z += o.z * wgt;
-        acc.w += o.w * wgt;
+    float4 acc[4];
+#pragma unroll
+    for (int p = 0; p < 4; ++p) acc[p] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s0 = 0; s0 < ns; s0 += kCombChunk) {
+        float mv[kCombChunk], lv[kCombChunk], xv[kCombChunk];
+        float4 o[kCombChunk][4];
+#pragma unroll
+        for (int j = 0; j < kCombChunk; ++j) {
+            mv[j] = 0.f;
+            lv[j] = 0.f;
+            xv[j] = 0.f;
+#pragma unroll
+            for (int p = 0; p < 4; ++p) o[j][p] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (s0 + j < ns) {
+                const int64_t row = base0 + static_cast<int64_t>(s0 + j) * a.H;
+                const float* ml = ka.ws_ml + row * 4;
+                mv[j] = ml[0];
+                lv[j] = ml[1];
+                xv[j] = ml[2];
+                const float4* src = reinterpret_cast<const float4*>(ka.ws_o + row * 512 + d);
+#pragma unroll
+                for (int p = 0; p < 4; ++p) o[j][p] = src[32 * p];
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < kCombChunk; ++j) {  // in split order
+            if (!(lv[j] > 0.f)) continue;
+            const float wgt = exp2f(mv[j] - M);
+            L += lv[j] * wgt;
+            LX += xv[j] * wgt;
+#pragma unroll
+            for (int p = 0; p < 4; ++p) {
+                acc[p].x += o[j][p].x * wgt;
+                acc[p].y += o[j][p].y * wgt;
+                acc[p].z += o[j][p].z * wgt;
+                acc[p].w += o[j][p].w * wgt;
+            }
+        }
     }
     const float inv = L > 0.f ? 1.f / L : 0.f;
     float* dst = a.out + (static_cast<int64_t>(r) * a.H + h) * a.d_c + d;
-    *reinterpret_cast<float4*>(dst) = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
-    if (threadIdx.x == 0 && a.lse)
+#pragma unroll
+    for (int p = 0; p < 4; ++p)
+        *reinterpret_cast<float4*>(dst + 128 * p) =
+            make_float4(acc[p].x * inv, acc[p].y * inv, acc[p].z * inv, acc[p].w * inv);
+    if ((threadIdx.x & 31) == 0 && a.lse)
         a.lse[static_cast<int64_t>(r) * a.H + h] = L > 0.f ? (M + log2f(LX)) * 0.6931471805599453f : -INFINITY;
 }
 
@@ -649,7 +699,8 @@ sa_status sparse_mla_launch(const MlaArgs& a, int nsplit, void* ws, size_t ws_by
     e = cudaGetLastError();
     if (e != cudaSuccess) return launch_status(e);
     if (nsplit > 1) {
-        mla_combine_kernel<<<a.rows * a.H, 128, 0, st>>>(ka);
+        const int64_t heads = static_cast<int64_t>(a.rows) * a.H;
+        mla_combine_kernel<<<static_cast<unsigned>((heads + kCombHeads - 1) / kCombHeads), kCombThreads, 0, st>>>(ka);
         e = cudaGetLastError();
     }
     return launch_status(e);

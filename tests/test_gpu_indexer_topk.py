@@ -71,14 +71,25 @@ def test_indexer_cuda_core_fp8_small_dim():
 
 
 def _topk_case(rows, n, k, seed, lo=-3, hi=3, ld=None):
+    """Integer scores: the selection counting the scores itself, and started
+    from a first-digit histogram (counted here on the host, as the indexer
+    counts it), both against the oracle bit for bit."""
     g = torch.Generator(device=DEV)
     g.manual_seed(seed)
     ld = ld or ((max(n) + 3) // 4 * 4)
     s = torch.randint(lo, hi + 1, (rows, ld), generator=g, device=DEV).float()
     nv = torch.tensor(n, dtype=torch.int32, device=DEV)
     got = sa.topk_select(s, nv, k).cpu().numpy()
-    want = oracle.topk(s.double().cpu().numpy(), np.array(n), k)
+    s_np = s.cpu().numpy()
+    want = oracle.topk(s_np.astype(np.float64), np.array(n), k)
     assert np.array_equal(got, want)
+    counts = np.stack([np.bincount(_order_key_np(s_np[i, : n[i]]) >> 20, minlength=sa.HIST_BINS)
+                       for i in range(rows)]).astype(np.int32)
+    hist = sa.topk_histogram(rows, DEV)
+    hist.copy_(torch.from_numpy(counts))
+    got_h = sa.topk_select(s, nv, k, hist=hist).cpu().numpy()
+    assert np.array_equal(got_h, want)
+    assert int(hist.abs().sum()) == 0  # left cleared for the next step
     assert sa.check_device_error() == 0
 
 
