@@ -169,6 +169,16 @@ __device__ __forceinline__ bool warp_wait(uint64_t* b, uint32_t parity, const Wa
     return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 
+// ---------------------------------------------------------------- dependent launch
+// Lets the next kernel of the stream, when it was launched with programmatic
+// serialization, be scheduled now: its CTAs take free SM resources and wait in
+// pdl_wait() until this grid has completed and its writes are visible.
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// Waits until the previous kernel of the stream has completed and its writes
+// are visible; returns at once when this launch did not overlap it.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_desc(const void* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");

@@ -19,6 +19,25 @@ bool encode_tiled(CUtensorMap* map, CUtensorMapDataType dt, int rank, const void
                   const uint64_t* strides_bytes, const uint32_t* box, CUtensorMapSwizzle swz);
 sa_status launch_status(cudaError_t e);
 
+// Launch with programmatic serialization: the kernel may be scheduled while
+// the previous kernel of the stream still runs (once that kernel's CTAs have
+// all called pdl_trigger() or exited) and must call pdl_wait() before it
+// reads anything the previous kernel writes.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 struct IdxArgs {
     const float* w;
     const int32_t* page_table;
