@@ -10,12 +10,17 @@
 // (N = R rows x H_I heads), issued as four tcgen05.mma kind::f8f6f4 of
 // K = 32 into a TMEM accumulator; the epilogue thread that owns a key (TMEM
 // lane) applies ReLU, the weights and the head sum in registers and writes one
-// fp32 score per row.  A persistent CTA per SM walks a balanced contiguous
-// range of (row group, key tile) items; a TMA producer warp streams 16 KB key
-// tiles (two 64-token pages) through a 6-stage ring, an MMA warp issues, and
-// 4 or 8 epilogue warps drain a ring of 2 or 4 TMEM accumulators.  The producer
-// looks up 32 items at a time (one per lane), so its issue loop holds no
-// dependent global loads.
+// fp32 score per row.  Persistent CTAs walk balanced contiguous ranges of
+// (row group, key tile) items; a TMA producer warp streams 16 KB key tiles
+// (two 64-token pages) through a ring, an MMA warp issues, and 4 or 8
+// epilogue warps drain a ring of 2 or 4 TMEM accumulators.  The producer looks
+// up 32 items at a time (one per lane), so its issue loop holds no dependent
+// global loads.  A ring stage stays busy from its TMA issue (about 3.4 us to
+// land under full load) until its MMAs complete, so the bytes in flight per
+// SM set the rate: one-row groups (decode) therefore run two CTAs per SM, each
+// with a 5-stage ring, at most 128 registers per thread and 256 TMEM columns
+// (4.7 TB/s on the ragged workload against 3.3 TB/s with one 6-stage CTA).
+// Grouped rows (prefill) keep one CTA per SM with a 6-stage ring.
 //
 // CUDA-core path (fp32 or fp8, d_I <= 128, H_I <= 64): one thread per key.
 #include <cuda_fp8.h>
@@ -38,7 +43,6 @@ __device__ __forceinline__ void hist_add_global(int32_t* hist, bool active, uint
 
 constexpr int kPage = 64;
 constexpr int kTileKeys = 128;
-constexpr int kStages = 6;
 constexpr int kStageBytes = kTileKeys * 128;  // 128 keys x 128 fp8
 constexpr int kMaxRows = 4096;
 
@@ -145,18 +149,26 @@ struct TcCfg {
     static constexpr int kTmemCols = (kAcc * N <= 32) ? 32 : (kAcc * N <= 64 ? 64 : (kAcc * N <= 128 ? 128 : (kAcc * N <= 256 ? 256 : 512)));
     static constexpr int kQBytes = N * 128;
     static constexpr int kThreads = 32 * (NEPI + 2);
-    // shared layout (offsets from a 1024-aligned base)
+    // key-tile ring: one-row groups (decode) keep five stages so that two CTAs
+    // fit on an SM (shared memory and tensor memory) and stream side by side
+    static constexpr int kStages = R == 1 ? 5 : 6;
+    // registers per thread: one-row groups with up to 64 heads stay within 128
+    // so that two CTAs fit (each CTA's warps are allocated in groups of four);
+    // otherwise whatever one CTA of kThreads can have
+    static constexpr int kTwoPerSm = R == 1 && NH <= 64;
+    static constexpr int kMaxReg = kTwoPerSm ? 128 : ((65536 / kThreads) & ~7) > 255 ? 255 : ((65536 / kThreads) & ~7);
+    // shared layout (offsets from a 1024-aligned base); the three group tables
+    // (prefix, group start, group length) follow, (rows + 1) ints each, rounded
     static constexpr int kOffStages = 0;
     static constexpr int kOffQ = kOffStages + kStages * kStageBytes;
     static constexpr int kOffW = kOffQ + 2 * kQBytes;
-    static constexpr int kOffPrefix = kOffW + NEPI * R * NH * 4;
-    static constexpr int kOffGStart = kOffPrefix + (kMaxRows + 1) * 4;
-    static constexpr int kOffGnk = kOffGStart + (kMaxRows + 1) * 4;
-    static constexpr int kSmemBytes = kOffGnk + (kMaxRows + 1) * 4 + 1024;
+    static constexpr int kOffTables = kOffW + NEPI * R * NH * 4;
+    static int table_ints(int rows) { return (rows + 1 + 3) & ~3; }
+    static size_t smem_bytes(int rows) { return kOffTables + 3 * static_cast<size_t>(table_ints(rows)) * 4 + 1024; }
 };
 
 template <int NH, int R, int NEPI>
-__global__ void __launch_bounds__(TcCfg<NH, R, NEPI>::kThreads, 1)
+__global__ void __launch_bounds__((TcCfg<NH, R, NEPI>::kThreads)) __maxnreg__((TcCfg<NH, R, NEPI>::kMaxReg))
     idx_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
                   const IdxArgs a) {
     using C = TcCfg<NH, R, NEPI>;
@@ -166,11 +178,12 @@ __global__ void __launch_bounds__(TcCfg<NH, R, NEPI>::kThreads, 1)
     uint8_t* s_stage = sm + C::kOffStages;
     uint8_t* s_q = sm + C::kOffQ;
     float* s_w = reinterpret_cast<float*>(sm + C::kOffW);
-    int* s_prefix = reinterpret_cast<int*>(sm + C::kOffPrefix);
-    int* s_gstart = reinterpret_cast<int*>(sm + C::kOffGStart);
-    int* s_gnk = reinterpret_cast<int*>(sm + C::kOffGnk);  // longest visible length in the group
+    const int tab = (a.rows + 1 + 3) & ~3;
+    int* s_prefix = reinterpret_cast<int*>(sm + C::kOffTables);
+    int* s_gstart = s_prefix + tab;
+    int* s_gnk = s_gstart + tab;  // longest visible length in the group
 
-    __shared__ uint64_t bar_full[kStages], bar_empty[kStages], bar_qfull[2], bar_qempty[2], bar_accfull[C::kAcc],
+    __shared__ uint64_t bar_full[C::kStages], bar_empty[C::kStages], bar_qfull[2], bar_qempty[2], bar_accfull[C::kAcc],
         bar_accempty[C::kAcc], bar_final;
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort;
@@ -182,7 +195,7 @@ __global__ void __launch_bounds__(TcCfg<NH, R, NEPI>::kThreads, 1)
 
     if (tid == 0) {
         s_abort = 0;
-        for (int i = 0; i < kStages; ++i) {
+        for (int i = 0; i < C::kStages; ++i) {
             mbar_init(&bar_full[i], 1);
             mbar_init(&bar_empty[i], 1);
         }
@@ -304,7 +317,7 @@ __global__ void __launch_bounds__(TcCfg<NH, R, NEPI>::kThreads, 1)
                 }
                 ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
                 if (!ok) break;
-                if (++stage == kStages) {
+                if (++stage == C::kStages) {
                     stage = 0;
                     phase ^= 1;
                 }
@@ -314,9 +327,9 @@ __global__ void __launch_bounds__(TcCfg<NH, R, NEPI>::kThreads, 1)
         if (lane == 0) {
             int dummy = 0;
             WaitCtx dw{a.err, reinterpret_cast<volatile int*>(&dummy)};
-            for (int64_t i = n_issued - kStages; i < n_issued; ++i) {
+            for (int64_t i = n_issued - C::kStages; i < n_issued; ++i) {
                 if (i < 0) continue;
-                mbar_wait(&bar_full[i % kStages], static_cast<uint32_t>((i / kStages) & 1), dw, kErrIdxWait | 7);
+                mbar_wait(&bar_full[i % C::kStages], static_cast<uint32_t>((i / C::kStages) & 1), dw, kErrIdxWait | 7);
             }
         }
         __syncwarp();
@@ -353,7 +366,7 @@ __global__ void __launch_bounds__(TcCfg<NH, R, NEPI>::kThreads, 1)
                 __syncwarp();
                 if (s_abort) break;
                 ++acc;
-                if (++stage == kStages) {
+                if (++stage == C::kStages) {
                     stage = 0;
                     phase ^= 1;
                 }
@@ -564,9 +577,20 @@ sa_status launch_tc(const void* q, const void* kc, const IdxArgs& a, cudaStream_
     if (!encode_tiled(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, q, qdims, qstr, qbox, CU_TENSOR_MAP_SWIZZLE_128B))
         return SA_ECUDA;
     auto kern = idx_tc_kernel<NH, R, NEPI>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    const size_t smem = C::smem_bytes(a.rows);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return launch_status(e);
-    kern<<<sm_count(), C::kThreads, C::kSmemBytes, st>>>(tk, tq, a);
+    // persistent CTAs: two per SM where shared memory, registers and tensor
+    // memory (two accumulator rings) allow, each walking its own item range
+    // persistent CTAs: two per SM for one-row groups (two accumulator rings
+    // fit in tensor memory, two CTAs' shared memory and registers fit the SM)
+    int per_sm = 1;
+    if (C::kTwoPerSm && 2 * C::kTmemCols <= 512 && 2 * (smem + 2048) <= 227 * 1024) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);  // all of it as shared
+        if (e != cudaSuccess) return launch_status(e);
+        per_sm = 2;
+    }
+    kern<<<sm_count() * per_sm, C::kThreads, smem, st>>>(tk, tq, a);
     return launch_status(cudaGetLastError());
 }
 
