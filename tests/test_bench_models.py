@@ -1,0 +1,52 @@
+"""The algorithmic byte and flop models behind bench.py's roofline figures,
+checked against the same quantities written out by hand for each workload
+(no GPU: these are host arithmetic only)."""
+import bench
+import workloads as W
+
+
+def test_long_decode_step_bytes():
+    """32 queries x 32768 e4m3 keys of 128 bytes, then 2048 selected rows of
+    512 + 64 bf16 per query: 209,715,200 bytes per step."""
+    keys, rows = bench.decode_bytes(W.LONG)
+    assert keys == 32 * 32768 * 128 == 134_217_728
+    assert rows == 32 * 2048 * (512 + 64) * 2 == 75_497_472
+    assert keys + rows == 209_715_200
+
+
+def test_prefill_flops():
+    """Query i of the 4096-query chunk sees 61441 + i keys: the indexer does
+    2 * 64 heads * 128 dims flops per visible key, the attention
+    2 * 128 heads * (512 + 64 + 512) per selected row (score and aggregate)."""
+    idx, mla = bench.prefill_flops(W.PREFILL)
+    visible = 4096 * 61441 + 4095 * 4096 // 2
+    assert idx == 2 * 64 * 128 * visible == 4_260_641_112_064
+    assert mla == 4096 * 2048 * 2 * 128 * 1088 == 2_336_462_209_024
+
+
+def test_block_sparse_bytes():
+    """fp32 pooled keys of 2048 blocks for 8 x 32 (sequence, head) pairs; at
+    most 16 top blocks + the sink block + a 512-token window in the union."""
+    pooled, u_max = bench.block_bytes(W.BLOCK)
+    assert pooled == 8 * 32 * 2048 * 128 * 4 == 268_435_456
+    assert u_max == 16 * 64 + 64 + 512 == 1600
+
+
+def test_nsa_decode_bytes():
+    """Per (sequence, KV head): compressed K and V of 2048 blocks, K and V of
+    16 selected 64-token blocks and of the 512-token window (128 bf16 each),
+    and for each of the group's 8 heads its bf16 query, three fp32 gates and
+    fp32 output: 1,841,248 bytes, 32 of them per step."""
+    per_group = (2 * 2048 * 128 * 2 + 16 * 64 * 2 * 128 * 2 + 512 * 2 * 128 * 2
+                 + 8 * (128 * 2 + 3 * 4 + 128 * 4))
+    assert per_group == 1_841_248
+    assert bench.nsa_bytes(W.NSA) == 8 * 4 * per_group == 58_919_936
+
+
+def test_csa_decode_bytes():
+    """32 queries over 32768 compressed e4m3 keys (131072 raw tokens, 4:1),
+    then 2048 selected entries plus a 128-token raw window, each a 512-wide
+    bf16 row plus the 64 dims read as its RoPE key."""
+    keys, rows = bench.csa_bytes(W.CSA)
+    assert keys == 32 * (131072 // 4) * 128 == 134_217_728
+    assert rows == 32 * (2048 + 128) * (512 + 64) * 2 == 80_216_064
