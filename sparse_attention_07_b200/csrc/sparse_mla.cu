@@ -15,7 +15,7 @@
 //  * Prologue: the pool rows of all of the CTA's selected slots go into a table
 //    in shared memory (-1 for padded slots); the gather loop then does no
 //    dependent global loads.
-//  * Three producer warps gather the CTA's slice of every selected row with
+//  * Six producer warps gather the CTA's slice of every selected row with
 //    16-byte cp.async (one warp instruction per 512-byte row slice, written in
 //    the 128-byte swizzled layout the tensor cores read) into a 5-stage ring of
 //    64-key tiles; padded slots are zero-filled without a read.
@@ -57,7 +57,7 @@ constexpr int kORowBytes = 256 * 4 + 16;  // one head's output row staged in sha
 constexpr int kSmxWarps = 4;
 constexpr int kXchgWarp0 = kSmxWarps;
 constexpr int kProdWarp0 = kXchgWarp0 + 4;
-constexpr int kProdWarps = 3;
+constexpr int kProdWarps = 6;
 constexpr int kMmaWarp = kProdWarp0 + kProdWarps;
 constexpr int kThreads = 32 * (kMmaWarp + 1);
 constexpr uint32_t kTmemCols = 512;
