@@ -210,6 +210,37 @@ def absorb(U_K, q):
     return _f64(U_K).T @ _f64(q)
 
 
+def up_project(U_V, o_lat):
+    """[MLA-S] "“吸收矩阵”是交换线性计算的顺序": the output of a head is
+    U_V applied to its latent aggregate, o_h = U_V,h (sum_j a_j c_j), which
+    equals sum_j a_j (U_V,h c_j).  U_V [H, d_v, d_c], o_lat [rows, H, d_c]
+    -> [rows, H, d_v] float64."""
+    U, o = _f64(U_V), _f64(o_lat)
+    rows, H, _ = o.shape
+    out = np.zeros((rows, H, U.shape[1]))
+    for r in range(rows):
+        for h in range(H):
+            out[r, h] = U[h] @ o[r, h]
+    return out
+
+
+def mla_chain(q_c, U_K, U_V, q_rope, c, kr, sel, scale: float):
+    """The absorbed MLA decode of [MLA-S] end to end: per head the absorbed
+    query U_K,h^T q^C_h (absorb), sparse MLA over the selected latent rows
+    (sparse_mla), then the up-projection U_V,h (up_project).
+    q_c [rows, H, d_C], U_K [H, d_C, d_c], U_V [H, d_v, d_c], q_rope
+    [rows, H, d_R], c [n, d_c], kr [n, d_R], sel [rows, k] (-1 = empty).
+    Returns [rows, H, d_v] float64."""
+    qc, Uk = _f64(q_c), _f64(U_K)
+    rows, H, _ = qc.shape
+    q_lat = np.zeros((rows, H, Uk.shape[2]))
+    for r in range(rows):
+        for h in range(H):
+            q_lat[r, h] = absorb(Uk[h], qc[r, h])
+    o_lat, _ = sparse_mla(q_lat, q_rope, c, kr, sel, scale)
+    return up_project(U_V, o_lat)
+
+
 def dense_mass(alpha_dense, selected) -> float:
     """[Notes] §6: Z_i = sum_{j in S_i} alpha_ij."""
     a = _f64(alpha_dense)
@@ -260,24 +291,35 @@ def nsa_select_scores(p_cmp, l: int, d: int, l_sel: int):
     return out
 
 
+def bf16_round(x) -> np.ndarray:
+    """Round float64 values to the nearest bfloat16 value, ties to the even
+    significand: bf16 keeps 8 significant bits (1 implicit + 7 stored) with
+    the fp32 exponent range, so the step in the binade [2^e, 2^(e+1)) is
+    2^(e-7) and below 2^-126 (the subnormals) it is 2^-133.  Values are
+    returned as float64 holding the rounded value (finite inputs whose
+    rounding stays below the bf16 maximum)."""
+    x = _f64(x)
+    out = np.zeros_like(x)
+    nz = x != 0.0
+    _, ex = np.frexp(x[nz])                      # |x| = f * 2^ex, 0.5 <= f < 1
+    step_exp = np.maximum(ex.astype(np.int64) - 1, -126) - 7
+    q = np.ldexp(x[nz], -step_exp)               # exact: scaling by a power of two
+    out[nz] = np.ldexp(np.round(q), step_exp)    # np.round: half to even
+    return out
+
+
 def nsa_compress(X, block: int) -> np.ndarray:
     """The NSA compressed cache as stored: the mean of each complete block of
     rows of X [L, D] ([Ch11] §12.6 mean compression), kept in bf16 like the
-    token cache it summarises.  Rounding the mean to bf16 is a quantisation,
-    so it is taken in the precision the stored cache is built in: an fp32 sum
-    over the block's rows in token order, times 1/block, rounded to the
-    nearest bf16 (ties to even).  Returns [L // block, D] float64 holding
-    bf16 values."""
-    import torch
-    X = np.asarray(X, dtype=np.float32)
+    token cache it summarises, i.e. the block mean rounded to the nearest
+    bf16 value (ties to even).  The mean is taken in float64: for bf16 inputs
+    whose magnitudes within a block span less than 2^45 the float64 sum is
+    exact, so this is the exact mean rounded once.  Returns [L // block, D]
+    float64 holding bf16 values."""
+    X = _f64(X)
     nb = X.shape[0] // block
-    out = np.zeros((nb, X.shape[1]), dtype=np.float32)
-    for n in range(nb):
-        acc = np.zeros(X.shape[1], dtype=np.float32)
-        for i in range(block):
-            acc = acc + X[n * block + i]
-        out[n] = acc * np.float32(1.0 / block)
-    return torch.from_numpy(out).to(torch.bfloat16).to(torch.float64).numpy()
+    mean = X[: nb * block].reshape(nb, block, X.shape[1]).sum(axis=1) / block
+    return bf16_round(mean)
 
 
 def nsa_combine(o_cmp, o_sel, o_win, gates):
@@ -409,13 +451,13 @@ def pool_rows(page_table, pages_per_seq: int, seq: int, positions) -> np.ndarray
     return phys * PAGE + pos % PAGE
 
 
-def dsa_step(inp: dict, rows: Sequence[int], with_scores: bool = True) -> dict:
+def dsa_step(inp: dict, rows: Sequence[int], with_scores: bool = True, with_attention: bool = True) -> dict:
     """Indexer -> Top-K -> sparse MLA for the chosen query rows of a workload.
 
     ``inp`` is a dict made by ``workloads.dsa_inputs``.  Returns, per chosen
     row (in the order given): ``scores`` [n_rows, L_max] (NaN past the visible
-    length), ``idx`` [n_rows, k] int32 and ``out`` [n_rows,H,d_c], ``lse``
-    [n_rows,H] float64.
+    length), ``idx`` [n_rows, k] int32 and, unless ``with_attention`` is
+    False, ``out`` [n_rows,H,d_c], ``lse`` [n_rows,H] float64.
     """
     import torch
     cfg = inp["cfg"]
@@ -441,6 +483,8 @@ def dsa_step(inp: dict, rows: Sequence[int], with_scores: bool = True) -> dict:
     key0 = np.array([key0_of_seq[int(sor[r])] for r in rows], dtype=np.int64)
     scores = index_scores(q, w, keys, key0, n_vis, out_ld=cfg.L_max)
     idx = topk(np.nan_to_num(scores, nan=-np.inf), n_vis, cfg.topk)
+    if not with_attention:
+        return dict(idx=idx, scores=scores, n_visible=n_vis)
     # gather the selected latent rows of every chosen query row
     sel = np.full(idx.shape, -1, dtype=np.int64)
     flat = []
@@ -502,7 +546,7 @@ def csa_step(inp: dict, rows: Sequence[int]) -> dict:
     for r in rows:
         kv = csa_compress(*(_host64(inp[n][r]) for n in ("Ca", "Cb", "Za", "Zb")), _host64(inp["Ba"]),
                           _host64(inp["Bb"]), cfg.m)
-        kv = torch.from_numpy(kv).to(torch.bfloat16).to(torch.float64).numpy()
+        kv = bf16_round(kv)  # the entries are stored in bf16
         ki = csa_compress(*(_host64(inp[n][r]) for n in ("CIa", "CIb", "ZIa", "ZIb")), _host64(inp["BIa"]),
                           _host64(inp["BIb"]), cfg.m)
         ki = torch.from_numpy(ki).to(torch.float8_e4m3fn).to(torch.float64).numpy()

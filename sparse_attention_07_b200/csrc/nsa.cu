@@ -54,6 +54,21 @@ constexpr int kMaxG = 16;
 constexpr float kLog2e = 1.4426950408889634f;
 
 // --------------------------------------------------------------- compression
+// Bits of the bf16 value nearest to x (ties to the even significand), for
+// finite x whose rounding stays within the bf16 range: bf16 keeps 8
+// significant bits with the fp32 exponent range, so the step in the binade
+// [2^e, 2^(e+1)) is 2^(e-7), and 2^-133 among the subnormals.  Scaling by
+// that step is exact, rint() rounds half to even, and the rounded value is
+// exact in fp32, whose upper 16 bits are then the bf16 encoding.
+__device__ __forceinline__ uint32_t bf16_bits_rn(double x) {
+    if (x == 0.0) return __double_as_longlong(x) < 0 ? 0x8000u : 0u;
+    int ex;
+    (void)frexp(x, &ex);  // |x| = f * 2^ex, 0.5 <= f < 1
+    const int step = max(ex - 1, -126) - 7;
+    const double r = ldexp(rint(ldexp(x, -step)), step);
+    return __float_as_uint(static_cast<float>(r)) >> 16;
+}
+
 __global__ void __launch_bounds__(256) nsa_compress_kernel(const __nv_bfloat16* __restrict__ K,
                                                            const __nv_bfloat16* __restrict__ V, int64_t sb,
                                                            int64_t st, int64_t sh, int Hkv, int nb, int block,
@@ -69,21 +84,24 @@ __global__ void __launch_bounds__(256) nsa_compress_kernel(const __nv_bfloat16* 
     const int h = static_cast<int>((u / nb) % Hkv);
     const int64_t b = u / (static_cast<int64_t>(nb) * Hkv);
     const __nv_bfloat16* src = (which ? V : K) + b * sb + h * sh + static_cast<int64_t>(n) * block * st + lane * 4;
-    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+    // fp64 sums in token order: a bf16 value has 8 significant bits, so the
+    // sum of a block whose magnitudes span less than 2^45 is exact, and the
+    // stored value is the exact mean rounded once to bf16
+    double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
 #pragma unroll 8
-    for (int i = 0; i < block; ++i) {  // token order, plain fp32 adds
+    for (int i = 0; i < block; ++i) {
         const uint2 raw = *reinterpret_cast<const uint2*>(src + i * st);
         const __nv_bfloat162 x = *reinterpret_cast<const __nv_bfloat162*>(&raw.x);
         const __nv_bfloat162 y = *reinterpret_cast<const __nv_bfloat162*>(&raw.y);
-        a0 = __fadd_rn(a0, __low2float(x));
-        a1 = __fadd_rn(a1, __high2float(x));
-        a2 = __fadd_rn(a2, __low2float(y));
-        a3 = __fadd_rn(a3, __high2float(y));
+        a0 += static_cast<double>(__low2float(x));
+        a1 += static_cast<double>(__high2float(x));
+        a2 += static_cast<double>(__low2float(y));
+        a3 += static_cast<double>(__high2float(y));
     }
-    const float inv = 1.f / static_cast<float>(block);
+    const double nblk = static_cast<double>(block);
     uint2 o;
-    o.x = pack_bf16x2(__fmul_rn(a0, inv), __fmul_rn(a1, inv));
-    o.y = pack_bf16x2(__fmul_rn(a2, inv), __fmul_rn(a3, inv));
+    o.x = bf16_bits_rn(a0 / nblk) | (bf16_bits_rn(a1 / nblk) << 16);
+    o.y = bf16_bits_rn(a2 / nblk) | (bf16_bits_rn(a3 / nblk) << 16);
     __nv_bfloat16* dst = (which ? Vc : Kc) + ((b * Hkv + h) * c_ld + n) * kD + lane * 4;
     *reinterpret_cast<uint2*>(dst) = o;
 }

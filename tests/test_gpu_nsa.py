@@ -1,8 +1,9 @@
 """GPU parity: the NSA compressed cache and the NSA three-branch decode
 against the fp64 oracle.
 
-The compressed cache is a bf16 quantisation taken in fp32 on both sides, so
-it must match bit for bit.  The group's block choice of N(0,1) inputs is
+The compressed cache is the exact block mean rounded once to bf16 on both
+sides (the kernel's fp64 block sums are exact for these inputs), so it must
+match bit for bit.  The group's block choice of N(0,1) inputs is
 compared as a set; a block may differ only where fp32 and fp64 order two
 near-tied group probabilities differently (oracle probability within
 TIE_REL * max of the boundary one), and the output is then compared with the

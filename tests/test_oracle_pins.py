@@ -55,6 +55,47 @@ def test_absorbed_identity_random():
     np.testing.assert_allclose(out[0, 0], ref, rtol=0, atol=1e-12)
 
 
+def test_up_project_by_hand():
+    """[MLA-S] up-projection o = U_V o_lat on a 3x2 U_V worked by hand:
+    rows (1, 0), (0, 2), (1, 1) applied to (2, -1) give (2, -2, 1); a second
+    head with its own U_V = identity keeps its latent."""
+    U = np.array([[[1.0, 0.0], [0.0, 2.0], [1.0, 1.0]], [[1.0, 0.0], [0.0, 1.0], [0.0, 0.0]]])
+    o = np.array([[[2.0, -1.0], [5.0, 7.0]]])
+    got = oracle.up_project(U, o)
+    assert got.shape == (1, 2, 3)
+    assert got[0, 0].tolist() == [2.0, -2.0, 1.0]
+    assert got[0, 1].tolist() == [5.0, 7.0, 0.0]
+
+
+def test_mla_chain_equals_explicit_keys_and_values():
+    """[MLA-S] "“吸收矩阵”是交换线性计算的顺序": the absorbed chain (U_K^T q^C
+    as the query of the latent rows, latent aggregate, then U_V) equals
+    attention computed without absorption, with explicit content keys
+    k^C_j = U_K c_j, the RoPE keys, and values v_j = U_V c_j
+    (sum_j a_j U_V c_j = U_V sum_j a_j c_j).  Random inputs, empty slots,
+    several heads with their own U_K and U_V."""
+    rng = np.random.default_rng(17)
+    rows, H, d_C, d_c, d_R, d_v, n, k = 2, 3, 6, 10, 4, 5, 23, 9
+    q_c = rng.standard_normal((rows, H, d_C))
+    U_K = rng.standard_normal((H, d_C, d_c))
+    U_V = rng.standard_normal((H, d_v, d_c))
+    q_r = rng.standard_normal((rows, H, d_R))
+    c = rng.standard_normal((n, d_c))
+    kr = rng.standard_normal((n, d_R))
+    sel = rng.choice(n, size=(rows, k), replace=True)
+    sel[1, ::4] = -1
+    scale = 1.0 / math.sqrt(d_C + d_R)
+    got = oracle.mla_chain(q_c, U_K, U_V, q_r, c, kr, sel, scale)
+    for r in range(rows):
+        js = [j for j in sel[r] if j >= 0]
+        for h in range(H):
+            z = np.array([(q_c[r, h] @ (U_K[h] @ c[j]) + q_r[r, h] @ kr[j]) * scale for j in js])
+            a = np.exp(z - z.max())
+            a /= a.sum()
+            want = sum(a_j * (U_V[h] @ c[j]) for a_j, j in zip(a, js))
+            np.testing.assert_allclose(got[r, h], want, rtol=0, atol=1e-12)
+
+
 def test_content_plus_position_example(golden_dir):
     """MLA-S "分开以后": content 1,1 + RoPE 0,2, /sqrt(4) -> 0.5,1.5 -> 0.269,0.731."""
     g = _golden(golden_dir, "content_position.json")
@@ -457,24 +498,51 @@ def test_nsa_gates_mix_linearly_and_short_history_has_only_the_window():
     np.testing.assert_allclose(out, g[:, 2:3] * _sdpa(q, K[12:20], V[12:20], 0.25), atol=1e-12)
 
 
+def test_bf16_round_matches_torch_and_breaks_ties_to_even():
+    """oracle.bf16_round against torch's float32 -> bfloat16 conversion (one
+    round-to-nearest-even step; every float32 is exact in float64), and on
+    hand-made ties: 1 + 2^-8 lies halfway between 1 and 1 + 2^-7 and goes to
+    the even significand 1; 1 + 3*2^-8 goes to 1 + 2^-6; a subnormal tie
+    3*2^-134 goes to 2^-132."""
+    g = torch.Generator().manual_seed(5)
+    x = torch.cat([torch.randn(20000, generator=g) * 10.0 ** torch.randint(-30, 30, (20000,), generator=g),
+                   torch.randn(2000, generator=g) * 2.0 ** -130])
+    want = x.to(torch.bfloat16).to(torch.float64).numpy()
+    np.testing.assert_array_equal(oracle.bf16_round(x.to(torch.float64).numpy()), want)
+    ties = np.array([1 + 2.0 ** -8, 1 + 3 * 2.0 ** -8, -(1 + 2.0 ** -8), 3 * 2.0 ** -134, 0.0, -0.0])
+    np.testing.assert_array_equal(oracle.bf16_round(ties),
+                                  [1.0, 1 + 2.0 ** -6, -1.0, 2.0 ** -132, 0.0, 0.0])
+    # just off the tie: the nearer neighbour
+    assert oracle.bf16_round(np.array([1 + 2.0 ** -8 + 2.0 ** -30]))[0] == 1 + 2.0 ** -7
+
+
 def test_nsa_compress_stored_cache():
-    """The stored cache is the block mean rounded to bf16: exact on blocks of
-    small integers (their fp32 sums are exact), equal to torch's fp64 mean
-    rounded to bf16 on N(0,1) bf16 data except where that mean sits within an
-    fp32 rounding of a bf16 tie, and never more than half a bf16 ulp (plus
-    the fp32 sum's error) away from the exact mean."""
+    """The stored cache is the exact block mean rounded to the nearest bf16
+    ([Ch11] §12.6 mean compression, kept in the token cache's bf16): exact on
+    blocks of small integers (their means are multiples of 1/64, exact in
+    fp32, so torch's conversion rounds them once); on N(0,1) bf16 data each
+    entry is the bf16 value nearest to the exact rational mean (computed with
+    fractions), ties to even."""
+    from fractions import Fraction
     g = torch.Generator().manual_seed(21)
     Xi = torch.randint(-8, 9, (4 * 64 + 17, 32), generator=g).to(torch.float64)
-    want = Xi[:256].reshape(4, 64, 32).mean(dim=1).to(torch.bfloat16).to(torch.float64).numpy()
+    want = Xi[:256].reshape(4, 64, 32).mean(dim=1).to(torch.float32).to(torch.bfloat16).to(torch.float64).numpy()
     np.testing.assert_array_equal(oracle.nsa_compress(Xi.numpy(), 64), want)
-    X = torch.randn(64 * 40, 128, generator=g).to(torch.bfloat16).to(torch.float64)
-    exact = X.reshape(40, 64, 128).mean(dim=1)
-    got = oracle.nsa_compress(X.numpy(), 64)
-    ref = exact.to(torch.bfloat16).to(torch.float64).numpy()
-    assert (got == ref).mean() > 0.999
-    ulp = 2.0 ** (np.floor(np.log2(np.maximum(np.abs(exact.numpy()), 1e-30))) - 7)
-    assert np.all(np.abs(got - exact.numpy()) <= 0.5 * ulp + 1e-6)
-    assert oracle.nsa_compress(X.numpy()[:63], 64).shape == (0, 128)
+    X = torch.randn(64 * 6, 16, generator=g).to(torch.bfloat16).to(torch.float64).numpy()
+    got = oracle.nsa_compress(X, 64)
+    assert got.shape == (6, 16)
+    for n in range(6):
+        for d in range(16):
+            exact = sum(Fraction(v) for v in X[n * 64:(n + 1) * 64, d]) / 64
+            v = Fraction(got[n, d])
+            # the bf16 step in the exact mean's binade (no subnormals here)
+            step = Fraction(2) ** (math.floor(math.log2(abs(float(exact)))) - 7)
+            assert (v / step).denominator == 1  # v is on that grid (or the binade edge)
+            err = abs(exact - v)
+            assert err <= step / 2
+            if err == step / 2:  # a tie: the even significand
+                assert (v / step).numerator % 2 == 0
+    assert oracle.nsa_compress(X[:63], 64).shape == (0, 16)
 
 
 # ------------------------------------------------------------ CSA compression
