@@ -1,8 +1,7 @@
 """GPU parity: the per-head projections around sparse MLA (query absorption
-with U_K, up-projection with U_V) against the fp64 oracle, the pages' worked
-absorption example on the GPU, and the whole chain q^C -> q_lat -> sparse MLA
--> U_V against attention computed with explicit content keys U_K c_j and
-values U_V c_j."""
+with U_K, up-projection with U_V) against the fp64 oracle (oracle.absorb,
+oracle.up_project), the pages' worked absorption example on the GPU, and the
+whole chain q^C -> q_lat -> sparse MLA -> U_V against oracle.mla_chain."""
 import json
 import os
 
@@ -50,11 +49,12 @@ def test_up_project_vs_oracle(rows, H):
     o_lat = torch.randn(rows, H, d_c, generator=g, device=DEV) * 0.1
     U_V = _bf16((H, d_v, d_c), g, 1.0 / np.sqrt(d_c))
     got = _f64(sa.mla_up_project(o_lat, U_V))
-    o_b = _f64(o_lat.to(torch.bfloat16))  # the kernel's operand rounding
-    ref = np.einsum("hvj,rhj->rhv", _f64(U_V), o_b)
+    # the kernel's tensor-core operand is the latent output rounded to bf16
+    o_b = _f64(o_lat.to(torch.bfloat16))
+    ref = oracle.up_project(_f64(U_V), o_b)
     assert np.abs(got - ref).max() <= 1e-5 + 1e-5 * np.abs(ref).max()
     # and against the unrounded latent output: within the bf16 input rounding
-    ref32 = np.einsum("hvj,rhj->rhv", _f64(U_V), _f64(o_lat))
+    ref32 = oracle.up_project(_f64(U_V), _f64(o_lat))
     assert np.abs(got - ref32).max() <= 2e-3
     assert sa.check_device_error() == 0
 
@@ -77,8 +77,9 @@ def test_absorbed_example_on_the_gpu():
 
 
 def test_absorb_mla_up_chain():
-    """q^C -> absorbed query -> sparse MLA -> U_V equals attention with explicit
-    content keys k^C_j = U_K c_j and values v_j = U_V c_j."""
+    """q^C -> absorbed query -> sparse MLA -> U_V on the GPU against the
+    oracle's absorbed chain (itself pinned to the explicit-keys form
+    k^C_j = U_K c_j, v_j = U_V c_j)."""
     g = torch.Generator(device=DEV)
     g.manual_seed(21)
     rows, H, d_C, d_c, d_R, d_v, n = 2, 16, 128, 512, 64, 128, 300
@@ -96,17 +97,8 @@ def test_absorb_mla_up_chain():
     q_lat = sa.mla_absorb_query(q_c, U_K)
     o_lat = sa.sparse_mla_decode(q_lat, q_rope, c, kr, idx, scale, pages_per_seq=pool // 64, seq_of_row=seq)
     out = _f64(sa.mla_up_project(o_lat, U_V))
-    qn, Uk, Uv, qr, cn, krn = _f64(q_c), _f64(U_K), _f64(U_V), _f64(q_rope), _f64(c), _f64(kr)
-    ref = np.zeros((rows, H, d_v))
-    for r in range(rows):
-        sel = idx[r].cpu().numpy()
-        sel = sel[sel >= 0]
-        for h in range(H):
-            kc = cn[sel] @ Uk[h].T                     # k^C_j = U_K c_j
-            z = (kc @ qn[r, h] + krn[sel] @ qr[r, h]) * scale
-            a = np.exp(z - z.max())
-            a /= a.sum()
-            ref[r, h] = a @ (cn[sel] @ Uv[h].T)        # v_j = U_V c_j
+    sel = idx.cpu().numpy().astype(np.int64)  # one sequence: pool row = position
+    ref = oracle.mla_chain(_f64(q_c), _f64(U_K), _f64(U_V), _f64(q_rope), _f64(c), _f64(kr), sel, scale)
     # q_lat is rounded to bf16 before the scores and o_lat before U_V
     assert_attention_close(out, ref, "absorb -> sparse MLA -> U_V")
     assert sa.check_device_error() == 0
