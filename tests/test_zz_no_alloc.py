@@ -22,8 +22,11 @@ FAKE = ctypes.c_void_p(0x1000)  # aligned, never dereferenced: the call rejects 
 
 @pytest.mark.gpu
 def test_static_scratch_decode_matches_workspace_decode():
-    from _gpu import MLA_MAX_ABS, MLA_MEAN_ABS, LSE_ABS
-
+    """Two calls in a row through the static array against the workspace
+    call: the same kernels with the same key split and a combine that adds the
+    splits in a fixed order, so the outputs and LSEs must be identical bit for
+    bit (a tolerance would hide stale scratch contents or a race on the
+    array).  The outputs start as NaN so a value not written shows up."""
     cfg = W.small_dsa(W.LONG, n_seqs=3, rows=3, lens=(5000, 2100, 4097), topk=2048)
     inp = W.dsa_inputs(cfg, DEV, seed=31)
     need = sa.sparse_mla_workspace_size(cfg.rows, cfg.H, cfg.topk, cfg.d_c)
@@ -43,15 +46,10 @@ def test_static_scratch_decode_matches_workspace_decode():
         outs.append((out, lse))
     torch.cuda.synchronize()
     assert sa.check_device_error() == 0
-
-    want = ref.double().cpu().numpy()
-    want_lse = lse_ref.double().cpu().numpy()
+    assert torch.isfinite(ref).all()
     for out, lse in outs:
-        got = out.double().cpu().numpy()
-        assert np.isfinite(got).all()
-        err = np.abs(got - want)
-        assert err.max() <= MLA_MAX_ABS and err.mean() <= MLA_MEAN_ABS, (err.max(), err.mean())
-        assert np.abs(lse.double().cpu().numpy() - want_lse).max() <= LSE_ABS
+        assert torch.equal(out, ref), (out - ref).abs().max().item()
+        assert torch.equal(lse, lse_ref)
 
 
 def test_static_scratch_rejects_shapes_beyond_the_array():
