@@ -40,7 +40,7 @@ L2_FLUSH_BYTES = 256 << 20  # > 126 MB L2
 # kernel of a workload, from one ncu capture, with the sha256 prefix of the
 # kernel source it was taken on (the figure is reported only while they match).
 TRAFFIC = {
-    "long": {"kernel": "sparse_mla.cu", "bytes_per_launch": 83550720, "src_sha": "8f5c50233ab005df"},
+    "long": {"kernel": "sparse_mla.cu", "stage": "attn", "bytes_per_launch": 83550720, "src_sha": "8f5c50233ab005df"},
     "nsa": {"kernel": "nsa.cu", "bytes_per_launch": 59232768, "src_sha": "46cccc0328e4c5e2"},
 }
 
@@ -68,12 +68,34 @@ def prefill_flops(cfg: W.DSAConfig):
     return idx, mla
 
 
-def block_bytes(cfg: W.BlockConfig):
-    """Pooled-key scan plus the union's K and V rows, for every (sequence, head)."""
-    pooled = cfg.B * cfg.H * cfg.n_blocks * cfg.D * 4
-    # the union holds at most top*block + sink*block + window tokens
-    u_max = min(cfg.L, cfg.top_blocks * cfg.block + cfg.sink_blocks * cfg.block + cfg.window)
-    return pooled, u_max
+def block_union_tokens(cfg: W.BlockConfig, sel: np.ndarray) -> int:
+    """Tokens attended over all (sequence, head) pairs: the union of the
+    chosen blocks (sel [B, H, top], -1 padded), the sink blocks and the
+    window, each token counted once per pair."""
+    total = 0
+    w0 = max(0, cfg.L - cfg.window)
+    for b in range(sel.shape[0]):
+        for h in range(sel.shape[1]):
+            m = np.zeros(cfg.L, dtype=bool)
+            m[w0:] = True
+            m[: min(cfg.L, cfg.sink_blocks * cfg.block)] = True
+            for n in sel[b, h]:
+                if n >= 0:
+                    m[n * cfg.block:(n + 1) * cfg.block] = True
+            total += int(m.sum())
+    return total
+
+
+def block_bytes(cfg: W.BlockConfig, union_tokens: int):
+    """Algorithmic bytes of one block-sparse decode step: for every (sequence,
+    head) the pooled keys of every complete block (fp32), the K and V rows of
+    the attended union (bf16), the query and the output; `union_tokens` is
+    the union size summed over the pairs.  Returns (bytes, union_tokens)."""
+    pairs = cfg.B * cfg.H
+    pooled = pairs * cfg.n_blocks * cfg.D * 4
+    kv = union_tokens * 2 * cfg.D * 2
+    qo = pairs * cfg.D * (2 + 4)
+    return pooled + kv + qo, union_tokens
 
 
 def nsa_bytes(cfg: W.NSAConfig):
@@ -235,6 +257,11 @@ class BlockStep:
         self.pooled = sa.block_mean_pool(inp["K"], c.block)  # once, when the blocks completed
         self.out = torch.empty(c.B, c.H, c.D, dtype=torch.float32, device=inp["q"].device)
         self.launches_per_step = 1
+        # the union each pair attends to (for the byte model), from one call outside the timing
+        sel = torch.empty(c.B, c.H, c.top_blocks, dtype=torch.int32, device=inp["q"].device)
+        sa.block_sparse_attn(inp["q"], self.pooled, inp["K"], inp["V"], c.block, c.top_blocks, c.sink_blocks,
+                             c.window, c.scale, out=self.out, sel_blocks=sel)
+        self.union_tokens = block_union_tokens(c, sel.cpu().numpy())
 
     def indexer(self):
         i, c = self.inp, self.cfg
@@ -466,18 +493,26 @@ def cpu_baseline(inp, cfg, budget_s: float = 12.0):
     threads = oracle.threads()
     if isinstance(cfg, W.DSAConfig):
         rows_all = list(range(cfg.rows))
-        t0 = time.perf_counter()
-        oracle.dsa_step(inp, rows_all[:1], with_scores=False)
-        one = time.perf_counter() - t0
-        n = int(max(1, min(len(rows_all), threads * max(1, budget_s // max(one * 1.0, 1e-3) // 1))))
-        n = max(1, min(n, len(rows_all), threads * 4))
-        rows = rows_all[:n]
-        t0 = time.perf_counter()
-        oracle.dsa_step(inp, rows, with_scores=False)
-        dt = time.perf_counter() - t0
-        unit_n = n
         what = "query rows" if cfg.prefill_start < 0 else "query tokens"
+
+        def timed(n_threads, budget):
+            oracle.set_threads(n_threads)
+            t0 = time.perf_counter()
+            oracle.dsa_step(inp, rows_all[:1], with_scores=False)
+            one = time.perf_counter() - t0
+            n = int(max(1, min(len(rows_all), n_threads * 4, n_threads * (budget // max(one, 1e-3)))))
+            t0 = time.perf_counter()
+            oracle.dsa_step(inp, rows_all[:n], with_scores=False)
+            return n, time.perf_counter() - t0
+
+        n, dt = timed(threads, budget_s)
+        n1, dt1 = timed(1, budget_s * 0.6)
+        oracle.set_threads(threads)
+        unit_n = n
         sample = f"{n} of {cfg.rows} {what} of the workload (indexer over every visible key, top-{cfg.topk}, sparse MLA)"
+        return {"value": unit_n / dt, "cores": threads, "kind": "oracle", "sample": sample, "seconds": round(dt, 3),
+                "one_core": {"value": n1 / dt1, "cores": 1, "seconds": round(dt1, 3),
+                             "sample": f"{n1} of {cfg.rows} {what}, the same oracle limited to one host thread"}}
     elif isinstance(cfg, W.CSAConfig):
         t0 = time.perf_counter()
         oracle.csa_step(inp, [0])
@@ -550,30 +585,26 @@ def describe(cfg, flush_note):
             "batch": cfg.B, "seq_len": cfg.L, "heads": cfg.H, "l2": flush_note}
 
 
-def run_native(args):
-    ws, rank, local = dist_env()
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if ws > 1:
-        import datetime
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
-    import sparse_attention_07_b200 as sa
-    sa.lib()
-    cfg = workload(args.config)
+def make_step(cfg, dev, rank, sa):
+    """Seeded inputs of a workload (each rank its own seed) and its step."""
     if isinstance(cfg, W.DSAConfig):
         inp = W.dsa_inputs(cfg, dev, seed=rank_seed(cfg.seed, rank))
-        step = DecodeStep(inp, sa)
-    elif isinstance(cfg, W.NSAConfig):
+        return inp, DecodeStep(inp, sa)
+    if isinstance(cfg, W.NSAConfig):
         inp = W.nsa_inputs(cfg, dev, seed=rank_seed(cfg.seed, rank))
-        step = NsaStep(inp, sa)
-    elif isinstance(cfg, W.CSAConfig):
+        return inp, NsaStep(inp, sa)
+    if isinstance(cfg, W.CSAConfig):
         inp = W.csa_inputs(cfg, dev, seed=rank_seed(cfg.seed, rank))
-        step = CsaStep(inp, sa)
-    else:
-        inp = W.block_inputs(cfg, dev, seed=rank_seed(cfg.seed, rank))
-        step = BlockStep(inp, sa)
-    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+        return inp, CsaStep(inp, sa)
+    inp = W.block_inputs(cfg, dev, seed=rank_seed(cfg.seed, rank))
+    return inp, BlockStep(inp, sa)
+
+
+def measure(cfg, args, dev, local, rank, ws, sa, flush, config_key):
+    """Warm-up, then the timed steps (graph replays), the per-stage steps and
+    the end-to-end steps of one workload; returns the result fields of its
+    JSON line (without the top-level run keys) and the inputs."""
+    inp, step = make_step(cfg, dev, rank, sa)
     for _ in range(args.warmup):
         flush.zero_()
         step.indexer()
@@ -593,6 +624,7 @@ def run_native(args):
         step_ms, stage_ms = time_steps(step, args.steps, flush)
     if graph_ms is not None:
         step_ms = graph_ms
+    del graph
     if ws > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
@@ -608,7 +640,7 @@ def run_native(args):
     first = t_idx
 
     hbm, bf16_burst, bf16_sus, peak_src = peaks()
-    res = {"impl": "native"}
+    res = {}
     if isinstance(cfg, W.DSAConfig):
         prefill = cfg.prefill_start >= 0
         units = cfg.rows * ws
@@ -616,49 +648,59 @@ def run_native(args):
         metric = "sparse-MLA prefill tokens/s (indexer+topk+attn)" if prefill else DECODE_METRIC
         keys_b, rows_b = decode_bytes(cfg)
         score_b = int(cfg.n_visible().sum()) * 4
-        fi, fm = prefill_flops(cfg)
-        # a prefill step lasts milliseconds (sustained peak); a decode step is a short burst
-        bf16_peak = bf16_sus if prefill else bf16_burst
-        fp8_peak = bf16_peak * 2.0  # fp8 dense rate = 2x bf16 (nominal ratio)
-        kern = {
-            "indexer": {"kernel": "idx_tc_kernel" if cfg.idx_dtype == "e4m3" else "idx_cc_kernel", "us": t_idx * 1e3,
-                        "bytes": keys_b, "flop": fi, "flop_peak": fp8_peak},
-            "topk": {"kernel": "topk_kernel", "us": t_topk * 1e3, "bytes": score_b},
-            "attn": {"kernel": "mla_kernel" + ("" if prefill else " (+ mla_combine_kernel)"), "us": t_attn * 1e3,
-                     "bytes": rows_b, "flop": fm, "flop_peak": bf16_peak},
-        }
-        for v in kern.values():
-            v["hbm_gbs"] = round(v["bytes"] / (v["us"] * 1e-6) / 1e9, 1)
-            v["hbm_frac"] = round(v["hbm_gbs"] / hbm, 4)
-            if "flop" in v:
-                v["tflops"] = round(v["flop"] / (v["us"] * 1e-6) / 1e12, 1)
-            v["us"] = round(v["us"], 2)
-        dom_name = max(kern, key=lambda n: kern[n]["us"])
-        dom = kern[dom_name]
-        tr = TRAFFIC.get(args.config, {})
-        traffic = None
-        if tr.get("bytes_per_launch") and tr.get("src_sha") == src_sha(
-                "sparse_attention_07_b200/csrc/" + tr.get("kernel", "")) and dom_name == "attn":
-            traffic = tr["bytes_per_launch"]
         if prefill:
-            # both big kernels are contractions: the roofline is the tensor pipe
-            peak = dom["flop_peak"]
-            roof = {"bound": "tensor", "achieved": dom["tflops"], "peak": peak, "unit": "TFLOP/s",
-                    "frac": round(dom["tflops"] / peak, 4), "traffic": traffic, "kernel": dom["kernel"],
-                    "peak_source": (f"{peak_src} bf16 sustained x 2 (nominal fp8/bf16 ratio)"
-                                    if dom_name == "indexer" else f"{peak_src} bf16 sustained")}
+            # a compute-bound chunk: both big kernels are contractions, so they
+            # are reported against the tensor pipe (the sustained peak: the
+            # chunk lasts milliseconds); fp8 = 2x bf16 (nominal ratio)
+            fi, fm = prefill_flops(cfg)
+            kern = {
+                "indexer": {"kernel": "idx_tc_kernel", "us": t_idx * 1e3, "flop": fi, "peak_tflops": bf16_sus * 2.0,
+                            "peak_source": f"{peak_src} bf16 sustained x 2 (nominal fp8/bf16 ratio)"},
+                "topk": {"kernel": "topk_kernel", "us": t_topk * 1e3, "bytes": score_b},
+                "attn": {"kernel": "mla_kernel", "us": t_attn * 1e3, "flop": fm, "peak_tflops": bf16_sus,
+                         "peak_source": f"{peak_src} bf16 sustained"},
+            }
+            for v in kern.values():
+                if "flop" in v:
+                    v["tflops"] = round(v["flop"] / (v["us"] * 1e-6) / 1e12, 1)
+                    v["tensor_frac"] = round(v["tflops"] / v["peak_tflops"], 4)
+                else:
+                    v["hbm_gbs"] = round(v["bytes"] / (v["us"] * 1e-6) / 1e9, 1)
+                    v["hbm_frac"] = round(v["hbm_gbs"] / hbm, 4)
+                v["us"] = round(v["us"], 2)
+            dom_name = max(("indexer", "attn"), key=lambda n: kern[n]["us"])
+            dom = kern[dom_name]
+            roof = {"bound": "tensor", "achieved": dom["tflops"], "peak": dom["peak_tflops"], "unit": "TFLOP/s",
+                    "frac": dom["tensor_frac"], "traffic": None, "kernel": dom["kernel"],
+                    "peak_source": dom["peak_source"]}
         else:
+            kern = {
+                "indexer": {"kernel": "idx_tc_kernel" if cfg.idx_dtype == "e4m3" else "idx_cc_kernel",
+                            "us": t_idx * 1e3, "bytes": keys_b},
+                "topk": {"kernel": "topk_kernel", "us": t_topk * 1e3, "bytes": score_b},
+                "attn": {"kernel": "mla_kernel (+ mla_combine_kernel)", "us": t_attn * 1e3, "bytes": rows_b},
+            }
+            for v in kern.values():
+                v["hbm_gbs"] = round(v["bytes"] / (v["us"] * 1e-6) / 1e9, 1)
+                v["hbm_frac"] = round(v["hbm_gbs"] / hbm, 4)
+                v["us"] = round(v["us"], 2)
+            dom_name = max(kern, key=lambda n: kern[n]["us"])
+            dom = kern[dom_name]
+            tr = TRAFFIC.get(config_key, {})
+            traffic = None
+            if tr.get("bytes_per_launch") and tr.get("stage") == dom_name and tr.get("src_sha") == src_sha(
+                    "sparse_attention_07_b200/csrc/" + tr.get("kernel", "")):
+                traffic = tr["bytes_per_launch"]
             roof = {"bound": "hbm", "achieved": dom["hbm_gbs"], "peak": hbm, "unit": "GB/s",
                     "frac": dom["hbm_frac"], "traffic": traffic, "kernel": dom["kernel"],
                     "peak_source": f"{peak_src} hbm_gbs"}
-        for v in kern.values():
-            v.pop("flop_peak", None)
-        step_gbs = (keys_b + rows_b) / (ms * 1e-3) / 1e9
-        res["step_roofline"] = {"bytes_per_step": keys_b + rows_b, "indexer_key_bytes": keys_b,
-                                "gathered_row_bytes": rows_b, "achieved": round(step_gbs, 1), "peak": hbm,
-                                "unit": "GB/s", "frac": round(step_gbs / hbm, 4)}
+            step_gbs = (keys_b + rows_b) / (ms * 1e-3) / 1e9
+            res["step_roofline"] = {"bytes_per_step": keys_b + rows_b, "indexer_key_bytes": keys_b,
+                                    "gathered_row_bytes": rows_b, "achieved": round(step_gbs, 1), "peak": hbm,
+                                    "unit": "GB/s", "frac": round(step_gbs / hbm, 4),
+                                    "peak_source": f"{peak_src} hbm_gbs"}
         res["kernels"] = kern
-        if not prefill:
+        if not prefill and config_key == "long":
             res["projections"] = time_projections(step, min(args.steps, 20), flush, hbm)
     elif isinstance(cfg, W.CSAConfig):
         units = cfg.n_seqs * ws
@@ -687,7 +729,7 @@ def run_native(args):
         metric = "NSA decode queries/s (compression + group block choice + selection + window, gated)"
         nbytes = nsa_bytes(cfg)
         ach = nbytes / (first * 1e-3) / 1e9
-        tr = TRAFFIC.get(args.config, {})
+        tr = TRAFFIC.get(config_key, {})
         traffic = tr.get("bytes_per_launch") if tr.get("src_sha") == src_sha(
             "sparse_attention_07_b200/csrc/" + tr.get("kernel", "nsa.cu")) else None
         roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": hbm, "unit": "GB/s", "frac": round(ach / hbm, 4),
@@ -697,18 +739,14 @@ def run_native(args):
         units = cfg.B * ws
         unit = "queries/s"
         metric = "block-sparse decode queries/s (pooled-block scan+top-k+block attention)"
-        pooled_b, u_max = block_bytes(cfg)
-        ach = pooled_b / (first * 1e-3) / 1e9
+        nbytes, u_tokens = block_bytes(cfg, step.union_tokens)
+        ach = nbytes / (first * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": hbm, "unit": "GB/s", "frac": round(ach / hbm, 4),
-                "traffic": None, "kernel": "block_sparse_kernel (pooled-key bytes only)",
-                "peak_source": f"{peak_src} hbm_gbs"}
+                "traffic": None, "kernel": "block_sparse_kernel", "bytes_per_launch": nbytes,
+                "union_tokens": u_tokens, "peak_source": f"{peak_src} hbm_gbs"}
     value = units / (ms * 1e-3)
     res.update({
-        "metric": metric, "value": round(value, 1), "unit": unit, "n_gpus": ws, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "e4m3 indexer / bf16 MLA, fp32 accumulate" if isinstance(cfg, (W.DSAConfig, W.CSAConfig))
-        else "bf16, fp32 accumulate",
-        "data": "synthetic (seeded, shapes and value distributions of the workload)",
+        "metric": metric, "value": round(value, 1), "unit": unit, "ms_per_step": round(ms, 5),
         "config": dict(describe(cfg, f"flushed between steps ({L2_FLUSH_BYTES >> 20} MiB write, outside the events)"),
                        timing=("step: one CUDA-graph replay of the step's launches per timed step; stage times: "
                                "the same number of stream-launched steps with an event between stages"
@@ -723,6 +761,39 @@ def run_native(args):
     if ws == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline(inp, cfg)
         res["cpu_baseline"]["unit"] = unit
+    del step
+    return res, inp
+
+
+def run_native(args):
+    ws, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    import sparse_attention_07_b200 as sa
+    sa.lib()
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    cfg = workload(args.config)
+    main_res, inp = measure(cfg, args, dev, local, rank, ws, sa, flush, args.config)
+    del inp
+    res = {"impl": "native"}
+    res.update(main_res)
+    res.update({"n_gpus": ws, "steps": args.steps, "warmup": args.warmup, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None,
+                "dtype": "e4m3 indexer / bf16 MLA, fp32 accumulate" if isinstance(cfg, (W.DSAConfig, W.CSAConfig))
+                else "bf16, fp32 accumulate",
+                "data": "synthetic (seeded, shapes and value distributions of the workload)"})
+    if args.config == "long" and not args.no_l128k:
+        # the metric's second length: the ragged workload (64 rows, histories
+        # 8K-128K in shuffled 64-token pages), measured the same way
+        torch.cuda.empty_cache()
+        gate, inp = measure(W.RAGGED, args, dev, local, rank, ws, sa, flush, "ragged")
+        del inp
+        gate.pop("metric", None)
+        res["l128k"] = gate
     if rank == 0:
         print(json.dumps(res), flush=True)
     if ws > 1:
@@ -884,6 +955,8 @@ def main(argv=None):
                    choices=sorted(list(W.DSA_CONFIGS) + list(W.BLOCK_CONFIGS) + list(W.NSA_CONFIGS) +
                                   list(W.CSA_CONFIGS) + ["crossover"]))
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-l128k", action="store_true",
+                   help="long decode only: skip the nested L=128K (ragged) measurement")
     args = p.parse_args(argv)
     if args.warmup < 3 and args.impl == "native":
         args.warmup = 3

@@ -66,6 +66,7 @@ def _load():
         lib.sa_oracle_block_sparse.argtypes = [I, I, I, I, I, I, D, P, P, P, P, P, P]
         lib.sa_oracle_block_attend.argtypes = [I, I, I, P, I, I, I, D, P, P, P, P]
         lib.sa_oracle_threads.restype = I
+        lib.sa_oracle_set_threads.argtypes = [I]
         _lib = lib
     return _lib
 
@@ -73,6 +74,11 @@ def _load():
 def threads() -> int:
     """Host threads the C oracle runs on (OpenMP)."""
     return int(_load().sa_oracle_threads())
+
+
+def set_threads(n: int) -> None:
+    """Limit the C oracle to n host threads (n >= 1)."""
+    _load().sa_oracle_set_threads(int(n))
 
 
 def _f64(a) -> np.ndarray:

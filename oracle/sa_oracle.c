@@ -253,3 +253,15 @@ int sa_oracle_threads(void)
     return 1;
 #endif
 }
+
+/* Set the number of host threads the loops above may use (n >= 1); used to
+ * time the oracle on one core beside all cores. */
+void sa_oracle_set_threads(int n)
+{
+#ifdef _OPENMP
+    extern void omp_set_num_threads(int);
+    omp_set_num_threads(n < 1 ? 1 : n);
+#else
+    (void)n;
+#endif
+}

@@ -25,11 +25,23 @@ def test_prefill_flops():
 
 
 def test_block_sparse_bytes():
-    """fp32 pooled keys of 2048 blocks for 8 x 32 (sequence, head) pairs; at
-    most 16 top blocks + the sink block + a 512-token window in the union."""
-    pooled, u_max = bench.block_bytes(W.BLOCK)
-    assert pooled == 8 * 32 * 2048 * 128 * 4 == 268_435_456
-    assert u_max == 16 * 64 + 64 + 512 == 1600
+    """fp32 pooled keys of 2048 blocks for 8 x 32 (sequence, head) pairs, plus
+    K and V (128 bf16 each) of every attended token, plus a bf16 query and an
+    fp32 output per pair."""
+    nbytes, u = bench.block_bytes(W.BLOCK, 256 * 1300)
+    assert u == 256 * 1300
+    assert nbytes == 8 * 32 * 2048 * 128 * 4 + 256 * 1300 * 512 + 256 * (256 + 512)
+
+
+def test_block_union_tokens_by_hand():
+    """L = 1000, block 64, sink 1 block, window 100 (tokens 900..999): chosen
+    blocks 0 (the sink itself), 3 (192..255) and 14 (896..959, overlapping the
+    window by 60 tokens) add 64 + 4 tokens to the 164 of sink and window; a
+    second head with no chosen block has only sink and window."""
+    cfg = W.BlockConfig(name="t", seed=0, B=1, L=1000, H=2, top_blocks=3, sink_blocks=1, window=100)
+    import numpy as np
+    sel = np.array([[[0, 3, 14], [-1, -1, -1]]])
+    assert bench.block_union_tokens(cfg, sel) == (164 + 64 + 4) + 164
 
 
 def test_nsa_decode_bytes():
