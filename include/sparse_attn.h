@@ -87,12 +87,28 @@ int sa_version(void);
  * Waits for `stream`, then reads and clears this GPU's device error word.
  * Kernels that wait on barriers give every wait a time limit; when one runs
  * out the kernel records a nonzero site code here, abandons its work
- * (outputs of that launch are then undefined) and returns.  *code_out gets
- * the code (0 = none).  Returns SA_ETIMEOUT if a code was set, SA_ECUDA if
- * the stream reported an error, else SA_OK.  This is the only call that
- * synchronises.
+ * (outputs of that launch are then undefined) and returns.  The sparse-MLA
+ * kernels also record code 0x700 when a selected position lies past the
+ * page table or maps to a page outside the pool (row 0 of the pool is read
+ * instead).  *code_out gets the code (0 = none; the first code recorded
+ * wins).  Returns SA_ETIMEOUT if a code was set, SA_ECUDA if the stream
+ * reported an error, else SA_OK.  This call and sa_set_wait_limit_ns are
+ * the only calls that synchronise.
  */
 sa_status sa_check_device_error(int* code_out, sa_stream_t stream);
+
+/*
+ * Sets, for the current GPU, the time limit of the kernels' waits on other
+ * parties (a ring slot filled by another warp, a partner CTA's signal), in
+ * nanoseconds; 0 restores the default of one second.  Waits of a CTA for its
+ * own copies and tensor-core work in flight before it exits always keep the
+ * one-second limit, so a kernel whose wait ran out still drains its own work
+ * and frees its tensor memory before it returns.  A short limit makes a
+ * kernel give up (and record its site code) instead of waiting: a way to
+ * exercise the failure path.  The setting applies to launches made after
+ * this call returns (it writes device memory synchronously).
+ */
+sa_status sa_set_wait_limit_ns(unsigned long long limit_ns);
 
 /*
  * Lightning indexer ([Notes] §9, index score I_{t,s}; [MLA-S] "DSA：先用便宜的

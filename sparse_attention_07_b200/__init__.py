@@ -30,7 +30,7 @@ EXPORTS = (
     "sa_block_mean_pool", "sa_block_sparse_attn", "sa_sparse_mla_decode_static",
     "sa_dense_mla_workspace_size", "sa_dense_mla_decode", "sa_mla_absorb_query", "sa_mla_up_project",
     "sa_nsa_compress", "sa_nsa_decode", "sa_csa_compress", "sa_csa_window_index",
-    "sa_index_scores_hist", "sa_topk_select_hist",
+    "sa_index_scores_hist", "sa_topk_select_hist", "sa_set_wait_limit_ns",
 )
 
 # Size of the library's static device array behind sparse_mla_decode_static
@@ -57,6 +57,7 @@ def lib():
         L.sa_status_string.argtypes = [I]
         L.sa_version.restype = I
         L.sa_check_device_error.argtypes = [ctypes.POINTER(I), P]
+        L.sa_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong]
         L.sa_index_scores.argtypes = [P, P, P, I64, I, P, I, P, P, I, I, I, I64, P, P]
         L.sa_topk_select.argtypes = [P, I64, P, I, I, P, P]
         L.sa_index_scores_hist.argtypes = [P, P, P, I64, I, P, I, P, P, I, I, I, I64, P, P, P]
@@ -115,6 +116,12 @@ def check_device_error() -> int:
     if st not in (SA_OK, SA_ETIMEOUT):
         raise SparseAttnError("sa_check_device_error", st)
     return code.value
+
+
+def set_wait_limit_ns(limit_ns: int) -> None:
+    """Time limit of the kernels' waits on other parties for the current GPU
+    (0: the default of one second).  Synchronous."""
+    _check("sa_set_wait_limit_ns", lib().sa_set_wait_limit_ns(int(limit_ns)))
 
 
 HIST_BINS = 4096

@@ -153,10 +153,15 @@ struct TcCfg {
     // fit on an SM (shared memory and tensor memory) and stream side by side
     static constexpr int kStages = R == 1 ? 5 : 6;
     // registers per thread: one-row groups with up to 64 heads stay within 128
-    // so that two CTAs fit (each CTA's warps are allocated in groups of four);
-    // otherwise whatever one CTA of kThreads can have
+    // so that two CTAs fit; otherwise whatever one CTA of kThreads can have.
+    // The register file is split over the SM's four sub-partitions (16K
+    // registers each) and a CTA's warps are spread over them, so the bound is
+    // set by the sub-partition holding ceil(warps / 4) warps (10 warps: 168,
+    // not 65536 / 320).
     static constexpr int kTwoPerSm = R == 1 && NH <= 64;
-    static constexpr int kMaxReg = kTwoPerSm ? 128 : ((65536 / kThreads) & ~7) > 255 ? 255 : ((65536 / kThreads) & ~7);
+    static constexpr int kWarpsPerSubpart = (kThreads / 32 + 3) / 4;
+    static constexpr int kRegCap = (16384 / (32 * kWarpsPerSubpart)) & ~7;
+    static constexpr int kMaxReg = kTwoPerSm ? 128 : (kRegCap > 255 ? 255 : kRegCap);
     // shared layout (offsets from a 1024-aligned base); the three group tables
     // (prefix, group start, group length) follow, (rows + 1) ints each, rounded
     static constexpr int kOffStages = 0;
@@ -326,7 +331,7 @@ __global__ void __launch_bounds__((TcCfg<NH, R, NEPI>::kThreads)) __maxnreg__((T
         // drain: every load still in flight lands before the CTA can exit
         if (lane == 0) {
             int dummy = 0;
-            WaitCtx dw{a.err, reinterpret_cast<volatile int*>(&dummy)};
+            WaitCtx dw(a.err, reinterpret_cast<volatile int*>(&dummy), kWaitLimitNs);  // drain: fixed limit
             for (int64_t i = n_issued - C::kStages; i < n_issued; ++i) {
                 if (i < 0) continue;
                 mbar_wait(&bar_full[i % C::kStages], static_cast<uint32_t>((i / C::kStages) & 1), dw, kErrIdxWait | 7);
@@ -374,7 +379,7 @@ __global__ void __launch_bounds__((TcCfg<NH, R, NEPI>::kThreads)) __maxnreg__((T
         }
         if (lane == 0) {  // all issued MMAs complete before TMEM is released
             int dummy = 0;
-            WaitCtx dw{a.err, reinterpret_cast<volatile int*>(&dummy)};
+            WaitCtx dw(a.err, reinterpret_cast<volatile int*>(&dummy), kWaitLimitNs);  // drain: fixed limit
             tc_commit(&bar_final);
             mbar_wait(&bar_final, 0, dw, kErrIdxWait | 8);
         }

@@ -12,7 +12,7 @@ namespace sa {
 namespace {
 
 constexpr int kMaxDevices = 64;
-__device__ int g_error_word;  // one per GPU that loads the library
+__device__ ErrBlock g_error_block;  // one per GPU that loads the library: error word + wait limit
 int* g_error_ptr[kMaxDevices] = {};
 int g_sm_count[kMaxDevices] = {};
 std::mutex g_mu;
@@ -36,8 +36,8 @@ int* device_error_word() {
     std::lock_guard<std::mutex> lk(g_mu);
     if (!g_error_ptr[d]) {
         void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_error_word) != cudaSuccess) return nullptr;
-        g_error_ptr[d] = static_cast<int*>(p);
+        if (cudaGetSymbolAddress(&p, g_error_block) != cudaSuccess) return nullptr;
+        g_error_ptr[d] = &static_cast<ErrBlock*>(p)->err;
     }
     return g_error_ptr[d];
 }
@@ -100,6 +100,13 @@ const char* sa_status_string(sa_status s) {
 }
 
 int sa_version(void) { return 100; }
+
+sa_status sa_set_wait_limit_ns(unsigned long long limit_ns) {
+    int* w = device_error_word();
+    if (!w) return SA_ECUDA;
+    void* lim = reinterpret_cast<char*>(w) + offsetof(ErrBlock, wait_limit_ns);
+    return cudaMemcpy(lim, &limit_ns, sizeof(limit_ns), cudaMemcpyHostToDevice) == cudaSuccess ? SA_OK : SA_ECUDA;
+}
 
 sa_status sa_check_device_error(int* code_out, sa_stream_t stream) {
     if (!code_out) return SA_EINVAL;

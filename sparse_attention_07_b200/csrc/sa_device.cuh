@@ -1,5 +1,5 @@
 // sa_device.cuh — inline-PTX building blocks for the sm_100a kernels:
-// mbarriers with time-bounded waits, TMA (tiled and gather4) loads, tcgen05
+// mbarriers with time-bounded waits, TMA tiled loads and bulk copies, tcgen05
 // (TMEM allocation, UMMA descriptors, MMA issue, TMEM loads/stores) and
 // cluster / distributed-shared-memory access.
 //
@@ -12,6 +12,7 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
+#include <stddef.h>
 #include <stdint.h>
 
 namespace sa {
@@ -25,10 +26,29 @@ enum : int {
     kErrTopkRow = 0x300,   // top-k: invalid row state
     kErrMixedGroup = 0x400,  // indexer: internal grouping inconsistency
     kErrGemmWait = 0x500,    // per-head projection GEMM waits
-    kErrNsaWait = 0x600      // NSA decode waits (low byte = ring slot)
+    kErrNsaWait = 0x600,     // NSA decode waits (low byte = ring slot)
+    kErrMlaIndex = 0x700     // sparse MLA: a position past the page table or a page outside the pool
 };
 
 constexpr unsigned long long kWaitLimitNs = 1000ull * 1000ull * 1000ull;  // 1 s
+
+// The device error word and, 8 bytes after it, the time limit of waits on
+// other parties (0: kWaitLimitNs), which the host may change
+// (sa_set_wait_limit_ns).  Waits for this CTA's own copies and tensor-core
+// work in flight (drains before exit) always use kWaitLimitNs.
+struct ErrBlock {
+    int err;
+    int pad;
+    unsigned long long wait_limit_ns;
+};
+
+// The limit in nanoseconds as 32 bits (at most about 4.29 s).
+__device__ __forceinline__ uint32_t wait_limit_of(const int* err) {
+    if (!err) return static_cast<uint32_t>(kWaitLimitNs);
+    const unsigned long long v = *reinterpret_cast<const volatile unsigned long long*>(
+        reinterpret_cast<const char*>(err) + offsetof(ErrBlock, wait_limit_ns));
+    return v == 0 ? static_cast<uint32_t>(kWaitLimitNs) : (v > 0xFFFFFFFFull ? 0xFFFFFFFFu : static_cast<uint32_t>(v));
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -116,17 +136,6 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t* b, uint32_t parity) {
     return ok != 0;
 }
 
-__device__ __forceinline__ bool mbar_test_wait_acq_cluster(uint64_t* b, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tmbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(b)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
 // Arrive on an mbarrier of a CTA of the cluster without ordering this thread's
 // earlier memory accesses (for "I have finished reading" signals whose reads
 // have already returned their values).
@@ -134,10 +143,16 @@ __device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t cluster_add
     asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
-// Context for bounded waits: the device error word and the CTA's abort flag.
+// Context for bounded waits: the device error word, the CTA's abort flag and
+// the time limit (read once from the error block, or given: drains pass
+// kWaitLimitNs).
 struct WaitCtx {
     int* err;             // global error word (may be null)
     volatile int* abort;  // shared-memory abort flag of this CTA
+    uint32_t limit_ns;
+    __device__ WaitCtx(int* e, volatile int* ab) : err(e), abort(ab), limit_ns(wait_limit_of(e)) {}
+    __device__ WaitCtx(int* e, volatile int* ab, unsigned long long lim)
+        : err(e), abort(ab), limit_ns(static_cast<uint32_t>(lim)) {}
 };
 
 // Wait until the phase with the given parity has completed.  Returns false if
@@ -152,7 +167,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, const Wa
     for (;;) {
         if (poll()) return true;
         if (*w.abort) return false;
-        if (global_ns() - t0 > kWaitLimitNs) {
+        if (global_ns() - t0 > w.limit_ns) {
             record_error(w.err, site);
             *w.abort = 1;
             return false;
@@ -200,49 +215,10 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const void* map, uint64_t
         : "memory");
 }
 
-// Four rows (y0..y3) of a 2D tensor, each `box width` elements from column x,
-// land as four consecutive rows of the destination tile (swizzle applied).
-__device__ __forceinline__ void tma_gather4(void* dst, const void* map, uint64_t* bar, int x, int y0, int y1,
-                                            int y2, int y3) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes [%0], [%1, "
-        "{%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3)
-        : "memory");
-}
-
 // 16-byte global -> shared copy through L2 (cp.async.cg); src_bytes = 0
 // writes 16 zero bytes and reads nothing.
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
-}
-
-// L2 cache policies for data that a later kernel reads again (evict_last) or
-// that is read for the last time (evict_first).
-__device__ __forceinline__ uint64_t l2_evict_last() {
-    uint64_t p;
-    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
-    return p;
-}
-
-__device__ __forceinline__ uint64_t l2_evict_first() {
-    uint64_t p;
-    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
-    return p;
-}
-
-// cp_async16 with an L2 cache policy.
-__device__ __forceinline__ void cp_async16_hint(uint32_t dst, const void* src, uint32_t src_bytes, uint64_t pol) {
-    asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2, %3;" ::"r"(dst), "l"(src),
-                 "r"(src_bytes), "l"(pol)
-                 : "memory");
-}
-
-// 16-byte global store with an L2 cache policy.
-__device__ __forceinline__ void st_v4_hint(float4* p, uint32_t a, uint32_t b, uint32_t c, uint32_t d, uint64_t pol) {
-    asm volatile("st.global.L2::cache_hint.v4.b32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(p), "r"(a), "r"(b), "r"(c),
-                 "r"(d), "l"(pol)
-                 : "memory");
 }
 
 // Arrive on `bar` once every cp.async this thread issued so far has landed
@@ -252,11 +228,6 @@ __device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
 }
 
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
-
-// Bring the line holding `p` into L2 (no data returned to the SM).
-__device__ __forceinline__ void prefetch_l2(const void* p) {
-    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
-}
 
 // 2^x with the hardware approximation (ex2.approx.ftz: -inf -> +0, results
 // below 2^-126 flush to zero).
@@ -431,61 +402,6 @@ __device__ __forceinline__ void st_cluster_v4(uint32_t addr, uint32_t a, uint32_
                  : "memory");
 }
 
-// Asynchronous 16-byte store into the shared memory of a CTA of the cluster;
-// on arrival it completes 16 bytes of transaction count on `cluster_mbar`, an
-// mbarrier of the same CTA.  No fence is needed: the receiver waits on its
-// barrier.
-__device__ __forceinline__ void st_async_v4(uint32_t cluster_addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d,
-                                            uint32_t cluster_mbar) {
-    asm volatile(
-        "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
-            cluster_addr),
-        "r"(a), "r"(b), "r"(c), "r"(d), "r"(cluster_mbar)
-        : "memory");
-}
-
-// Bulk copy of `bytes` (multiple of 16) from this CTA's shared memory into the
-// shared memory of a CTA of the cluster; completes `bytes` of transaction count
-// on `cluster_mbar` (an mbarrier of the destination CTA).  Commits one group.
-__device__ __forceinline__ void bulk_copy_to_cluster(uint32_t cluster_dst, const void* src, uint32_t bytes,
-                                                     uint32_t cluster_mbar) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n\t"
-        "cp.async.bulk.commit_group;" ::"r"(cluster_dst),
-        "r"(smem_u32(src)), "r"(bytes), "r"(cluster_mbar)
-        : "memory");
-}
-
-// Wait until every bulk copy this thread committed has finished reading its source.
-__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
-
-// Wait until at most N of the bulk copies this thread committed are still reading their source.
-template <int N>
-__device__ __forceinline__ void bulk_wait_read() {
-    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
-}
-
-// Bulk copy of `bytes` (multiple of 16, both addresses 16-byte aligned) from
-// global memory into this CTA's shared memory; completes `bytes` of transaction
-// count on `bar` (an mbarrier of this CTA, armed with expect_tx by the caller).
-__device__ __forceinline__ void bulk_copy_g2s(void* sdst, const void* gsrc, uint32_t bytes, uint64_t* bar) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-            smem_u32(sdst)),
-        "l"(gsrc), "r"(bytes), "r"(smem_u32(bar))
-        : "memory");
-}
-
-// bulk_copy_g2s with an L2 cache policy.
-__device__ __forceinline__ void bulk_copy_g2s_hint(void* sdst, const void* gsrc, uint32_t bytes, uint64_t* bar,
-                                                   uint64_t pol) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::
-            "r"(smem_u32(sdst)),
-        "l"(gsrc), "r"(bytes), "r"(smem_u32(bar)), "l"(pol)
-        : "memory");
-}
-
 // Bulk copy of `bytes` (multiple of 16, both addresses 16-byte aligned) from
 // this CTA's shared memory to global memory.  Commits one group.
 __device__ __forceinline__ void bulk_copy_s2g(void* gdst, const void* ssrc, uint32_t bytes) {
@@ -526,11 +442,6 @@ __device__ __forceinline__ uint32_t ld_cluster_u32(uint32_t addr) {
 // Named barrier over `nthreads` threads (multiple of 32), id 1..15.
 __device__ __forceinline__ void named_sync(uint32_t id, uint32_t nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-
-__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
-    __half2 v = __floats2half2_rn(lo, hi);
-    return *reinterpret_cast<uint32_t*>(&v);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

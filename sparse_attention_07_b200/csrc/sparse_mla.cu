@@ -82,11 +82,14 @@ struct MlaKernelArgs {
     float* ws_ml;  // [rows][nsplit][H][4] partial (m, l of bf16 P, l of fp32 P, unused)
 };
 
+// Pool row of position p of sequence `seq`, or -2 when p lies past the page
+// table or its page is outside the pool (the caller's preconditions are
+// broken: the caller records that and reads row 0 of the pool instead).
 __device__ __forceinline__ int64_t pool_row(const MlaArgs& a, int seq, int p) {
-    if (p / kPage >= a.pages_per_seq) return 0;  // position past the table: precondition broken
+    if (p / kPage >= a.pages_per_seq) return -2;
     const int pg = a.page_table ? a.page_table[static_cast<int64_t>(seq) * a.pages_per_seq + p / kPage]
                                 : seq * a.pages_per_seq + p / kPage;
-    if (pg < 0 || pg >= a.pool_pages) return 0;  // precondition broken: read a row inside the pool
+    if (pg < 0 || pg >= a.pool_pages) return -2;
     return static_cast<int64_t>(pg) * kPage + (p % kPage);
 }
 
@@ -176,7 +179,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1) mla_ker
         mbar_init(&bar_sfull, 1);
         mbar_init(&bar_sfree, 4);  // the exchange warps read S
         for (int i = 0; i < kMlaXBuf; ++i) {
-            mbar_init(&bar_lfull[i], 1);          // exchange thread 0, after its fence
+            mbar_init(&bar_lfull[i], 1);          // exchange thread 0
             mbar_init(&bar_lfree[i], kSmxWarps);  // this CTA's softmax warps
             mbar_init(&bar_xfull[i], 1);          // the partner's exchange thread 0
             mbar_init(&bar_xfree[i], kSmxWarps);  // the partner's softmax warps
@@ -238,6 +241,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1) mla_ker
         // pool rows of every slot of this CTA's tiles (-1: padded slot), four
         // selection reads in flight per thread
         const int n = nt * kNK, nthr = kThreads - 128;
+        bool broken = false;
         for (int i0 = tid - 128; i0 < n; i0 += 4 * nthr) {
             int pos[4];
 #pragma unroll
@@ -248,9 +252,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1) mla_ker
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
                 const int i = i0 + u * nthr;
-                if (i < n) sRows[i] = pos[u] >= 0 ? static_cast<int>(pool_row(a, seq, pos[u])) : -1;
+                if (i < n) {
+                    int row = pos[u] >= 0 ? static_cast<int>(pool_row(a, seq, pos[u])) : -1;
+                    if (row == -2) {
+                        broken = true;
+                        row = 0;
+                    }
+                    sRows[i] = row;
+                }
             }
         }
+        if (broken) record_error(a.err, kErrMlaIndex);
     }
     tc_fence_before();
     cluster_sync_all();  // query, row table and slot are in place, and the partner has started
@@ -353,7 +365,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1) mla_ker
                     t_last = global_ns();
                 } else {
                     if (*wc.abort) break;
-                    if (global_ns() - t_last > kWaitLimitNs) {
+                    if (global_ns() - t_last > wc.limit_ns) {
                         record_error(a.err, kErrMlaWait | 4);
                         s_abort = 1;
                         break;
@@ -361,7 +373,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1) mla_ker
                 }
             }
             int dummy = 0;
-            WaitCtx dw{a.err, reinterpret_cast<volatile int*>(&dummy)};
+            WaitCtx dw(a.err, reinterpret_cast<volatile int*>(&dummy), kWaitLimitNs);  // drain: fixed limit
             tc_commit(&bar_final);
             mbar_wait(&bar_final, 0, dw, kErrMlaWait | 11);
         }
@@ -405,7 +417,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1) mla_ker
             for (int c = 0; c < 16; ++c) st_cg_v4(dst + c * 128 + h, v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
             named_sync(2, 128);
             if (h == 0) {
-                __threadfence();  // the partial scores are in L2 before either softmax is told
+                // release arrivals (this CTA's softmax at CTA scope, the partner's at
+                // cluster scope): the stores of all 128 exchange threads precede them
+                // through the named barrier, and each softmax acquires its arrival
                 mbar_arrive(&bar_lfull[xb]);
                 mbar_arrive_cluster(xfull_remote + 8 * xb);
             }
@@ -446,7 +460,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1) mla_ker
             __syncwarp();
             if (lane == 0) {
                 mbar_arrive(&bar_lfree[xb]);
-                mbar_arrive_cluster(xfree_remote + 8 * xb);  // the partner may refill its buffer
+                mbar_arrive_cluster_relaxed(xfree_remote + 8 * xb);  // the partner may refill its buffer
             }
 #pragma unroll
             for (int j = 0; j < kNK; ++j) {
