@@ -270,15 +270,20 @@ sa_status sa_mla_up_project(const float* o_lat, const void* U_V, int rows, int H
  *    stream capture begins.
  *  - Shapes whose partial states need more than SA_STATIC_SCRATCH_BYTES
  *    (sa_sparse_mla_workspace_size(rows, H, k, d_c) > SA_STATIC_SCRATCH_BYTES)
- *    return SA_EUNSUPPORTED and launch nothing; use sa_sparse_mla_decode with
- *    a caller workspace for those.
+ *    return SA_EUNSUPPORTED and launch nothing (no allocation and no launch
+ *    happens before this check; the size depends on the device's SM count,
+ *    which sets the key splits); use sa_sparse_mla_decode with a caller
+ *    workspace for those.  The array holds the exchange area of every SM
+ *    slot and the split-key states of up to 80 (row, split) pairs of 128
+ *    heads, i.e. every call with k <= 4096 on a GPU of up to 160 SMs (the
+ *    library's limit; the B200 has 148).
  *  - All calls share the one array.  Calls that may overlap on the GPU (on
  *    different streams, or on different host threads without ordering)
  *    race on it and give undefined outputs; order them on one stream.  Every
  *    byte a call reads from the array was written earlier in the same call,
  *    so nothing left by a previous call leaks into a result.
  */
-#define SA_STATIC_SCRATCH_BYTES ((size_t)40 << 20)
+#define SA_STATIC_SCRATCH_BYTES (((size_t)40 << 20) + ((size_t)256 << 10))
 
 sa_status sa_sparse_mla_decode_static(const void* q_lat, const void* q_rope,
                                       const void* c_cache, int64_t c_ld, const void* kr_cache, int64_t kr_ld,

@@ -35,7 +35,7 @@ EXPORTS = (
 
 # Size of the library's static device array behind sparse_mla_decode_static
 # (SA_STATIC_SCRATCH_BYTES in include/sparse_attn.h).
-STATIC_SCRATCH_BYTES = 40 << 20
+STATIC_SCRATCH_BYTES = (40 << 20) + (256 << 10)
 
 
 class SparseAttnError(RuntimeError):

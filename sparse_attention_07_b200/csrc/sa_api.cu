@@ -308,6 +308,14 @@ namespace {
 // Split-key partial states of sa_sparse_mla_decode_static live here; every
 // GPU that loads the library holds this array until the process exits.
 static __device__ __align__(256) unsigned char g_static_scratch[SA_STATIC_SCRATCH_BYTES];
+// The exchange area of every slot plus the split-key states (outputs, then
+// (m, l) words, each rounded to 256 bytes) of kMlaScratchSlots / 2 (row,
+// split) pairs of 128 heads: every decode with k <= 4096 on up to
+// kMlaScratchSlots SMs (splits are chosen so that rows * splits <= SMs / 2).
+static_assert(SA_STATIC_SCRATCH_BYTES >= static_cast<size_t>(kMlaScratchSlots) * kMlaXBuf * kMlaXBytes +
+                                             static_cast<size_t>(kMlaScratchSlots / 2) * 128 * 512 * 4 +
+                                             ((static_cast<size_t>(kMlaScratchSlots / 2) * 128 * 16 + 255) & ~size_t(255)),
+              "the static array covers k <= 4096 on every supported GPU");
 void* g_static_scratch_ptr[kMaxDevices] = {};
 
 // Device address of the array on the current device.  The array's name in
@@ -342,7 +350,7 @@ sa_status sa_sparse_mla_decode_static(const void* q_lat, const void* q_rope, con
     if (s != SA_OK) return s;
     const int ns = mla_decode_splits(rows, k);
     const size_t need = mla_workspace_bytes(rows, H, k, d_c, ns);
-    if (need > SA_STATIC_SCRATCH_BYTES) return SA_EUNSUPPORTED;  // checked before any CUDA call
+    if (need > SA_STATIC_SCRATCH_BYTES) return SA_EUNSUPPORTED;  // no allocation or launch before this check
     void* ws = static_scratch();
     if (ws == nullptr) return SA_ECUDA;
     return sparse_mla_launch(a, ns, ws, SA_STATIC_SCRATCH_BYTES, reinterpret_cast<cudaStream_t>(stream));

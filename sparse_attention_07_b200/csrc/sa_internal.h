@@ -86,7 +86,7 @@ struct MlaArgs {
 constexpr int kMlaXBuf = 4;
 constexpr int kMlaXBytes = 128 * 64 * 4;
 constexpr int kMlaScratchSlots = 160;
-constexpr int kMaxTilesPerCta = 64;  // 64-key tiles per CTA (the supported size: prefill k <= 4096, decode splits)
+constexpr int kMaxTilesPerCta = 64;  // 64-key tiles per CTA (the row table in shared memory)
 
 size_t mla_exchange_bytes();
 size_t mla_workspace_bytes(int rows, int H, int k, int d_c, int nsplit);

@@ -201,3 +201,14 @@ def test_csa_validation(L):
 
 def test_check_device_error_rejects_null(L):
     assert L.sa_check_device_error(None, None) == sa.SA_EINVAL
+
+
+def test_static_scratch_size_matches_the_header():
+    """The binding's copy of SA_STATIC_SCRATCH_BYTES (used for its host-side
+    check) equals the header's definition."""
+    import re
+    hdr = open(os.path.join(ROOT, "include", "sparse_attn.h")).read()
+    m = re.search(r"#define SA_STATIC_SCRATCH_BYTES \((.*)\)\n", hdr)
+    assert m, "definition not found"
+    expr = m.group(1).replace("(size_t)", "")
+    assert eval(expr, {}) == sa.STATIC_SCRATCH_BYTES
