@@ -551,14 +551,28 @@ def cpu_baseline(inp, cfg, budget_s: float = 12.0):
     return {"value": unit_n / dt, "cores": threads, "kind": "oracle", "sample": sample, "seconds": round(dt, 3)}
 
 
-def workload(name: str):
+def workload(name: str, profile_rows: int = 0):
+    """The named workload; with profile_rows > 0, only its first query rows
+    (decode: sequences; prefill: chunk tokens; block/NSA/CSA: sequences), a
+    smaller case of the same kernels for profiler captures."""
+    from dataclasses import replace
     if name in W.DSA_CONFIGS:
-        return W.DSA_CONFIGS[name]
+        cfg = W.DSA_CONFIGS[name]
+        if profile_rows > 0:
+            n = min(profile_rows, cfg.rows)
+            if cfg.prefill_start >= 0:
+                cfg = replace(cfg, name=f"{cfg.name} (first {n} queries)", rows=n)
+            else:
+                cfg = replace(cfg, name=f"{cfg.name} (first {n} sequences)", n_seqs=n, rows=n, lens=cfg.lens[:n])
+        return cfg
     if name in W.NSA_CONFIGS:
-        return W.NSA_CONFIGS[name]
+        cfg = W.NSA_CONFIGS[name]
+        return replace(cfg, B=min(profile_rows, cfg.B)) if profile_rows > 0 else cfg
     if name in W.CSA_CONFIGS:
-        return W.CSA_CONFIGS[name]
-    return W.BLOCK_CONFIGS[name]
+        cfg = W.CSA_CONFIGS[name]
+        return replace(cfg, n_seqs=min(profile_rows, cfg.n_seqs)) if profile_rows > 0 else cfg
+    cfg = W.BLOCK_CONFIGS[name]
+    return replace(cfg, B=min(profile_rows, cfg.B)) if profile_rows > 0 else cfg
 
 
 def describe(cfg, flush_note):
@@ -776,7 +790,7 @@ def run_native(args):
     import sparse_attention_07_b200 as sa
     sa.lib()
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
-    cfg = workload(args.config)
+    cfg = workload(args.config, args.profile_rows)
     main_res, inp = measure(cfg, args, dev, local, rank, ws, sa, flush, args.config)
     del inp
     res = {"impl": "native"}
@@ -786,7 +800,7 @@ def run_native(args):
                 "dtype": "e4m3 indexer / bf16 MLA, fp32 accumulate" if isinstance(cfg, (W.DSAConfig, W.CSAConfig))
                 else "bf16, fp32 accumulate",
                 "data": "synthetic (seeded, shapes and value distributions of the workload)"})
-    if args.config == "long" and not args.no_l128k:
+    if args.config == "long" and not args.no_l128k and args.profile_rows == 0:
         # the metric's second length: the ragged workload (64 rows, histories
         # 8K-128K in shuffled 64-token pages), measured the same way
         torch.cuda.empty_cache()
@@ -957,6 +971,8 @@ def main(argv=None):
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-l128k", action="store_true",
                    help="long decode only: skip the nested L=128K (ragged) measurement")
+    p.add_argument("--profile-rows", type=int, default=0,
+                   help="profiler captures: run only the first N query rows / sequences of the workload")
     args = p.parse_args(argv)
     if args.warmup < 3 and args.impl == "native":
         args.warmup = 3
