@@ -40,7 +40,11 @@ L2_FLUSH_BYTES = 256 << 20  # > 126 MB L2
 # kernel of a workload, from one ncu capture, with the sha256 prefix of the
 # kernel source it was taken on (the figure is reported only while they match).
 TRAFFIC = {
-    "long": {"kernel": "sparse_mla.cu", "stage": "attn", "bytes_per_launch": 83550720, "src_sha": "8f5c50233ab005df"},
+    # mla_kernel only (the split combine's traffic is not in the figure)
+    "long": {"kernel": "sparse_mla.cu", "stage": "attn", "bytes_per_launch": 83498752, "src_sha": "e3cf022e6dc9925d"},
+    # captured on the first 16 sequences, scaled by the key bytes to the full launch (x 3.955)
+    "ragged": {"kernel": "index_scores.cu", "stage": "indexer", "bytes_per_launch": 595079675,
+               "src_sha": "a5cd3903e39303e6"},
     "nsa": {"kernel": "nsa.cu", "bytes_per_launch": 59232768, "src_sha": "46cccc0328e4c5e2"},
 }
 
