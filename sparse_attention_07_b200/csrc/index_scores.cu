@@ -231,6 +231,8 @@ __global__ void __launch_bounds__((TcCfg<NH, R, NEPI>::kThreads)) __maxnreg__((T
     if (R == 1 || a.seq_of_row == nullptr) {
         G = rows;
         for (int g = tid; g <= rows; g += blockDim.x) s_gstart[g] = g;
+        // the group lengths below read entries other warps wrote (g + 1)
+        __syncthreads();
     } else {
         int* flag = tmp + kMaxRows;
         for (int r = tid; r < rows; r += blockDim.x)
