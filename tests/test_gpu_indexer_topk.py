@@ -144,6 +144,52 @@ def test_topk_edge_rows():
     _topk_case(4, [32768] * 4, 2048, 25, lo=-100000, hi=100000, ld=32768)
 
 
+def _topk_check(s, n, k):
+    """Float scores [rows, ld] on the GPU: the selection counting the scores
+    itself and started from the host-counted first-digit histogram, both
+    against the oracle bit for bit."""
+    rows = s.shape[0]
+    nv = torch.tensor(n, dtype=torch.int32, device=DEV)
+    s_np = s.cpu().numpy()
+    want = oracle.topk(s_np.astype(np.float64), np.array(n), k)
+    assert np.array_equal(sa.topk_select(s, nv, k).cpu().numpy(), want)
+    counts = np.stack([np.bincount(_order_key_np(s_np[i, : n[i]]) >> 20, minlength=sa.HIST_BINS)
+                       for i in range(rows)]).astype(np.int32)
+    hist = sa.topk_histogram(rows, DEV)
+    hist.copy_(torch.from_numpy(counts))
+    assert np.array_equal(sa.topk_select(s, nv, k, hist=hist).cpu().numpy(), want)
+    assert int(hist.abs().sum()) == 0
+    assert sa.check_device_error() == 0
+
+
+def test_topk_first_digit_settles_the_row():
+    """Exactly k keys lie in the bins above the rest (value 7 against 1 and 2):
+    the first digit alone fixes the selection, no refinement pass runs and the
+    positions come from the passes over the slice."""
+    g = torch.Generator(device=DEV)
+    g.manual_seed(31)
+    rows, ld, k = 3, 40000, 2048
+    s = torch.randint(1, 3, (rows, ld), generator=g, device=DEV).float()
+    n = [40000, 33333, 9001]
+    for r in range(rows):
+        top = torch.randperm(n[r], generator=g, device=DEV)[:k]
+        s[r, top] = 7.0
+    _topk_check(s, n, k)
+
+
+def test_topk_selected_list_overflow():
+    """Spread values with a large k: more than 4096 keys of a CTA's slice lie
+    above the boundary digit, so the selected-position list overflows and the
+    slice passes place the selection; a smaller k on the same rows takes the
+    list path (the two must agree with the oracle alike)."""
+    g = torch.Generator(device=DEV)
+    g.manual_seed(33)
+    s = torch.randn(2, 65536, generator=g, device=DEV) * 100.0
+    n = [65536, 60001]
+    _topk_check(s, n, 20000)
+    _topk_check(s, n, 3000)
+
+
 def _order_key_np(x):
     u = np.asarray(x, dtype=np.float32).view(np.uint32).copy()
     u[u == 0x80000000] = 0
