@@ -403,7 +403,7 @@ sa_status sa_block_sparse_attn(const void* q, const float* pooled, int64_t poole
         stride_b % 4 || stride_t % 4 || stride_h % 4)
         return SA_EINVAL;
     return block_sparse_launch(q, pooled, pooled_ld, K, V, stride_b, stride_t, stride_h, B, H, D, L, block,
-                               top_blocks, sink_blocks, window, scale, out, sel_blocks,
+                               top_blocks, sink_blocks, window, scale, out, sel_blocks, device_error_word(),
                                reinterpret_cast<cudaStream_t>(stream));
 }
 

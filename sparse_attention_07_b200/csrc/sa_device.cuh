@@ -27,7 +27,8 @@ enum : int {
     kErrMixedGroup = 0x400,  // indexer: internal grouping inconsistency
     kErrGemmWait = 0x500,    // per-head projection GEMM waits
     kErrNsaWait = 0x600,     // NSA decode waits (low byte = ring slot)
-    kErrMlaIndex = 0x700     // sparse MLA: a position past the page table or a page outside the pool
+    kErrMlaIndex = 0x700,    // sparse MLA: a position past the page table or a page outside the pool
+    kErrBlockWait = 0x800    // block-sparse decode waits (low byte = site)
 };
 
 constexpr unsigned long long kWaitLimitNs = 1000ull * 1000ull * 1000ull;  // 1 s
@@ -212,6 +213,24 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const void* map, uint64_t
         "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, "
         "%5}], [%2];" ::"r"(smem_u32(dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_load_4d(void* dst, const void* map, uint64_t* bar, int x, int y, int z, int w) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, "
+        "%5, %6}], [%2];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z), "r"(w)
+        : "memory");
+}
+
+// Contiguous global -> shared bulk copy into this CTA's shared memory,
+// completing `bytes` transactions on `bar`.  Both addresses 16-byte aligned,
+// bytes a multiple of 16.
+__device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
         : "memory");
 }
 

@@ -103,7 +103,7 @@ sa_status block_mean_pool_launch(const void* K, int64_t sb, int64_t st_, int64_t
 sa_status block_sparse_launch(const void* q, const float* pooled, int64_t pooled_ld, const void* K, const void* V,
                               int64_t sb, int64_t st_, int64_t sh, int B, int H, int D, int L, int block,
                               int top_blocks, int sink_blocks, int window, float scale, float* out,
-                              int32_t* sel_blocks, cudaStream_t st);
+                              int32_t* sel_blocks, int* err, cudaStream_t st);
 
 // NSA three-branch decode (nsa.cu).
 constexpr int kNsaMaxSmem = 227 * 1024 - 4096;  // dynamic part; the kernel also has ~3 KB of static shared memory

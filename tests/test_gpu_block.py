@@ -75,3 +75,26 @@ def test_block_sparse_full_size_sampled():
     assert (np.diff(s, axis=-1) > 0).all() and (s >= 0).all() and (s < cfg.n_blocks).all()
     assert torch.isfinite(out).all()
     assert sa.check_device_error() == 0
+
+
+def test_block_sparse_unaligned_fallback():
+    """K and V as views 8 bytes past a 16-byte boundary: the tensor-map path
+    needs 16-byte alignment, so the per-thread-load kernel serves the call;
+    both paths agree with the oracle alike."""
+    cfg = W.BlockConfig(name="t", seed=0, B=2, L=1000, H=3, top_blocks=4, sink_blocks=1, window=100)
+    inp = W.block_inputs(cfg, DEV, seed=77)
+    shape = inp["K"].shape
+    kbuf = torch.empty(inp["K"].numel() + 4, dtype=inp["K"].dtype, device=DEV)
+    vbuf = torch.empty(inp["V"].numel() + 4, dtype=inp["V"].dtype, device=DEV)
+    K = kbuf[4:].view(shape)
+    V = vbuf[4:].view(shape)
+    K.copy_(inp["K"])
+    V.copy_(inp["V"])
+    assert K.data_ptr() % 16 == 8
+    pooled = sa.block_mean_pool(K, cfg.block)
+    sel = torch.empty(cfg.B, cfg.H, cfg.top_blocks, dtype=torch.int32, device=DEV)
+    out = sa.block_sparse_attn(inp["q"], pooled, K, V, cfg.block, cfg.top_blocks, cfg.sink_blocks, cfg.window,
+                               cfg.scale, sel_blocks=sel)
+    torch.cuda.synchronize()
+    _check_pairs(cfg, inp, out, sel, [(b, h) for b in range(cfg.B) for h in range(cfg.H)])
+    assert sa.check_device_error() == 0
