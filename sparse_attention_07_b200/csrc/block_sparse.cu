@@ -326,6 +326,10 @@ constexpr int kCSmem = kRingBytes + 1024;
 // inside the K/V ring (whose first tiles are issued once the selection is done)
 static_assert(kPoolRing + kMaxBlocks * 4 <= kRingBytes, "pooled ring and scores fit the K/V ring");
 static_assert(kMaxTop <= 64 && kPoolChunk % kW2 == 0 && kSegTok % kW2 == 0, "shapes");
+constexpr int kSelBits = 11;                  // block choice: histogram of the keys' top bits
+constexpr int kSelBins = 1 << kSelBits;
+constexpr int kSelCap = 256;                  // keys the choosing warp holds (8 per lane)
+static_assert(kSelBins * 4 + kSelCap * 8 <= kPoolRing && kSelBins % kT2 == 0, "selection scratch in the pooled ring");
 constexpr int kBlkW = kPoolChunk / kW2;       // pooled blocks per warp and chunk
 constexpr int kTokW = kSegTok / kW2;          // tokens per warp and segment
 
@@ -397,6 +401,7 @@ __global__ void __cluster_dims__(kC, 1, 1) __launch_bounds__(kT2, 2)
     __shared__ __align__(16) float s_wo[kW2][kD];
     __shared__ float s_state[kC][kD + 2];         // each CTA's (o, m, l), pushed to CTA 0
     __shared__ int s_abort;
+    __shared__ int s_wsel[kW2], s_bstar, s_nge, s_nc;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const uint32_t rank = cluster_rank();
@@ -464,12 +469,85 @@ __global__ void __cluster_dims__(kC, 1, 1) __launch_bounds__(kT2, 2)
         }
     }
 
-    // (2) this CTA's best ntop blocks: each warp over its share of the scores,
-    //     then warp 0 over the warps' lists
+    // The window and sink segments come first in the union's order and do not
+    // depend on the choice: with one CTA per pair (which takes the segments
+    // from the first one on) the first tile pair is loaded now, into the half of
+    // the ring that the choice below leaves alone.
+    const int win_lo = max(0, L - a.window);
+    const int sink_hi = min(win_lo, a.sink_blocks * blk);
+    const int n_sink = (sink_hi + kSegTok - 1) / kSegTok;
+    const int n_win = (L - win_lo + kSegTok - 1) / kSegTok;
+    const bool early = kC == 1 && n_win + n_sink > 0;
+    if (early && tid == 0) {
+        const int lo = n_win > 0 ? win_lo : 0;
+        fence_proxy_async_smem();
+        mbar_arrive_expect_tx(&bar_kv[1], 2u * kTileBytes);
+        tma_load_4d(ring + 1 * 2 * kTileBytes, &maps.K, &bar_kv[1], 0, lo, h, b);
+        tma_load_4d(ring + 1 * 2 * kTileBytes + kTileBytes, &maps.V, &bar_kv[1], 0, lo, h, b);
+        ++kv_issued;
+    }
+
+    // (2) this CTA's best ntop blocks.  A histogram of the scores' keys
+    //     (top 11 bits) in the consumed pooled ring finds the bin of the
+    //     ntop-th largest; the keys at or above it (few, unless many scores
+    //     tie) are listed and one warp picks the best of them.  Lists too long
+    //     for the warp fall back to arg-max rounds in every warp over all keys.
+    const int nmine = bhi - blo;
+    const int want = min(ntop, nmine);
+    uint32_t* hsel = reinterpret_cast<uint32_t*>(ring);                 // [kSelBins]
+    uint64_t* cand = reinterpret_cast<uint64_t*>(ring + kSelBins * 4);  // [kSelCap]
+    for (int i = tid; i < kSelBins; i += kT2) hsel[i] = 0u;
+    if (tid == 0) {
+        s_bstar = kSelBins;  // no key qualifies unless a bin is found below
+        s_nge = 0;
+        s_nc = 0;
+    }
+    __syncthreads();
+    for (int i = tid; i < nmine; i += kT2) atomicAdd(&hsel[score_order_key(s_score[i]) >> (32 - kSelBits)], 1u);
+    __syncthreads();
     {
+        constexpr int kBinsPer = kSelBins / kT2;       // thread t: bins from the top, highest first
+        const int top_bin = kSelBins - 1 - kBinsPer * tid;
+        int c[kBinsPer], tot = 0;
+#pragma unroll
+        for (int j = 0; j < kBinsPer; ++j) {
+            c[j] = static_cast<int>(hsel[top_bin - j]);
+            tot += c[j];
+        }
+        int incl = tot;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int t = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += t;
+        }
+        if (lane == 31) s_wsel[warp] = incl;
+        __syncthreads();
+        int above = incl - tot;
+        for (int w = 0; w < warp; ++w) above += s_wsel[w];
+        if (want > 0 && above < want && want <= above + tot) {
+            int acc = above;
+#pragma unroll
+            for (int j = 0; j < kBinsPer; ++j) {
+                acc += c[j];
+                if (acc >= want) {
+                    s_bstar = top_bin - j;
+                    s_nge = acc;
+                    break;
+                }
+            }
+        }
+    }
+    __syncthreads();
+    const bool fast = s_nge <= kSelCap;
+    if (fast) {
+        const uint32_t bstar = static_cast<uint32_t>(s_bstar);
+        for (int i = tid; i < nmine; i += kT2) {
+            const uint32_t kk = score_order_key(s_score[i]);
+            if ((kk >> (32 - kSelBits)) >= bstar) cand[atomicAdd(&s_nc, 1)] = block_key2(s_score[i], blo + i);
+        }
+    } else {
         constexpr int kPerLane = kMaxPer / kT2;  // scores per lane (4 or 16)
         uint64_t v[kPerLane];
-        const int nmine = bhi - blo;
 #pragma unroll
         for (int j = 0; j < kPerLane; ++j) {
             const int i = (warp * kPerLane + j) * 32 + lane;  // warp w: its 32 * kPerLane scores
@@ -479,15 +557,27 @@ __global__ void __cluster_dims__(kC, 1, 1) __launch_bounds__(kT2, 2)
     }
     __syncthreads();
     if (warp == 0) {
-        constexpr int kM = kW2 * kMaxTop / 32;  // 16 per lane
-        uint64_t v[kM];
-#pragma unroll
-        for (int j = 0; j < kM; ++j) {
-            const int i = j * 32 + lane, w = i / kMaxTop, t = i % kMaxTop;
-            v[j] = t < ntop ? s_wtop[w][t] : 0ull;
-        }
         uint64_t* mine = &s_wtop[0][0];  // reused: warp 0 only from here, after the barrier
-        warp_top<kM>(v, ntop, mine, lane);
+        if (fast) {
+            constexpr int kCP = kSelCap / 32;
+            const int nc = s_nc;
+            uint64_t v[kCP];
+#pragma unroll
+            for (int j = 0; j < kCP; ++j) {
+                const int i = j * 32 + lane;
+                v[j] = i < nc ? cand[i] : 0ull;
+            }
+            warp_top<kCP>(v, ntop, mine, lane);
+        } else {
+            constexpr int kM = kW2 * kMaxTop / 32;  // 16 per lane
+            uint64_t v[kM];
+#pragma unroll
+            for (int j = 0; j < kM; ++j) {
+                const int i = j * 32 + lane, w = i / kMaxTop, t = i % kMaxTop;
+                v[j] = t < ntop ? s_wtop[w][t] : 0ull;
+            }
+            warp_top<kM>(v, ntop, mine, lane);
+        }
         __syncwarp();
         cluster_wait();  // every CTA of the cluster has started
         for (int i = lane; i < kC * ntop; i += 32) {
@@ -538,35 +628,35 @@ __global__ void __cluster_dims__(kC, 1, 1) __launch_bounds__(kT2, 2)
     }
     __syncthreads();
 
-    // (3) the union as 64-token segments; this CTA's share of them
-    const int win_lo = max(0, L - a.window);
-    const int sink_hi = min(win_lo, a.sink_blocks * blk);
-    const int n_sink = (sink_hi + kSegTok - 1) / kSegTok, n_ch = s_ncseg;
-    const int n_win = (L - win_lo + kSegTok - 1) / kSegTok;
+    // (3) the union as 64-token segments (window, sink, chosen blocks); this
+    //     CTA's share of them.  Segment i of the share uses ring stage
+    //     (i + 1) % kKvStages (stage 1 is the one free during the choice).
+    const int n_ch = s_ncseg;
     const int nseg = n_sink + n_ch + n_win;
     const int g0 = static_cast<int>(static_cast<int64_t>(rank) * nseg / kC);
     const int g1 = static_cast<int>(static_cast<int64_t>(rank + 1) * nseg / kC);
     auto seg_of = [&](int g, int& lo, int& hi) {
-        if (g < n_sink) {
-            lo = g * kSegTok;
-            hi = min(lo + kSegTok, sink_hi);
-        } else if (g < n_sink + n_ch) {
-            lo = s_cseg[g - n_sink] * blk;
-            hi = min(lo + blk, win_lo);
-        } else {
-            lo = win_lo + (g - n_sink - n_ch) * kSegTok;
+        if (g < n_win) {
+            lo = win_lo + g * kSegTok;
             hi = min(lo + kSegTok, L);
+        } else if (g < n_win + n_sink) {
+            lo = (g - n_win) * kSegTok;
+            hi = min(lo + kSegTok, sink_hi);
+        } else {
+            lo = s_cseg[g - n_win - n_sink] * blk;
+            hi = min(lo + blk, win_lo);
         }
     };
     const int nmy = g1 - g0;
-    if (tid == 0) {  // the pooled ring is consumed (barrier above): first K/V tiles
+    if (tid == 0) {  // the choice is done (barrier above): the first K/V tiles
         fence_proxy_async_smem();
-        for (int i = 0; i < kKvStages && i < nmy; ++i) {
+        for (int i = early ? 1 : 0; i < kKvStages && i < nmy; ++i) {
+            const int st = (i + 1) % kKvStages;
             int lo, hi;
             seg_of(g0 + i, lo, hi);
-            mbar_arrive_expect_tx(&bar_kv[i], 2u * kTileBytes);
-            tma_load_4d(ring + i * 2 * kTileBytes, &maps.K, &bar_kv[i], 0, lo, h, b);
-            tma_load_4d(ring + i * 2 * kTileBytes + kTileBytes, &maps.V, &bar_kv[i], 0, lo, h, b);
+            mbar_arrive_expect_tx(&bar_kv[st], 2u * kTileBytes);
+            tma_load_4d(ring + st * 2 * kTileBytes, &maps.K, &bar_kv[st], 0, lo, h, b);
+            tma_load_4d(ring + st * 2 * kTileBytes + kTileBytes, &maps.V, &bar_kv[st], 0, lo, h, b);
             ++kv_issued;
         }
     }
@@ -575,7 +665,7 @@ __global__ void __cluster_dims__(kC, 1, 1) __launch_bounds__(kT2, 2)
     float m = -INFINITY, l = 0.f;
     float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int i = 0; i < nmy; ++i) {
-        const int st = i % kKvStages;
+        const int st = (i + 1) % kKvStages;
         int lo, hi;
         seg_of(g0 + i, lo, hi);
         const bool got = mbar_wait(&bar_kv[st], static_cast<uint32_t>((i / kKvStages) & 1), wc, kErrBlockWait | 2);
@@ -636,7 +726,7 @@ __global__ void __cluster_dims__(kC, 1, 1) __launch_bounds__(kT2, 2)
         for (int c = max(0, pool_issued - kPoolStages); c < pool_issued; ++c)
             mbar_wait(&bar_pool[c % kPoolStages], static_cast<uint32_t>((c / kPoolStages) & 1), dw, kErrBlockWait | 3);
         for (int i = max(0, kv_issued - kKvStages); i < kv_issued; ++i)
-            mbar_wait(&bar_kv[i % kKvStages], static_cast<uint32_t>((i / kKvStages) & 1), dw, kErrBlockWait | 4);
+            mbar_wait(&bar_kv[(i + 1) % kKvStages], static_cast<uint32_t>((i / kKvStages) & 1), dw, kErrBlockWait | 4);
     }
 
     // (5) the warps' states, then the CTAs' states (in CTA 0)

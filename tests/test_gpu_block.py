@@ -98,3 +98,29 @@ def test_block_sparse_unaligned_fallback():
     torch.cuda.synchronize()
     _check_pairs(cfg, inp, out, sel, [(b, h) for b in range(cfg.B) for h in range(cfg.H)])
     assert sa.check_device_error() == 0
+
+
+@pytest.mark.parametrize("B,H", [(1, 2), (2, 80)])
+def test_block_sparse_all_scores_tied(B, H):
+    """A zero query scores every block 0: the choice is the lowest top_blocks
+    blocks (ties go to the lower block), taken by the fallback rounds since
+    the tied keys outnumber what the choosing warp holds; the output is the
+    uniform average over the union.  (1, 2) runs clusters of four CTAs per
+    pair, (2, 80) one CTA per pair."""
+    cfg = W.BlockConfig(name="t", seed=0, B=B, L=64 * 700, H=H, top_blocks=16, sink_blocks=1, window=512)
+    inp = W.block_inputs(cfg, DEV, seed=5)
+    q = torch.zeros_like(inp["q"])
+    pooled = sa.block_mean_pool(inp["K"], cfg.block)
+    sel = torch.empty(cfg.B, cfg.H, cfg.top_blocks, dtype=torch.int32, device=DEV)
+    out = sa.block_sparse_attn(q, pooled, inp["K"], inp["V"], cfg.block, cfg.top_blocks, cfg.sink_blocks,
+                               cfg.window, cfg.scale, sel_blocks=sel)
+    torch.cuda.synchronize()
+    assert (sel.cpu().numpy() == np.arange(cfg.top_blocks)).all()
+    for b, h in [(0, 0), (B - 1, H - 1)]:
+        K = inp["K"][b, :, h].double().cpu().numpy()
+        V = inp["V"][b, :, h].double().cpu().numpy()
+        ref_out, ref_sel, _ = oracle.block_sparse(np.zeros(128), K, V, cfg.block, cfg.top_blocks, cfg.sink_blocks,
+                                                  cfg.window, cfg.scale)
+        assert (ref_sel == np.arange(cfg.top_blocks)).all()
+        assert_attention_close(out[b, h].cpu().numpy(), ref_out, f"tied ({b},{h})")
+    assert sa.check_device_error() == 0
