@@ -43,8 +43,10 @@ TRAFFIC = {
     # mla_kernel only (the split combine's traffic is not in the figure)
     "long": {"kernel": "sparse_mla.cu", "stage": "attn", "bytes_per_launch": 83498752, "src_sha": "e3cf022e6dc9925d"},
     # captured on the first 16 sequences, scaled by the key bytes to the full launch (x 3.955)
-    "ragged": {"kernel": "index_scores.cu", "stage": "indexer", "bytes_per_launch": 595079675,
-               "src_sha": "a5cd3903e39303e6"},
+    "ragged": {"kernel": "index_scores.cu", "stage": "indexer", "bytes_per_launch": 595101949,
+               "src_sha": "510c9df4d95be2b1"},
+    # block_sparse_cluster_kernel<1> on the full block workload (one pass: no scaling)
+    "block": {"kernel": "block_sparse.cu", "bytes_per_launch": 483272448, "src_sha": "e02282be07fa6780"},
     "nsa": {"kernel": "nsa.cu", "bytes_per_launch": 59232768, "src_sha": "46cccc0328e4c5e2"},
 }
 
@@ -704,7 +706,7 @@ def measure(cfg, args, dev, local, rank, ws, sa, flush, config_key):
                 v["us"] = round(v["us"], 2)
             dom_name = max(kern, key=lambda n: kern[n]["us"])
             dom = kern[dom_name]
-            tr = TRAFFIC.get(config_key, {})
+            tr = TRAFFIC.get(config_key, {}) if not args.profile_rows else {}  # records are of the full workloads
             traffic = None
             if tr.get("bytes_per_launch") and tr.get("stage") == dom_name and tr.get("src_sha") == src_sha(
                     "sparse_attention_07_b200/csrc/" + tr.get("kernel", "")):
@@ -747,7 +749,7 @@ def measure(cfg, args, dev, local, rank, ws, sa, flush, config_key):
         metric = "NSA decode queries/s (compression + group block choice + selection + window, gated)"
         nbytes = nsa_bytes(cfg)
         ach = nbytes / (first * 1e-3) / 1e9
-        tr = TRAFFIC.get(config_key, {})
+        tr = TRAFFIC.get(config_key, {}) if not args.profile_rows else {}  # records are of the full workloads
         traffic = tr.get("bytes_per_launch") if tr.get("src_sha") == src_sha(
             "sparse_attention_07_b200/csrc/" + tr.get("kernel", "nsa.cu")) else None
         roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": hbm, "unit": "GB/s", "frac": round(ach / hbm, 4),
@@ -759,8 +761,11 @@ def measure(cfg, args, dev, local, rank, ws, sa, flush, config_key):
         metric = "block-sparse decode queries/s (pooled-block scan+top-k+block attention)"
         nbytes, u_tokens = block_bytes(cfg, step.union_tokens)
         ach = nbytes / (first * 1e-3) / 1e9
+        tr = TRAFFIC.get(config_key, {}) if not args.profile_rows else {}  # records are of the full workloads
+        traffic = tr.get("bytes_per_launch") if tr and tr.get("src_sha") == src_sha(
+            "sparse_attention_07_b200/csrc/" + tr.get("kernel", "block_sparse.cu")) else None
         roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": hbm, "unit": "GB/s", "frac": round(ach / hbm, 4),
-                "traffic": None, "kernel": "block_sparse_kernel", "bytes_per_launch": nbytes,
+                "traffic": traffic, "kernel": "block_sparse_cluster_kernel", "bytes_per_launch": nbytes,
                 "union_tokens": u_tokens, "peak_source": f"{peak_src} hbm_gbs"}
     value = units / (ms * 1e-3)
     res.update({
