@@ -47,7 +47,7 @@ TRAFFIC = {
                "src_sha": "510c9df4d95be2b1"},
     # block_sparse_cluster_kernel<1> on the full block workload (one pass: no scaling)
     "block": {"kernel": "block_sparse.cu", "bytes_per_launch": 483272448, "src_sha": "e02282be07fa6780"},
-    "nsa": {"kernel": "nsa.cu", "bytes_per_launch": 59232768, "src_sha": "46cccc0328e4c5e2"},
+    "nsa": {"kernel": "nsa.cu", "bytes_per_launch": 59074304, "src_sha": "bd2295e266d64125"},
 }
 
 

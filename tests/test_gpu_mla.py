@@ -143,3 +143,32 @@ def test_sparse_mla_split_merge_repeatable():
     assert_attention_close(out0.cpu().numpy(), ref_out, "split merge")
     assert_lse_close(lse0.cpu().numpy(), ref_lse, "lse")
     assert sa.check_device_error() == 0
+
+
+def test_sparse_mla_bad_position_is_reported():
+    """A selected position past the sequence's page table, then a page-table
+    entry outside the pool: the kernel reads pool row 0 for those slots
+    (never an address outside the pool), records code 0x700 in the device
+    error word, and the rows without a bad slot keep their exact result."""
+    cfg, inp, idx = _case(2, 128, 64, 500, seed=9)
+    ref_out, _ = _oracle(cfg, inp, idx)
+    bad = idx.clone()
+    bad[0, 3] = cfg.pages_per_seq * 64 + 5
+    out, _ = _run(sa.sparse_mla_decode, cfg, inp, bad)
+    assert sa.check_device_error() == 0x700
+    assert np.isfinite(out).all()
+    assert_attention_close(out[1:], ref_out[1:], "row beside the bad slot")
+    pool_pages = inp["c_cache"].shape[0] // 64
+    good = idx.clone()
+    good[1, 0] = 0  # a slot on page 0 of row 1
+    saved = inp["page_table"].clone()
+    inp["page_table"][1, 0] = pool_pages + 3
+    try:
+        out, _ = _run(sa.sparse_mla_decode, cfg, inp, good)
+        assert sa.check_device_error() == 0x700
+        assert np.isfinite(out).all()
+    finally:
+        inp["page_table"].copy_(saved)
+    out, _ = _run(sa.sparse_mla_decode, cfg, inp, idx)
+    assert sa.check_device_error() == 0
+    assert_attention_close(out, ref_out, "after the reports")
