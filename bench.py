@@ -34,6 +34,7 @@ if ROOT not in sys.path:
 import workloads as W  # noqa: E402
 
 DECODE_METRIC = "sparse-MLA decode queries/s (indexer+topk+attn) at L=32K/128K; % HBM roofline"
+L2_BYTES = 126 * 10**6  # B200 L2
 L2_FLUSH_BYTES = 256 << 20  # > 126 MB L2
 
 # dram__bytes_read.sum + dram__bytes_write.sum per launch of the roofline
@@ -72,6 +73,20 @@ def prefill_flops(cfg: W.DSAConfig):
     idx = float((nv * 2 * cfg.H_I * cfg.d_I).sum())
     mla = float((np.minimum(nv, cfg.topk) * cfg.H * 2 * (cfg.d_c + cfg.d_R + cfg.d_c)).sum())
     return idx, mla
+
+
+def step_working_set(cfg, step) -> int:
+    """Distinct bytes one step reads (its working set for L2 purposes)."""
+    if isinstance(cfg, W.DSAConfig):
+        if cfg.prefill_start >= 0:  # every query row of the chunk reads the same history
+            esize = 1 if cfg.idx_dtype == "e4m3" else 4
+            return int(cfg.n_seqs * cfg.L_max * (cfg.d_I * esize + (cfg.d_c + cfg.d_R) * 2))
+        return int(sum(decode_bytes(cfg)))
+    if isinstance(cfg, W.CSAConfig):
+        return int(sum(csa_bytes(cfg)))
+    if isinstance(cfg, W.NSAConfig):
+        return int(nsa_bytes(cfg))
+    return int(block_bytes(cfg, step.union_tokens)[0])
 
 
 def block_union_tokens(cfg: W.BlockConfig, sel: np.ndarray) -> int:
@@ -462,9 +477,20 @@ def time_projections(step, K: int, flush, hbm: float):
     return res
 
 
-def e2e_steps(step, K: int, flush):
-    """Same step through the public API with the step's query inputs copied in
-    from pinned host memory and the output read back, inside the events."""
+E2E_SLOTS = 3  # steps in flight in the end-to-end pipeline
+
+
+def e2e_steps(step, K: int, flush, flush_each: bool):
+    """The step through the public API as a serving loop runs it: every step's
+    query inputs are copied in from pinned host memory and its output is read
+    back to pinned host memory, on their own streams, so that the copies of
+    neighbouring steps overlap the compute.  Per step, on the compute stream:
+    the inputs move from the step's slot into the step's input tensors (a
+    device copy), L2 is flushed when the step's working set would fit in it
+    (`flush_each`), the step runs, and its output moves to the slot (a device
+    copy) for the read-back.  A slot is reused only after its read-back
+    finished.  One pair of events brackets all K steps (all copies, flushes
+    and device copies inside); returns [per-step ms] * K."""
     inp = step.inp
     if isinstance(step, DecodeStep):
         names = ["q_idx", "w", "q_lat", "q_rope"]
@@ -475,22 +501,55 @@ def e2e_steps(step, K: int, flush):
     else:
         names = ["q"]
     result = step.out
+    # two slots when a step's output is large (the prefill chunk's is 1 GB)
+    S = E2E_SLOTS if result.numel() * result.element_size() <= (256 << 20) else 2
     host_in = {n: inp[n].cpu().pin_memory() for n in names}
-    host_out = torch.empty(result.shape, dtype=result.dtype).pin_memory()
+    host_out = [torch.empty(result.shape, dtype=result.dtype).pin_memory() for _ in range(S)]
+    dev_in = [{n: torch.empty_like(inp[n]) for n in names} for _ in range(S)]
+    dev_out = [torch.empty_like(result) for _ in range(S)]
     h2d = sum(t.numel() * t.element_size() for t in host_in.values())
-    d2h = host_out.numel() * host_out.element_size()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
-    for e0, e1 in ev:
-        flush.zero_()
-        e0.record()
-        for n, t in host_in.items():
-            inp[n].copy_(t, non_blocking=True)
-        step.indexer()
-        step.rest()
-        host_out.copy_(result, non_blocking=True)
-        e1.record()
+    d2h = host_out[0].numel() * host_out[0].element_size()
+    s_in, s_comp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    in_done = [torch.cuda.Event() for _ in range(K)]
+    comp_done = [torch.cuda.Event() for _ in range(K)]
+    out_done = [torch.cuda.Event() for _ in range(K)]
+    cur = torch.cuda.current_stream()
+    for st in (s_in, s_comp, s_out):
+        st.wait_stream(cur)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(cur)
+    for st in (s_in, s_comp, s_out):
+        st.wait_event(e0)
+    for i in range(K):
+        slot = i % S
+        with torch.cuda.stream(s_in):
+            if i >= S:
+                s_in.wait_event(comp_done[i - S])  # the slot's inputs were taken
+            for n, t in host_in.items():
+                dev_in[slot][n].copy_(t, non_blocking=True)
+            in_done[i].record(s_in)
+        with torch.cuda.stream(s_comp):
+            s_comp.wait_event(in_done[i])
+            if i >= S:
+                s_comp.wait_event(out_done[i - S])  # the slot's output was read back
+            for n in names:
+                inp[n].copy_(dev_in[slot][n], non_blocking=True)
+            if flush_each:
+                flush.zero_()
+            step.indexer()
+            step.rest()
+            dev_out[slot].copy_(result, non_blocking=True)
+            comp_done[i].record(s_comp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(comp_done[i])
+            host_out[slot].copy_(dev_out[slot], non_blocking=True)
+            out_done[i].record(s_out)
+    for st in (s_in, s_comp, s_out):
+        cur.wait_stream(st)
+    e1.record(cur)
     torch.cuda.synchronize()
-    return [a.elapsed_time(b) for a, b in ev], h2d, d2h
+    per = e0.elapsed_time(e1) / K
+    return [per] * K, h2d, d2h
 
 
 def cpu_baseline(inp, cfg, budget_s: float = 12.0):
@@ -648,7 +707,10 @@ def measure(cfg, args, dev, local, rank, ws, sa, flush, config_key):
     if ws > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
-    e2e_ms, h2d, d2h = e2e_steps(step, args.steps, flush)
+    # L2 flushed inside the end-to-end loop only where a step's working set is
+    # under twice the L2 size (larger ones evict their own data)
+    flush_each = step_working_set(cfg, step) < 2 * L2_BYTES
+    e2e_ms, h2d, d2h = e2e_steps(step, args.steps, flush, flush_each)
     err = sa.check_device_error()
     if err != 0:
         raise RuntimeError(f"device error word 0x{err:x}")
@@ -777,7 +839,13 @@ def measure(cfg, args, dev, local, rank, ws, sa, flush, config_key):
                                "step and stage times: stream-launched steps with an event between stages")),
         "roofline": roof,
         "e2e": {"value": round(units / (e2e * 1e-3), 1), "unit": unit, "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h},
+                "d2h_bytes_per_step": d2h,
+                "timing": (f"{args.steps} steps in one event pair, up to {E2E_SLOTS} in flight: copy-in, compute "
+                           "and copy-out streams; per step the inputs are copied in from pinned host memory, "
+                           "moved to the step's tensors, "
+                           + ("L2 is flushed (working set under twice the L2), " if flush_each else
+                              "no flush (working set over twice the L2), ")
+                           + "the step runs and its output is read back to pinned host memory")},
         "gpu_launches": step.launches_per_step * args.steps,
         "clocks": clk.summary(),
     })
