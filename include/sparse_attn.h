@@ -315,6 +315,11 @@ sa_status sa_block_mean_pool(const void* K, int64_t stride_b, int64_t stride_t, 
  *   q [B][H][D] bf16; K, V as in sa_block_mean_pool; out [B][H][D] fp32;
  *   sel_blocks [B][H][top_blocks] int32 (ascending, -1 padded) or NULL.
  * Supported: D = 128, block = 64, 1 <= top_blocks <= 64, L/block <= 4096.
+ * K and V need 8-byte alignment and strides that are multiples of 4
+ * elements; with 16-byte alignment and strides that are multiples of 8
+ * elements the chosen K/V blocks are loaded as tensor-map tiles (faster),
+ * otherwise with per-thread loads (same results).  Waits record codes
+ * 0x801-0x804 in the device error word when they run out.
  */
 sa_status sa_block_sparse_attn(const void* q, const float* pooled, int64_t pooled_ld,
                                const void* K, const void* V, int64_t stride_b, int64_t stride_t,
@@ -325,8 +330,9 @@ sa_status sa_block_sparse_attn(const void* q, const float* pooled, int64_t poole
 /*
  * NSA compressed cache ([Ch11] §12.6 mean compression; [MLA-S] NSA: only
  * complete blocks are summarised):
- *   Kc[b][h][n][d] = bf16( (sum_{i<block} K[b][n*block+i][h][d]) * (1/block) )
- * with the sum taken in fp32 in token order and rounded to the nearest bf16;
+ *   Kc[b][h][n][d] = bf16( (sum_{i<block} K[b][n*block+i][h][d]) / block )
+ * with the sum taken in fp64 (exact for bf16 blocks of moderate dynamic
+ * range) and the mean rounded once to the nearest bf16, ties to even;
  * Vc likewise from V; for every complete block n < L / block.  Run when a
  * block completes (the decode reads the cache).
  *   K, V bf16, element (b,t,h,d) at b*stride_b + t*stride_t + h*stride_h + d

@@ -14,8 +14,8 @@
 // mixed by independent gates: out = g_c o_c + g_s o_s + g_w o_w.
 //
 // nsa_compress: one warp per (sequence, KV head, block, K|V) sums the block's
-// rows in fp32 in token order and stores mean rounded to bf16 (the compressed
-// cache, built when a block completes).
+// rows in fp64 and stores the mean rounded once to bf16 (the compressed cache,
+// built when a block completes).
 //
 // nsa_decode: a cluster of kC CTAs per (sequence, KV head).  Every CTA streams
 // its share of the data through one ring of 32-row items (one TMA box each,
