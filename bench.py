@@ -48,7 +48,7 @@ TRAFFIC = {
                "src_sha": "510c9df4d95be2b1"},
     # block_sparse_cluster_kernel<1> on the full block workload (one pass: no scaling)
     "block": {"kernel": "block_sparse.cu", "bytes_per_launch": 483272448, "src_sha": "e02282be07fa6780"},
-    "nsa": {"kernel": "nsa.cu", "bytes_per_launch": 59074304, "src_sha": "bd2295e266d64125"},
+    "nsa": {"kernel": "nsa.cu", "bytes_per_launch": 59074304, "src_sha": "e49c849dfa2ed8a1"},
 }
 
 
