@@ -37,7 +37,8 @@ def _check_pairs(cfg, inp, out, sel, pairs):
 
 
 @pytest.mark.parametrize("L,top,sink,win", [(1000, 4, 1, 100), (4096, 16, 1, 512), (700, 64, 2, 0),
-                                            (130, 16, 1, 512), (64 * 33, 16, 0, 64)])
+                                            (130, 16, 1, 512), (64 * 33, 16, 0, 64),
+                                            (50, 4, 1, 100), (64 * 5 + 7, 64, 8, 10), (64 * 9, 3, 0, 1000)])
 def test_block_sparse_small(L, top, sink, win):
     cfg = W.BlockConfig(name="t", seed=0, B=2, L=L, H=3, top_blocks=top, sink_blocks=sink, window=win)
     inp = W.block_inputs(cfg, DEV, seed=L + top)
