@@ -257,19 +257,19 @@ def test_decode_step_repeats_bit_identical():
     hist = sa.topk_histogram(cfg.rows, DEV)
     scores = torch.empty(cfg.rows, cfg.L_max, dtype=torch.float32, device=DEV)
     first = None
-    for rnd in range(24):
+    for rep in range(24):
         sa.index_scores(inp["q_idx"], inp["w"], inp["k_idx_cache"], nv, cfg.pages_per_seq,
                         page_table=inp["page_table"], seq_of_row=inp["seq_of_row"], scores=scores,
-                        hist=hist if rnd % 2 else None)
-        idx = sa.topk_select(scores, nv, cfg.topk, hist=hist if rnd % 2 else None)
+                        hist=hist if rep % 2 else None)
+        idx = sa.topk_select(scores, nv, cfg.topk, hist=hist if rep % 2 else None)
         sa.sparse_mla_decode(inp["q_lat"], inp["q_rope"], inp["c_cache"], inp["kr_cache"], idx, cfg.scale,
                              cfg.pages_per_seq, page_table=inp["page_table"], seq_of_row=inp["seq_of_row"])
         got = (torch.where(visible, scores, torch.zeros_like(scores)), idx.clone())
         if first is None:
             first = got
         else:
-            assert torch.equal(got[0], first[0]), f"round {rnd}: index scores differ from round 0"
-            assert torch.equal(got[1], first[1]), f"round {rnd}: Top-K sets differ from round 0"
+            assert torch.equal(got[0], first[0]), f"repeat {rep}: index scores differ from the first"
+            assert torch.equal(got[1], first[1]), f"repeat {rep}: Top-K sets differ from the first"
     assert int(hist.abs().sum()) == 0
     assert sa.check_device_error() == 0
     _check_scores(inp, first[0], rows=[0, 31, 63])
