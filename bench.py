@@ -229,16 +229,26 @@ def peaks():
 class DecodeStep:
     """Buffers and launches of one indexer -> Top-K -> sparse-MLA step."""
 
-    def __init__(self, inp, sa):
+    def __init__(self, inp, sa, topk_path: str = "scores"):
         self.sa, self.inp, self.cfg = sa, inp, inp["cfg"]
         cfg, dev = self.cfg, inp["q_idx"].device
-        self.scores = torch.empty(cfg.rows, cfg.L_max, dtype=torch.float32, device=dev)
         self.idx = torch.empty(cfg.rows, cfg.topk, dtype=torch.int32, device=dev)
         self.out = torch.empty(cfg.rows, cfg.H, cfg.d_c, dtype=torch.float32, device=dev)
         self.lse = torch.empty(cfg.rows, cfg.H, dtype=torch.float32, device=dev)
-        # the indexer counts each row's first Top-K digit; the Top-K starts from it and clears it
-        self.hist = sa.topk_histogram(cfg.rows, dev)
         self.prefill = cfg.prefill_start >= 0
+        # decode with one query row per sequence on the tensor-core indexer:
+        # the indexer keeps only the keys that can still be in the Top-K
+        # (candidates) and the Top-K selects from them; otherwise the indexer
+        # writes every score and counts each row's first Top-K digit, and the
+        # Top-K starts from those counts.  Both leave their counts cleared.
+        self.cand_path = (topk_path == "cand" and not self.prefill and inp["seq_of_row"] is None
+                          and cfg.idx_dtype == "e4m3" and cfg.d_I == 128 and cfg.H_I in (16, 32, 64, 128))
+        if self.cand_path:
+            self.scores = None
+            self.cand, self.cand_cnt, self.hist = sa.candidate_buffers(cfg.rows, cfg.pages_per_seq * 64, dev)
+        else:
+            self.scores = torch.empty(cfg.rows, cfg.L_max, dtype=torch.float32, device=dev)
+            self.hist = sa.topk_histogram(cfg.rows, dev)
         size = sa.sparse_mla_prefill_workspace_size if self.prefill else sa.sparse_mla_workspace_size
         self.ws = torch.empty(size(cfg.rows, cfg.H, cfg.topk, cfg.d_c), dtype=torch.uint8, device=dev)
         # decode splits keys (and adds the combine launch) when its workspace holds partial states
@@ -248,16 +258,35 @@ class DecodeStep:
 
     def indexer(self):
         i, c = self.inp, self.cfg
-        self.sa.index_scores(i["q_idx"], i["w"], i["k_idx_cache"], i["n_visible"], c.pages_per_seq,
-                             page_table=i["page_table"], seq_of_row=i["seq_of_row"], scores=self.scores,
-                             hist=self.hist)
+        if self.cand_path:
+            self.sa.index_candidates(i["q_idx"], i["w"], i["k_idx_cache"], i["n_visible"], c.pages_per_seq, c.topk,
+                                     self.cand, self.cand_cnt, self.hist, page_table=i["page_table"])
+        else:
+            self.sa.index_scores(i["q_idx"], i["w"], i["k_idx_cache"], i["n_visible"], c.pages_per_seq,
+                                 page_table=i["page_table"], seq_of_row=i["seq_of_row"], scores=self.scores,
+                                 hist=self.hist)
 
     def rest(self):
         self.topk()
         self.attn()
 
     def topk(self):
-        self.sa.topk_select(self.scores, self.inp["n_visible"], self.cfg.topk, idx_out=self.idx, hist=self.hist)
+        if self.cand_path:
+            self.sa.topk_from_candidates(self.cand, self.cand_cnt, self.inp["n_visible"], self.cfg.topk, self.hist,
+                                         idx_out=self.idx)
+        else:
+            self.sa.topk_select(self.scores, self.inp["n_visible"], self.cfg.topk, idx_out=self.idx,
+                                hist=self.hist)
+
+    def kept_candidates(self) -> int:
+        """Candidates the indexer keeps over all rows in one step (0 on the
+        score path); runs one indexer launch and one Top-K launch."""
+        if not self.cand_path:
+            return 0
+        self.indexer()
+        kept = int(self.cand_cnt.sum())
+        self.topk()
+        return kept
 
     def attn(self):
         i, c = self.inp, self.cfg
@@ -664,11 +693,11 @@ def describe(cfg, flush_note):
             "batch": cfg.B, "seq_len": cfg.L, "heads": cfg.H, "l2": flush_note}
 
 
-def make_step(cfg, dev, rank, sa):
+def make_step(cfg, dev, rank, sa, topk_path: str = "scores"):
     """Seeded inputs of a workload (each rank its own seed) and its step."""
     if isinstance(cfg, W.DSAConfig):
         inp = W.dsa_inputs(cfg, dev, seed=rank_seed(cfg.seed, rank))
-        return inp, DecodeStep(inp, sa)
+        return inp, DecodeStep(inp, sa, topk_path)
     if isinstance(cfg, W.NSAConfig):
         inp = W.nsa_inputs(cfg, dev, seed=rank_seed(cfg.seed, rank))
         return inp, NsaStep(inp, sa)
@@ -683,7 +712,7 @@ def measure(cfg, args, dev, local, rank, ws, sa, flush, config_key):
     """Warm-up, then the timed steps (graph replays), the per-stage steps and
     the end-to-end steps of one workload; returns the result fields of its
     JSON line (without the top-level run keys) and the inputs."""
-    inp, step = make_step(cfg, dev, rank, sa)
+    inp, step = make_step(cfg, dev, rank, sa, args.topk_path)
     for _ in range(args.warmup):
         flush.zero_()
         step.indexer()
@@ -691,6 +720,7 @@ def measure(cfg, args, dev, local, rank, ws, sa, flush, config_key):
     torch.cuda.synchronize()
     if sa.check_device_error() != 0:
         raise RuntimeError("device error word set during warm-up")
+    kept = step.kept_candidates() if isinstance(step, DecodeStep) else 0
 
     if ws > 1:
         torch.distributed.barrier()
@@ -756,12 +786,22 @@ def measure(cfg, args, dev, local, rank, ws, sa, flush, config_key):
                     "frac": dom["tensor_frac"], "traffic": None, "kernel": dom["kernel"],
                     "peak_source": dom["peak_source"]}
         else:
-            kern = {
-                "indexer": {"kernel": "idx_tc_kernel" if cfg.idx_dtype == "e4m3" else "idx_cc_kernel",
-                            "us": t_idx * 1e3, "bytes": keys_b},
-                "topk": {"kernel": "topk_kernel", "us": t_topk * 1e3, "bytes": score_b},
-                "attn": {"kernel": "mla_kernel (+ mla_combine_kernel)", "us": t_attn * 1e3, "bytes": rows_b},
-            }
+            if step.cand_path:
+                # the indexer keeps candidates instead of writing every score;
+                # the Top-K reads the first-digit counts and the candidates
+                kern = {
+                    "indexer": {"kernel": "idx_tc_kernel (candidates)", "us": t_idx * 1e3, "bytes": keys_b},
+                    "topk": {"kernel": "topk_cand_kernel", "us": t_topk * 1e3,
+                             "bytes": cfg.rows * 4096 * 4 + kept * 8, "candidates_per_step": kept},
+                    "attn": {"kernel": "mla_kernel (+ mla_combine_kernel)", "us": t_attn * 1e3, "bytes": rows_b},
+                }
+            else:
+                kern = {
+                    "indexer": {"kernel": "idx_tc_kernel" if cfg.idx_dtype == "e4m3" else "idx_cc_kernel",
+                                "us": t_idx * 1e3, "bytes": keys_b},
+                    "topk": {"kernel": "topk_kernel", "us": t_topk * 1e3, "bytes": score_b},
+                    "attn": {"kernel": "mla_kernel (+ mla_combine_kernel)", "us": t_attn * 1e3, "bytes": rows_b},
+                }
             for v in kern.values():
                 v["hbm_gbs"] = round(v["bytes"] / (v["us"] * 1e-6) / 1e9, 1)
                 v["hbm_frac"] = round(v["hbm_gbs"] / hbm, 4)
@@ -849,6 +889,9 @@ def measure(cfg, args, dev, local, rank, ws, sa, flush, config_key):
         "gpu_launches": step.launches_per_step * args.steps,
         "clocks": clk.summary(),
     })
+    if isinstance(step, DecodeStep):
+        res["config"]["indexer_output"] = ("Top-K candidates (keys at or above a proven bound on the row's k-th "
+                                           "largest)" if step.cand_path else "every score")
     if ws == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline(inp, cfg)
         res["cpu_baseline"]["unit"] = unit
@@ -1046,6 +1089,8 @@ def main(argv=None):
                    choices=sorted(list(W.DSA_CONFIGS) + list(W.BLOCK_CONFIGS) + list(W.NSA_CONFIGS) +
                                   list(W.CSA_CONFIGS) + ["crossover"]))
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--topk-path", choices=["cand", "scores"], default="scores",
+                   help="decode: the indexer keeps Top-K candidates (cand) or writes every score (scores)")
     p.add_argument("--no-l128k", action="store_true",
                    help="long decode only: skip the nested L=128K (ragged) measurement")
     p.add_argument("--profile-rows", type=int, default=0,

@@ -10,6 +10,9 @@
  *   sa_index_scores_hist / sa_topk_select_hist
  *                        the same two steps, the indexer also counting each row's
  *                        first-digit histogram for the Top-K
+ *   sa_index_candidates / sa_topk_from_candidates
+ *                        the same two steps for decode, the indexer keeping only
+ *                        the keys that can still be in the Top-K
  *   sa_sparse_mla_decode / sa_sparse_mla_prefill
  *                        softmax over the selected set of the absorbed content score
  *                        plus the RoPE score, scaled; output sum_j a_j c_j in latent space
@@ -412,6 +415,41 @@ sa_status sa_csa_window_index(const int32_t* topk_idx, int rows, int k, const in
  */
 sa_status sa_topk_select_hist(const float* scores, int64_t scores_ld, const int32_t* n_valid, int rows, int k,
                               int32_t* hist, int32_t* idx_out, sa_stream_t stream);
+
+/*
+ * The indexer and the Top-K of one decode step without the dense score rows
+ * ([Notes] §9: only the k largest I_{t,s} of each row are used; [MLA-S]
+ * "一次错选会丢掉什么？" orders them by (-score, position)).
+ * sa_index_candidates computes the scores of sa_index_scores_hist (one query
+ * row per sequence; dtype SA_E4M3, d_I = 128, H_I in {16, 32, 64, 128}) and
+ * counts them in hist as that call does, but keeps only candidates: while a
+ * row streams, the counts so far give a digit d with at least k keys at or
+ * above it, and a key whose digit (order key >> 20) is below the latest such d
+ * is dropped (it cannot be among the k largest; the counts only grow, so a
+ * bound read early is lower, never wrong).  Every key of the final Top-K is
+ * kept; how many others are kept depends on timing, not on the result.
+ *   cand     [rows][cand_ld] uint64: entries 0 .. cand_cnt[r]-1 of row r are
+ *            (order key << 32) | (0xFFFFFFFF - position), in no fixed order
+ *   cand_cnt [rows] int32, zeros on entry; hist [rows][4096] int32, zeros on
+ *            entry, 16-byte aligned
+ *   cand_ld >= pages_per_seq * 64 (<= 262144); n_visible[r] <= pages_per_seq * 64
+ * sa_topk_from_candidates then writes idx_out [rows][k] exactly as
+ * sa_topk_select does for the same scores (ascending positions, -1 padding),
+ * with n_valid = the same n_visible, and leaves hist and cand_cnt zeroed, so
+ * one set of buffers serves every step.  A row whose counts do not add up to
+ * min(n_valid[r], cand_ld) records code 0x301 in the device error word (its
+ * output is then undefined).  Shapes outside the tensor-core indexer return
+ * SA_EUNSUPPORTED.  The order key is the score's bit pattern with the sign
+ * bit set for non-negative scores and every bit flipped for negative ones
+ * (-0.0 as +0.0), so that keys order as the scores do.
+ */
+sa_status sa_index_candidates(const void* q, const float* w, const void* k_cache, int64_t pool_pages, sa_dtype dtype,
+                              const int32_t* page_table, int pages_per_seq, const int32_t* n_visible, int rows,
+                              int H_I, int d_I, int k, int64_t cand_ld, uint64_t* cand, int32_t* cand_cnt,
+                              int32_t* hist, sa_stream_t stream);
+
+sa_status sa_topk_from_candidates(const uint64_t* cand, int64_t cand_ld, int32_t* cand_cnt, const int32_t* n_valid,
+                                  int rows, int k, int32_t* hist, int32_t* idx_out, sa_stream_t stream);
 
 #ifdef __cplusplus
 }

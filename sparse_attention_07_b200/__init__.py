@@ -31,6 +31,7 @@ EXPORTS = (
     "sa_dense_mla_workspace_size", "sa_dense_mla_decode", "sa_mla_absorb_query", "sa_mla_up_project",
     "sa_nsa_compress", "sa_nsa_decode", "sa_csa_compress", "sa_csa_window_index",
     "sa_index_scores_hist", "sa_topk_select_hist", "sa_set_wait_limit_ns",
+    "sa_index_candidates", "sa_topk_from_candidates",
 )
 
 # Size of the library's static device array behind sparse_mla_decode_static
@@ -62,6 +63,8 @@ def lib():
         L.sa_topk_select.argtypes = [P, I64, P, I, I, P, P]
         L.sa_index_scores_hist.argtypes = [P, P, P, I64, I, P, I, P, P, I, I, I, I64, P, P, P]
         L.sa_topk_select_hist.argtypes = [P, I64, P, I, I, P, P, P]
+        L.sa_index_candidates.argtypes = [P, P, P, I64, I, P, I, P, I, I, I, I, I64, P, P, P, P]
+        L.sa_topk_from_candidates.argtypes = [P, I64, P, P, I, I, P, P, P]
         L.sa_sparse_mla_workspace_size.restype = SZ
         L.sa_sparse_mla_workspace_size.argtypes = [I, I, I, I]
         L.sa_sparse_mla_decode.argtypes = [P, P, P, I64, P, I64, I64, P, I, P, P, I, I, I, I, I, F, P, P, P, SZ, P]
@@ -168,6 +171,42 @@ def topk_select(scores, n_valid, k: int, idx_out=None, hist=None):
         st = lib().sa_topk_select_hist(_p(scores), scores.stride(0), _p(n_valid), rows, k, _p(hist), _p(idx_out),
                                        _stream())
         _check("sa_topk_select_hist", st)
+    return idx_out
+
+
+def candidate_buffers(rows: int, cand_ld: int, device):
+    """(cand [rows, cand_ld] uint64 as int64, cand_cnt [rows] int32 zeroed,
+    hist [rows, 4096] int32 zeroed) for index_candidates / topk_from_candidates:
+    the Top-K leaves the counts zeroed, so one set serves every step."""
+    return (torch.empty(rows, cand_ld, dtype=torch.int64, device=device),
+            torch.zeros(rows, dtype=torch.int32, device=device),
+            torch.zeros(rows, HIST_BINS, dtype=torch.int32, device=device))
+
+
+def index_candidates(q_idx, w, k_idx_cache, n_visible, pages_per_seq: int, k: int, cand, cand_cnt, hist,
+                     page_table=None):
+    """Indexer scores of one query row per sequence, kept only where they can
+    still be among the row's k largest: cand[r, :cand_cnt[r]] holds
+    (order key << 32) | (0xFFFFFFFF - position) (read as int64), and hist
+    counts every score's first digit."""
+    rows, H_I, d_I = q_idx.shape
+    pool_pages = k_idx_cache.shape[0] // 64
+    st = lib().sa_index_candidates(_p(q_idx), _p(w), _p(k_idx_cache), pool_pages, _dtype_code(q_idx),
+                                   _p(page_table), pages_per_seq, _p(n_visible), rows, H_I, d_I, k,
+                                   cand.stride(0), _p(cand), _p(cand_cnt), _p(hist), _stream())
+    _check("sa_index_candidates", st)
+    return cand
+
+
+def topk_from_candidates(cand, cand_cnt, n_valid, k: int, hist, idx_out=None):
+    """Exact Top-K positions [rows, k] int32 (as topk_select) from the output of
+    index_candidates; clears hist and cand_cnt."""
+    rows = cand.shape[0]
+    if idx_out is None:
+        idx_out = torch.empty(rows, k, dtype=torch.int32, device=cand.device)
+    st = lib().sa_topk_from_candidates(_p(cand), cand.stride(0), _p(cand_cnt), _p(n_valid), rows, k, _p(hist),
+                                       _p(idx_out), _stream())
+    _check("sa_topk_from_candidates", st)
     return idx_out
 
 

@@ -141,14 +141,16 @@ struct ItemWalk {
     }
 };
 
-template <int NH, int R, int NEPI>
+template <int NH, int R, int NEPI, bool kCand = false>
 struct TcCfg {
     static constexpr int N = R * NH;                     // MMA N (rows x heads)
     // accumulator buffers: four where they fit in TMEM (the MMA runs further ahead of the epilogue)
     static constexpr int kAcc = (4 * N <= 512) ? 4 : 2;
     static constexpr int kTmemCols = (kAcc * N <= 32) ? 32 : (kAcc * N <= 64 ? 64 : (kAcc * N <= 128 ? 128 : (kAcc * N <= 256 ? 256 : 512)));
     static constexpr int kQBytes = N * 128;
-    static constexpr int kThreads = 32 * (NEPI + 2);
+    // warps: NEPI epilogue, TMA producer, MMA issuer; candidate mode adds the
+    // warp that keeps the row's candidate bound up to date
+    static constexpr int kThreads = 32 * (NEPI + 2 + (kCand ? 1 : 0));
     // key-tile ring: one-row groups (decode) keep five stages so that two CTAs
     // fit on an SM (shared memory and tensor memory) and stream side by side
     static constexpr int kStages = R == 1 ? 5 : 6;
@@ -172,11 +174,12 @@ struct TcCfg {
     static size_t smem_bytes(int rows) { return kOffTables + 3 * static_cast<size_t>(table_ints(rows)) * 4 + 1024; }
 };
 
-template <int NH, int R, int NEPI>
-__global__ void __launch_bounds__((TcCfg<NH, R, NEPI>::kThreads)) __maxnreg__((TcCfg<NH, R, NEPI>::kMaxReg))
+template <int NH, int R, int NEPI, bool kCand>
+__global__ void __launch_bounds__((TcCfg<NH, R, NEPI, kCand>::kThreads)) __maxnreg__((TcCfg<NH, R, NEPI, kCand>::kMaxReg))
     idx_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
                   const IdxArgs a) {
-    using C = TcCfg<NH, R, NEPI>;
+    using C = TcCfg<NH, R, NEPI, kCand>;
+    static_assert(!kCand || R == 1, "candidates are emitted by one-row groups");
     constexpr int N = C::N;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -194,12 +197,20 @@ __global__ void __launch_bounds__((TcCfg<NH, R, NEPI>::kThreads)) __maxnreg__((T
     __shared__ int s_abort;
     __shared__ int s_warpbuf[40];
     __shared__ int s_G;
+    // candidate mode: (row + 1) << 32 | bound digit, published by the bound warp;
+    // the epilogue's current row, its tiles done in that row, and "finished"
+    __shared__ volatile unsigned long long s_bound;
+    __shared__ volatile int s_epi_row, s_epi_tiles, s_epi_done;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     WaitCtx wc{a.err, &s_abort};
 
     if (tid == 0) {
         s_abort = 0;
+        s_bound = 0ull;
+        s_epi_row = -1;
+        s_epi_tiles = 0;
+        s_epi_done = 0;
         for (int i = 0; i < C::kStages; ++i) {
             mbar_init(&bar_full[i], 1);
             mbar_init(&bar_empty[i], 1);
@@ -386,6 +397,70 @@ __global__ void __launch_bounds__((TcCfg<NH, R, NEPI>::kThreads)) __maxnreg__((T
             mbar_wait(&bar_final, 0, dw, kErrIdxWait | 8);
         }
         __syncwarp();
+    } else if (kCand && warp == NEPI + 2) {
+        // ------------------------------------------------ candidate bound
+        // Every kBoundTiles tiles of the epilogue's current row, the warp reads
+        // the row's first-digit counts (every CTA's keys so far) from the top
+        // and publishes the digit d at which they reach k: at least k keys
+        // already seen lie at or above d, so no key below d is among the k
+        // largest (the counts only grow, so a stale bound is lower, never
+        // wrong).  Lane l sums bins 4095-128l down to 3968-128l.
+        constexpr int kBoundTiles = 8;
+        // The wait limit applies to the epilogue's progress (a row or tile
+        // count that stops changing), not to the kernel's whole run.
+        int last_row = -1, last_tiles = 0, seen_row = -1, seen_tiles = 0;
+        unsigned long long t0 = global_ns();
+        while (!s_epi_done) {
+            const int row = s_epi_row, tiles = s_epi_tiles;
+            if (row != seen_row || tiles != seen_tiles) {
+                seen_row = row;
+                seen_tiles = tiles;
+                t0 = global_ns();
+            }
+            if (row < 0 || (row == last_row && tiles - last_tiles < kBoundTiles)) {
+                if (global_ns() - t0 > wc.limit_ns) {
+                    record_error(a.err, kErrIdxWait | 9);
+                    break;
+                }
+                __nanosleep(256);
+                continue;
+            }
+            const int32_t* hr = a.hist + static_cast<int64_t>(row) * kHistBins;
+            const int4* src = reinterpret_cast<const int4*>(hr + kHistBins - 128 * (lane + 1));
+            int tot = 0;
+#pragma unroll 8
+            for (int j = 0; j < 32; ++j) {
+                const int4 v = __ldcg(src + j);
+                tot += v.x + v.y + v.z + v.w;
+            }
+            int incl = tot;  // keys in this lane's bins and the bins above them
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int t = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += t;
+            }
+            const int above = incl - tot;
+            unsigned found = 0u;
+            if (above < a.k && a.k <= incl) {
+                int run = above;
+                for (int j = 31; j >= 0 && !found; --j) {  // highest bins first
+                    const int4 v = __ldcg(src + j);
+                    const int c4[4] = {v.w, v.z, v.y, v.x};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        run += c4[e];
+                        if (!found && run >= a.k) found = static_cast<unsigned>(kHistBins - 128 * (lane + 1) + 4 * j + 3 - e) + 1u;
+                    }
+                }
+            }
+            found = __reduce_max_sync(0xffffffffu, found);
+            if (lane == 0 && found != 0u)
+                s_bound = (static_cast<unsigned long long>(row + 1) << 32) | (found - 1u);
+            __syncwarp();
+            last_row = row;
+            last_tiles = tiles;
+        }
+        __syncwarp();
     } else {
         // ------------------------------------------------ epilogue (warps 0..NEPI-1)
         const int quarter = warp & 3;
@@ -407,6 +482,10 @@ __global__ void __launch_bounds__((TcCfg<NH, R, NEPI>::kThreads)) __maxnreg__((T
                     if constexpr (R == 1) {
 #pragma unroll
                         for (int x = 0; x < NH; ++x) wr[x] = a.w[static_cast<int64_t>(g_r0) * NH + x];
+                    }
+                    if (kCand && warp == 0 && lane == 0) {
+                        s_epi_tiles = 0;
+                        s_epi_row = g_r0;
                     }
                     __syncwarp();
                     for (int i = lane; i < R * NH; i += 32) {
@@ -455,7 +534,26 @@ __global__ void __launch_bounds__((TcCfg<NH, R, NEPI>::kThreads)) __maxnreg__((T
                     }
                     const float sc = (acc4[0] + acc4[1]) + (acc4[2] + acc4[3]);
                     const bool live = s < nvis[0] && g_cnt > 0;
-                    if (live) a.scores[static_cast<int64_t>(g_r0) * a.scores_ld + s] = sc;
+                    if constexpr (kCand) {
+                        // keys at or above the row's bound, as (key << 32) | ~position
+                        const uint32_t key = score_order_key(sc);
+                        const unsigned long long bnd = s_bound;
+                        const uint32_t thr = static_cast<int>(bnd >> 32) == g_r0 + 1 ? static_cast<uint32_t>(bnd) : 0u;
+                        const bool emit = live && (key >> 20) >= thr;
+                        const unsigned bm = __ballot_sync(0xffffffffu, emit);
+                        if (bm != 0u) {
+                            int base = 0;
+                            if (lane == 0) base = atomicAdd(a.cand_cnt + g_r0, __popc(bm));
+                            base = __shfl_sync(0xffffffffu, base, 0);
+                            // a count left over from a step whose Top-K did not run cannot write past the row
+                            const int slot = base + __popc(bm & ((1u << lane) - 1u));
+                            if (emit && slot < a.cand_ld)
+                                a.cand[static_cast<int64_t>(g_r0) * a.cand_ld + slot] =
+                                    (static_cast<uint64_t>(key) << 32) | (0xFFFFFFFFu - static_cast<uint32_t>(s));
+                        }
+                    } else {
+                        if (live) a.scores[static_cast<int64_t>(g_r0) * a.scores_ld + s] = sc;
+                    }
                     if (a.hist) hist_add_global(a.hist + static_cast<int64_t>(g_r0) * kHistBins, live,
                                                 score_order_key(sc) >> 20, lane);
                 } else {
@@ -492,9 +590,11 @@ __global__ void __launch_bounds__((TcCfg<NH, R, NEPI>::kThreads)) __maxnreg__((T
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bar_accempty[buf]);
+                if (kCand && warp == 0 && lane == 0) s_epi_tiles = s_epi_tiles + 1;
                 ++acc;
             }
         }
+        if (kCand && warp == 0 && lane == 0) s_epi_done = 1;
     }
 
     tc_fence_before();
@@ -568,9 +668,9 @@ sa_status launch_cc(const void* q, const void* kc, const IdxArgs& a, cudaStream_
     return launch_status(cudaGetLastError());
 }
 
-template <int NH, int R, int NEPI>
+template <int NH, int R, int NEPI, bool kCand = false>
 sa_status launch_tc(const void* q, const void* kc, const IdxArgs& a, cudaStream_t st) {
-    using C = TcCfg<NH, R, NEPI>;
+    using C = TcCfg<NH, R, NEPI, kCand>;
     CUtensorMap tk, tq;
     // keys: [pool rows][128 bytes]; rows outside the pool read as zero
     const uint64_t kdims[2] = {128, static_cast<uint64_t>(a.pool_pages) * kPage};
@@ -583,14 +683,13 @@ sa_status launch_tc(const void* q, const void* kc, const IdxArgs& a, cudaStream_
     const uint32_t qbox[2] = {128, static_cast<uint32_t>(C::N)};
     if (!encode_tiled(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, q, qdims, qstr, qbox, CU_TENSOR_MAP_SWIZZLE_128B))
         return SA_ECUDA;
-    auto kern = idx_tc_kernel<NH, R, NEPI>;
+    auto kern = idx_tc_kernel<NH, R, NEPI, kCand>;
     const size_t smem = C::smem_bytes(a.rows);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return launch_status(e);
-    // persistent CTAs: two per SM where shared memory, registers and tensor
-    // memory (two accumulator rings) allow, each walking its own item range
     // persistent CTAs: two per SM for one-row groups (two accumulator rings
-    // fit in tensor memory, two CTAs' shared memory and registers fit the SM)
+    // fit in tensor memory, two CTAs' shared memory and registers fit the SM),
+    // each walking its own item range
     int per_sm = 1;
     if (C::kTwoPerSm && 2 * C::kTmemCols <= 512 && 2 * (smem + 2048) <= 227 * 1024) {
         e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);  // all of it as shared
@@ -606,6 +705,16 @@ sa_status launch_tc(const void* q, const void* kc, const IdxArgs& a, cudaStream_
 sa_status index_scores_tc(const void* q, const void* kc, const IdxArgs& a, cudaStream_t st) {
     if (a.rows > kMaxRows) return SA_EUNSUPPORTED;
     const bool grouped = a.seq_of_row != nullptr;
+    if (a.cand) {  // candidates: one-row groups only
+        if (grouped) return SA_EUNSUPPORTED;
+        switch (a.H_I) {
+            case 16: return launch_tc<16, 1, 4, true>(q, kc, a, st);
+            case 32: return launch_tc<32, 1, 4, true>(q, kc, a, st);
+            case 64: return launch_tc<64, 1, 4, true>(q, kc, a, st);
+            case 128: return launch_tc<128, 1, 4, true>(q, kc, a, st);
+            default: return SA_EUNSUPPORTED;
+        }
+    }
     switch (a.H_I) {
         case 16: return grouped ? launch_tc<16, 16, 8>(q, kc, a, st) : launch_tc<16, 1, 4>(q, kc, a, st);
         case 32: return grouped ? launch_tc<32, 8, 8>(q, kc, a, st) : launch_tc<32, 1, 4>(q, kc, a, st);

@@ -198,6 +198,49 @@ sa_status sa_topk_select_hist(const float* scores, int64_t scores_ld, const int3
     return topk_impl(scores, scores_ld, n_valid, rows, k, hist, idx_out, stream);
 }
 
+sa_status sa_index_candidates(const void* q, const float* w, const void* k_cache, int64_t pool_pages, sa_dtype dtype,
+                              const int32_t* page_table, int pages_per_seq, const int32_t* n_visible, int rows,
+                              int H_I, int d_I, int k, int64_t cand_ld, uint64_t* cand, int32_t* cand_cnt,
+                              int32_t* hist, sa_stream_t stream) {
+    if (rows < 0 || H_I < 1 || d_I < 1 || k < 1 || pages_per_seq < 1 || pool_pages < 1) return SA_EINVAL;
+    if (cand_ld < static_cast<int64_t>(pages_per_seq) * 64) return SA_EINVAL;
+    if (rows == 0) return SA_OK;
+    if (!q || !w || !k_cache || !n_visible || !cand || !cand_cnt || !hist) return SA_EINVAL;
+    if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(w, 4) || !aligned(cand, 8) || !aligned(cand_cnt, 4) ||
+        !aligned(hist, 16))
+        return SA_EINVAL;
+    if (dtype != SA_E4M3 || d_I != 128 || rows > 4096) return SA_EUNSUPPORTED;
+    if (cand_ld > 262144 || pool_pages * 64 > (int64_t(1) << 31)) return SA_EUNSUPPORTED;
+    IdxArgs a;
+    a.w = w;
+    a.page_table = page_table;
+    a.pages_per_seq = pages_per_seq;
+    a.pool_pages = pool_pages;
+    a.n_visible = n_visible;
+    a.rows = rows;
+    a.H_I = H_I;
+    a.d_I = d_I;
+    a.scores_ld = cand_ld;
+    a.hist = hist;
+    a.cand = cand;
+    a.cand_ld = cand_ld;
+    a.cand_cnt = cand_cnt;
+    a.k = k;
+    a.err = device_error_word();
+    return index_scores_tc(q, k_cache, a, reinterpret_cast<cudaStream_t>(stream));
+}
+
+sa_status sa_topk_from_candidates(const uint64_t* cand, int64_t cand_ld, int32_t* cand_cnt, const int32_t* n_valid,
+                                  int rows, int k, int32_t* hist, int32_t* idx_out, sa_stream_t stream) {
+    if (rows < 0 || k < 1 || cand_ld < 1) return SA_EINVAL;
+    if (rows == 0) return SA_OK;
+    if (!cand || !cand_cnt || !n_valid || !hist || !idx_out) return SA_EINVAL;
+    if (!aligned(cand, 8) || !aligned(cand_cnt, 4) || !aligned(hist, 4) || !aligned(idx_out, 4)) return SA_EINVAL;
+    if (cand_ld > 262144) return SA_EUNSUPPORTED;
+    return topk_cand_launch(cand, cand_ld, cand_cnt, n_valid, rows, k, hist, idx_out, device_error_word(),
+                            reinterpret_cast<cudaStream_t>(stream));
+}
+
 size_t sa_sparse_mla_workspace_size(int rows, int H, int k, int d_c) {
     if (rows < 1 || H < 1 || k < 1 || d_c < 1) return 0;
     return mla_workspace_bytes(rows, H, k, d_c, mla_decode_splits(rows, k));

@@ -39,19 +39,26 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
 }
 
 struct IdxArgs {
-    const float* w;
-    const int32_t* page_table;
-    int pages_per_seq;
-    int64_t pool_pages;
-    const int32_t* seq_of_row;
-    const int32_t* n_visible;
-    int rows;
-    int H_I;
-    int d_I;
-    float* scores;
-    int64_t scores_ld;
-    int32_t* hist;  // [rows][kHistBins] first-digit counts of the scores written, or null
-    int* err;
+    const float* w = nullptr;
+    const int32_t* page_table = nullptr;
+    int pages_per_seq = 0;
+    int64_t pool_pages = 0;
+    const int32_t* seq_of_row = nullptr;
+    const int32_t* n_visible = nullptr;
+    int rows = 0;
+    int H_I = 0;
+    int d_I = 0;
+    float* scores = nullptr;
+    int64_t scores_ld = 0;
+    int32_t* hist = nullptr;  // [rows][kHistBins] first-digit counts of the scores written, or null
+    int* err = nullptr;
+    // candidate mode (one-row groups): no scores; every key whose first digit is
+    // at or above a proven lower bound on the row's k-th largest is written as
+    // (order key << 32) | ~position to cand[row][cand_cnt[row]++]
+    uint64_t* cand = nullptr;
+    int64_t cand_ld = 0;
+    int32_t* cand_cnt = nullptr;
+    int k = 0;
 };
 
 sa_status index_scores_tc(const void* q, const void* k_cache, const IdxArgs& a, cudaStream_t st);
@@ -59,6 +66,8 @@ sa_status index_scores_cc(const void* q, const void* k_cache, sa_dtype dt, const
 
 sa_status topk_select_launch(const float* scores, int64_t ld, const int32_t* n_valid, int rows, int k,
                              int32_t* hist, int32_t* idx_out, cudaStream_t st);
+sa_status topk_cand_launch(const uint64_t* cand, int64_t cand_ld, int32_t* cand_cnt, const int32_t* n_valid,
+                           int rows, int k, int32_t* hist, int32_t* idx_out, int* err, cudaStream_t st);
 
 struct MlaArgs {
     const void* q_lat;

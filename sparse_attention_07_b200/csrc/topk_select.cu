@@ -626,6 +626,219 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 2)
     }
 }
 
+// ------------------------------------------------------------ from candidates
+// The selection from the indexer's candidates (keys at or above a proven
+// lower bound on each row's k-th largest, as (order key << 32) | ~position)
+// and the row's first-digit counts, which cover every key of the row.  One
+// CTA per row: the counts give the boundary digit and the number of keys
+// above it (all of them are candidates); one pass over the candidates marks
+// those keys in a bitmap of the row's positions and lists the keys on the
+// boundary digit; 8/8/4-bit passes over that list find the final class; the
+// class's lowest positions join the selection, and a block scan of the
+// bitmap writes the positions in ascending order.  The counts and the
+// candidate count are cleared for the next step.
+constexpr int kCMaxN = 262144;          // positions per row (the bitmaps)
+constexpr int kCBmWords = kCMaxN / 32;  // 8192
+constexpr int kCBmPer = kCBmWords / kThreads;
+constexpr int kCListCap = 4096;         // boundary-digit keys held in shared memory
+constexpr int kCDynSmem = 2 * kCBmWords * 4 + kCListCap * 8;
+static_assert(kCBmPer * kThreads == kCBmWords, "bitmap words per thread");
+
+__global__ void __launch_bounds__(kThreads, 1)
+    topk_cand_kernel(const uint64_t* __restrict__ cand, int64_t ld, int32_t* __restrict__ cand_cnt,
+                     const int32_t* __restrict__ n_valid, int k, int32_t* __restrict__ hist,
+                     int32_t* __restrict__ out, int* err) {
+    extern __shared__ __align__(16) uint8_t s_dyn[];
+    uint32_t* s_sel = reinterpret_cast<uint32_t*>(s_dyn);         // [kCBmWords] selected positions
+    uint32_t* s_cls = s_sel + kCBmWords;                           // [kCBmWords] final-class members
+    uint32_t* s_lkey = s_cls + kCBmWords;                          // [kCListCap] boundary keys
+    uint32_t* s_lpos = s_lkey + kCListCap;                         // [kCListCap] their positions
+    __shared__ int s_h[kBins1];
+    __shared__ int s_suf[kBins1 + 1];
+    __shared__ int s_wsum[kWarps];
+    __shared__ int s_sel0[3], s_pass[3];
+    __shared__ int s_nl;
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int row = blockIdx.x;
+    int n = n_valid[row];
+    n = n < 0 ? 0 : (n > ld ? static_cast<int>(ld) : n);
+    int32_t* orow = out + static_cast<int64_t>(row) * k;
+    int32_t* hrow = hist + static_cast<int64_t>(row) * kHistBins;
+    const uint64_t* crow = cand + static_cast<int64_t>(row) * ld;
+    const int cnt = min(cand_cnt[row], n);
+
+    if (n <= k) {  // every position is selected; the rest is padding
+        for (int s = tid; s < k; s += kThreads) orow[s] = s < n ? s : -1;
+    } else {
+        // ---- 1. the boundary digit from the row's counts (highest bins first)
+        constexpr int kPer = kBins0 / kThreads;
+        const int b_hi = kBins0 - 1 - tid * kPer;
+        int hv[kPer], mine = 0;
+#pragma unroll
+        for (int j = 0; j < kPer; ++j) {
+            hv[j] = hrow[b_hi - j];
+            mine += hv[j];
+        }
+        if (tid == 0) {
+            s_sel0[0] = 0;
+            s_sel0[1] = 0;
+            s_sel0[2] = 0;
+            s_nl = 0;
+        }
+#pragma unroll
+        for (int j = 0; j < kCBmPer; ++j) {
+            s_sel[tid * kCBmPer + j] = 0u;
+            s_cls[tid * kCBmPer + j] = 0u;
+        }
+        int total = 0;
+        int above = block_exclusive(mine, lane, warp, s_wsum, total);
+        if (tid == 0 && total != n) record_error(err, kErrTopkRow | 1);  // the counts do not cover the row
+        if (above < k && k <= above + mine) {
+#pragma unroll
+            for (int j = 0; j < kPer; ++j) {
+                if (k <= above + hv[j]) {
+                    s_sel0[0] = b_hi - j;
+                    s_sel0[1] = above;
+                    s_sel0[2] = hv[j];
+                    break;
+                }
+                above += hv[j];
+            }
+        }
+        __syncthreads();
+        const uint32_t d0 = static_cast<uint32_t>(s_sel0[0]);
+        int remaining = k - s_sel0[1];
+        // ---- 2. candidates above the boundary digit are selected; those on it are listed
+        for (int i = tid; i < cnt; i += kThreads) {
+            const uint64_t v = crow[i];
+            const uint32_t key = static_cast<uint32_t>(v >> 32), pos = 0xFFFFFFFFu - static_cast<uint32_t>(v);
+            if (pos >= static_cast<uint32_t>(n)) continue;
+            const uint32_t d = key >> 20;
+            if (d > d0) {
+                atomicOr(&s_sel[pos >> 5], 1u << (pos & 31));
+            } else if (d == d0) {
+                const int slot = atomicAdd(&s_nl, 1);
+                if (slot < kCListCap) {
+                    s_lkey[slot] = key;
+                    s_lpos[slot] = pos;
+                }
+            }
+        }
+        __syncthreads();
+        const bool listed = s_nl <= kCListCap;
+        const int nlist = listed ? s_nl : cnt;
+        // boundary key j of the list (or candidate j when the list overflowed):
+        // returns false when it is not on the boundary digit
+        auto bkey = [&](int j, uint32_t& key, uint32_t& pos) -> bool {
+            if (listed) {
+                key = s_lkey[j];
+                pos = s_lpos[j];
+                return true;
+            }
+            const uint64_t v = crow[j];
+            key = static_cast<uint32_t>(v >> 32);
+            pos = 0xFFFFFFFFu - static_cast<uint32_t>(v);
+            return (key >> 20) == d0 && pos < static_cast<uint32_t>(n);
+        };
+        // ---- 3. refinement passes over the boundary keys (bits 19..12, 11..4, 3..0)
+        uint32_t prefix = d0 << 20, mask = 0xFFF00000u;
+        if (s_sel0[2] != remaining) {
+            for (int pass = 0; pass < 3; ++pass) {
+                const int shift = pass == 0 ? 12 : (pass == 1 ? 4 : 0);
+                const uint32_t dmask = pass == 2 ? 15u : 255u;
+                if (tid < kBins1) s_h[tid] = 0;
+                __syncthreads();
+                for (int j = tid; j < nlist; j += kThreads) {
+                    uint32_t key, pos;
+                    if (bkey(j, key, pos) && (key & mask) == prefix) atomicAdd(&s_h[(key >> shift) & dmask], 1);
+                }
+                __syncthreads();
+                if (tid < kBins1) {
+                    const int in = warp_suffix(s_h[tid], lane);
+                    s_suf[tid] = in;
+                    if (lane == 0) s_wsum[warp] = in;
+                }
+                __syncthreads();
+                if (tid < kBins1) {
+                    int add = 0;
+                    for (int w = warp + 1; w < kBins1 / 32; ++w) add += s_wsum[w];
+                    s_suf[tid] += add;
+                    if (tid == 0) {
+                        s_suf[kBins1] = 0;
+                        s_pass[0] = 0;
+                        s_pass[1] = 0;
+                        s_pass[2] = -1;
+                    }
+                }
+                __syncthreads();
+                if (tid < kBins1) {
+                    const int here = s_suf[tid], up = s_suf[tid + 1];
+                    if (here >= remaining && up < remaining) {
+                        s_pass[0] = tid;
+                        s_pass[1] = up;
+                        s_pass[2] = here - up;
+                    }
+                }
+                __syncthreads();
+                remaining -= s_pass[1];
+                prefix |= static_cast<uint32_t>(s_pass[0]) << shift;
+                mask |= dmask << shift;
+                const bool whole = s_pass[2] == remaining;
+                __syncthreads();  // s_pass is rewritten by the next pass
+                if (whole) break;
+            }
+        }
+        // ---- 4. boundary keys above the final class are selected; its members marked
+        for (int j = tid; j < nlist; j += kThreads) {
+            uint32_t key, pos;
+            if (!bkey(j, key, pos)) continue;
+            const uint32_t m = key & mask;
+            if (m > prefix) atomicOr(&s_sel[pos >> 5], 1u << (pos & 31));
+            else if (m == prefix) atomicOr(&s_cls[pos >> 5], 1u << (pos & 31));
+        }
+        __syncthreads();
+        // ---- 5. the class's `remaining` lowest positions join, then ordered writes
+        uint32_t bsel[kCBmPer];
+        int ncls = 0;
+#pragma unroll
+        for (int j = 0; j < kCBmPer; ++j) ncls += __popc(s_cls[tid * kCBmPer + j]);
+        int tot = 0;
+        int r = block_exclusive(ncls, lane, warp, s_wsum, tot);
+        int nsel = 0;
+#pragma unroll
+        for (int j = 0; j < kCBmPer; ++j) {
+            uint32_t bits = s_cls[tid * kCBmPer + j];
+            uint32_t selw = s_sel[tid * kCBmPer + j];
+            while (bits != 0u && r < remaining) {
+                const uint32_t low = bits & (0u - bits);
+                selw |= low;
+                bits ^= low;
+                ++r;
+            }
+            bsel[j] = selw;
+            nsel += __popc(selw);
+        }
+        __syncthreads();  // s_wsum is reused by the next scan
+        int pos = block_exclusive(nsel, lane, warp, s_wsum, tot);
+#pragma unroll
+        for (int j = 0; j < kCBmPer; ++j) {
+            uint32_t bits = bsel[j];
+            const int p0 = (tid * kCBmPer + j) * 32;
+            while (bits != 0u) {
+                const int b = __ffs(bits) - 1;
+                bits &= bits - 1u;
+                if (pos < k) orow[pos] = p0 + b;
+                ++pos;
+            }
+        }
+    }
+    // the row's counts and candidate count, cleared for the next step
+    __syncthreads();
+    for (int i = tid; i < kHistBins; i += kThreads) hrow[i] = 0;
+    if (tid == 0) cand_cnt[row] = 0;
+}
+
 }  // namespace
 
 sa_status topk_select_launch(const float* scores, int64_t ld, const int32_t* n_valid, int rows, int k,
@@ -635,6 +848,19 @@ sa_status topk_select_launch(const float* scores, int64_t ld, const int32_t* n_v
     cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kDynSmem);
     if (e != cudaSuccess) return launch_status(e);
     topk_kernel<<<rows * kCluster, kThreads, kDynSmem, st>>>(scores, ld, n_valid, k, chunk, hist, idx_out);
+    return launch_status(cudaGetLastError());
+}
+
+}  // namespace sa
+
+namespace sa {
+
+sa_status topk_cand_launch(const uint64_t* cand, int64_t cand_ld, int32_t* cand_cnt, const int32_t* n_valid,
+                           int rows, int k, int32_t* hist, int32_t* idx_out, int* err, cudaStream_t st) {
+    if (cand_ld > kCMaxN) return SA_EUNSUPPORTED;
+    cudaError_t e = cudaFuncSetAttribute(topk_cand_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kCDynSmem);
+    if (e != cudaSuccess) return launch_status(e);
+    topk_cand_kernel<<<rows, kThreads, kCDynSmem, st>>>(cand, cand_ld, cand_cnt, n_valid, k, hist, idx_out, err);
     return launch_status(cudaGetLastError());
 }
 
