@@ -229,11 +229,12 @@ def peaks():
 class DecodeStep:
     """Buffers and launches of one indexer -> Top-K -> sparse-MLA step."""
 
-    def __init__(self, inp, sa, topk_path: str = "scores"):
+    def __init__(self, inp, sa, topk_path: str = "scores", out_dtype=torch.bfloat16):
         self.sa, self.inp, self.cfg = sa, inp, inp["cfg"]
         cfg, dev = self.cfg, inp["q_idx"].device
         self.idx = torch.empty(cfg.rows, cfg.topk, dtype=torch.int32, device=dev)
-        self.out = torch.empty(cfg.rows, cfg.H, cfg.d_c, dtype=torch.float32, device=dev)
+        # the attention output as the up-projection reads it (bf16; fp32 accumulation)
+        self.out = torch.empty(cfg.rows, cfg.H, cfg.d_c, dtype=out_dtype, device=dev)
         self.lse = torch.empty(cfg.rows, cfg.H, dtype=torch.float32, device=dev)
         self.prefill = cfg.prefill_start >= 0
         # decode with one query row per sequence on the tensor-core indexer:
@@ -355,7 +356,7 @@ class CsaStep:
     """indexer over the compressed keys -> Top-K -> window slots + sparse
     attention over the selected entries and the window."""
 
-    def __init__(self, inp, sa):
+    def __init__(self, inp, sa, out_dtype=torch.bfloat16):
         self.sa, self.inp, self.cfg = sa, inp, inp["cfg"]
         c, dev = self.cfg, inp["q"].device
         S = c.n_seqs
@@ -371,7 +372,7 @@ class CsaStep:
         self.hist = sa.topk_histogram(S, dev)
         self.idx = torch.empty(S, c.topk, dtype=torch.int32, device=dev)
         self.slots = torch.empty(S, c.topk + c.window, dtype=torch.int32, device=dev)
-        self.out = torch.empty(S, c.H, c.c, dtype=torch.float32, device=dev)
+        self.out = torch.empty(S, c.H, c.c, dtype=out_dtype, device=dev)
         self.ws = torch.empty(max(1, sa.sparse_mla_workspace_size(S, c.H, c.topk + c.window, c.c)),
                               dtype=torch.uint8, device=dev)
         combine = sa.sparse_mla_workspace_size(S, c.H, c.topk + c.window, c.c) > \
@@ -693,17 +694,17 @@ def describe(cfg, flush_note):
             "batch": cfg.B, "seq_len": cfg.L, "heads": cfg.H, "l2": flush_note}
 
 
-def make_step(cfg, dev, rank, sa, topk_path: str = "scores"):
+def make_step(cfg, dev, rank, sa, topk_path: str = "scores", out_dtype=torch.bfloat16):
     """Seeded inputs of a workload (each rank its own seed) and its step."""
     if isinstance(cfg, W.DSAConfig):
         inp = W.dsa_inputs(cfg, dev, seed=rank_seed(cfg.seed, rank))
-        return inp, DecodeStep(inp, sa, topk_path)
+        return inp, DecodeStep(inp, sa, topk_path, out_dtype)
     if isinstance(cfg, W.NSAConfig):
         inp = W.nsa_inputs(cfg, dev, seed=rank_seed(cfg.seed, rank))
         return inp, NsaStep(inp, sa)
     if isinstance(cfg, W.CSAConfig):
         inp = W.csa_inputs(cfg, dev, seed=rank_seed(cfg.seed, rank))
-        return inp, CsaStep(inp, sa)
+        return inp, CsaStep(inp, sa, out_dtype)
     inp = W.block_inputs(cfg, dev, seed=rank_seed(cfg.seed, rank))
     return inp, BlockStep(inp, sa)
 
@@ -712,7 +713,8 @@ def measure(cfg, args, dev, local, rank, ws, sa, flush, config_key):
     """Warm-up, then the timed steps (graph replays), the per-stage steps and
     the end-to-end steps of one workload; returns the result fields of its
     JSON line (without the top-level run keys) and the inputs."""
-    inp, step = make_step(cfg, dev, rank, sa, args.topk_path)
+    inp, step = make_step(cfg, dev, rank, sa, args.topk_path,
+                          torch.bfloat16 if args.out_dtype == "bf16" else torch.float32)
     for _ in range(args.warmup):
         flush.zero_()
         step.indexer()
@@ -889,6 +891,9 @@ def measure(cfg, args, dev, local, rank, ws, sa, flush, config_key):
         "gpu_launches": step.launches_per_step * args.steps,
         "clocks": clk.summary(),
     })
+    if isinstance(step, (DecodeStep, CsaStep)):
+        res["config"]["attention_output"] = ("bf16 (fp32 softmax and accumulation, rounded once)"
+                                             if step.out.dtype == torch.bfloat16 else "fp32")
     if isinstance(step, DecodeStep):
         res["config"]["indexer_output"] = ("Top-K candidates (keys at or above a proven bound on the row's k-th "
                                            "largest)" if step.cand_path else "every score")
@@ -1089,6 +1094,8 @@ def main(argv=None):
                    choices=sorted(list(W.DSA_CONFIGS) + list(W.BLOCK_CONFIGS) + list(W.NSA_CONFIGS) +
                                   list(W.CSA_CONFIGS) + ["crossover"]))
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--out-dtype", choices=["bf16", "f32"], default="bf16",
+                   help="DSA / CSA: storage type of the attention output (the step's result)")
     p.add_argument("--topk-path", choices=["cand", "scores"], default="scores",
                    help="decode: the indexer keeps Top-K candidates (cand) or writes every score (scores)")
     p.add_argument("--no-l128k", action="store_true",

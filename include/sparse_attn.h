@@ -13,7 +13,7 @@
  *   sa_index_candidates / sa_topk_from_candidates
  *                        the same two steps for decode, the indexer keeping only
  *                        the keys that can still be in the Top-K
- *   sa_sparse_mla_decode / sa_sparse_mla_prefill
+ *   sa_sparse_mla_decode / sa_sparse_mla_prefill (_bf16: bf16 output)
  *                        softmax over the selected set of the absorbed content score
  *                        plus the RoPE score, scaled; output sum_j a_j c_j in latent space
  *   sa_block_mean_pool   mean-pooled block keys (run when blocks complete)
@@ -215,6 +215,29 @@ sa_status sa_sparse_mla_prefill(const void* q_lat, const void* q_rope,
                                 sa_stream_t stream);
 
 /*
+ * sa_sparse_mla_decode / sa_sparse_mla_prefill with the output stored as bf16:
+ * out [rows][H][d_c] bf16, each element the fp32 result of those calls
+ * rounded to the nearest bf16 (ties to even) — bit for bit the fp32 call's
+ * output so rounded.  Softmax and accumulation stay fp32; lse is fp32 as
+ * there.  Half the output bytes (the up-projection reads o_lat as bf16).
+ */
+sa_status sa_sparse_mla_decode_bf16(const void* q_lat, const void* q_rope,
+                                    const void* c_cache, int64_t c_ld, const void* kr_cache, int64_t kr_ld,
+                                    int64_t pool_pages, const int32_t* page_table, int pages_per_seq,
+                                    const int32_t* seq_of_row,
+                                    const int32_t* idx, int rows, int H, int k, int d_c, int d_R, float scale,
+                                    void* out, float* lse, void* workspace, size_t workspace_bytes,
+                                    sa_stream_t stream);
+
+sa_status sa_sparse_mla_prefill_bf16(const void* q_lat, const void* q_rope,
+                                     const void* c_cache, int64_t c_ld, const void* kr_cache, int64_t kr_ld,
+                                     int64_t pool_pages, const int32_t* page_table, int pages_per_seq,
+                                     const int32_t* seq_of_row,
+                                     const int32_t* idx, int rows, int H, int k, int d_c, int d_R, float scale,
+                                     void* out, float* lse, void* workspace, size_t workspace_bytes,
+                                     sa_stream_t stream);
+
+/*
  * Dense MLA decode: the same attention as sa_sparse_mla_decode over every
  * visible position instead of a selection (row r attends to positions
  * 0 .. n_visible[r]-1 of its sequence).  It is the short-sequence mode of the
@@ -252,6 +275,14 @@ sa_status sa_mla_absorb_query(const void* q_c, const void* U_K, int rows, int H,
 
 sa_status sa_mla_up_project(const float* o_lat, const void* U_V, int rows, int H, int d_c, int d_v, float* out,
                             sa_stream_t stream);
+
+/*
+ * sa_mla_up_project with o_lat [rows][H][d_c] bf16 (the output of the _bf16
+ * sparse-MLA calls): the same product, bit for bit the fp32 call's result on
+ * the fp32 o_lat that rounds to it (that call rounds o_lat to bf16 first).
+ */
+sa_status sa_mla_up_project_bf16(const void* o_lat, const void* U_V, int rows, int H, int d_c, int d_v, float* out,
+                                 sa_stream_t stream);
 
 /*
  * Sparse MLA decode for callers that cannot allocate device memory.  The

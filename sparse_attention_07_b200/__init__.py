@@ -31,7 +31,8 @@ EXPORTS = (
     "sa_dense_mla_workspace_size", "sa_dense_mla_decode", "sa_mla_absorb_query", "sa_mla_up_project",
     "sa_nsa_compress", "sa_nsa_decode", "sa_csa_compress", "sa_csa_window_index",
     "sa_index_scores_hist", "sa_topk_select_hist", "sa_set_wait_limit_ns",
-    "sa_index_candidates", "sa_topk_from_candidates",
+    "sa_index_candidates", "sa_topk_from_candidates", "sa_sparse_mla_decode_bf16", "sa_sparse_mla_prefill_bf16",
+    "sa_mla_up_project_bf16",
 )
 
 # Size of the library's static device array behind sparse_mla_decode_static
@@ -71,11 +72,14 @@ def lib():
         L.sa_sparse_mla_prefill_workspace_size.restype = SZ
         L.sa_sparse_mla_prefill_workspace_size.argtypes = [I, I, I, I]
         L.sa_sparse_mla_prefill.argtypes = [P, P, P, I64, P, I64, I64, P, I, P, P, I, I, I, I, I, F, P, P, P, SZ, P]
+        L.sa_sparse_mla_decode_bf16.argtypes = L.sa_sparse_mla_decode.argtypes
+        L.sa_sparse_mla_prefill_bf16.argtypes = L.sa_sparse_mla_prefill.argtypes
         L.sa_dense_mla_workspace_size.restype = SZ
         L.sa_dense_mla_workspace_size.argtypes = [I, I, I, I]
         L.sa_dense_mla_decode.argtypes = [P, P, P, I64, P, I64, I64, P, I, P, P, I, I, I, I, I, F, P, P, P, SZ, P]
         L.sa_mla_absorb_query.argtypes = [P, P, I, I, I, I, P, P]
         L.sa_mla_up_project.argtypes = [P, P, I, I, I, I, P, P]
+        L.sa_mla_up_project_bf16.argtypes = [P, P, I, I, I, I, P, P]
         L.sa_sparse_mla_decode_static.argtypes = [P, P, P, I64, P, I64, I64, P, I, P, P, I, I, I, I, I, F, P, P, P]
         L.sa_block_mean_pool.argtypes = [P, I64, I64, I64, I, I, I, I, I, P, I64, P]
         L.sa_block_sparse_attn.argtypes = [P, P, I64, P, P, I64, I64, I64, I, I, I, I, I, I, I, I, F, P, P, P]
@@ -220,23 +224,27 @@ def _mla_args(q_lat, q_rope, c_cache, kr_cache, idx, out, lse):
     k = idx.shape[1]
     if out is None:
         out = torch.empty(rows, H, d_c, dtype=torch.float32, device=q_lat.device)
+    if out.dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError(f"sparse MLA output must be float32 or bfloat16, not {out.dtype}")
     pool_pages = c_cache.shape[0] // 64
     return rows, H, d_c, d_R, k, out, lse, pool_pages
 
 
 def sparse_mla_decode(q_lat, q_rope, c_cache, kr_cache, idx, scale: float, pages_per_seq: int, page_table=None,
                       seq_of_row=None, out=None, lse=None, workspace=None):
-    """Sparse MLA (latent aggregate) [rows, H, d_c] fp32; optional lse [rows, H]."""
+    """Sparse MLA (latent aggregate) [rows, H, d_c], fp32 (or bf16 when `out`
+    is a bf16 tensor); optional lse [rows, H]."""
     rows, H, d_c, d_R, k, out, lse, pool_pages = _mla_args(q_lat, q_rope, c_cache, kr_cache, idx, out, lse)
     need = sparse_mla_workspace_size(rows, H, k, d_c)
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=q_lat.device)
     wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    st = lib().sa_sparse_mla_decode(_p(q_lat), _p(q_rope), _p(c_cache), c_cache.stride(0), _p(kr_cache),
-                                    kr_cache.stride(0), pool_pages, _p(page_table), pages_per_seq, _p(seq_of_row),
-                                    _p(idx), rows, H, k, d_c, d_R, float(scale), _p(out), _p(lse), _p(workspace),
-                                    wbytes, _stream())
-    _check("sa_sparse_mla_decode", st)
+    name = "sa_sparse_mla_decode_bf16" if out.dtype == torch.bfloat16 else "sa_sparse_mla_decode"
+    st = getattr(lib(), name)(_p(q_lat), _p(q_rope), _p(c_cache), c_cache.stride(0), _p(kr_cache),
+                              kr_cache.stride(0), pool_pages, _p(page_table), pages_per_seq, _p(seq_of_row),
+                              _p(idx), rows, H, k, d_c, d_R, float(scale), _p(out), _p(lse), _p(workspace),
+                              wbytes, _stream())
+    _check(name, st)
     return out
 
 
@@ -251,11 +259,12 @@ def sparse_mla_prefill(q_lat, q_rope, c_cache, kr_cache, idx, scale: float, page
         workspace = torch.empty(sparse_mla_prefill_workspace_size(rows, H, k, d_c), dtype=torch.uint8,
                                 device=q_lat.device)
     wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    st = lib().sa_sparse_mla_prefill(_p(q_lat), _p(q_rope), _p(c_cache), c_cache.stride(0), _p(kr_cache),
-                                     kr_cache.stride(0), pool_pages, _p(page_table), pages_per_seq, _p(seq_of_row),
-                                     _p(idx), rows, H, k, d_c, d_R, float(scale), _p(out), _p(lse), _p(workspace),
-                                     wbytes, _stream())
-    _check("sa_sparse_mla_prefill", st)
+    name = "sa_sparse_mla_prefill_bf16" if out.dtype == torch.bfloat16 else "sa_sparse_mla_prefill"
+    st = getattr(lib(), name)(_p(q_lat), _p(q_rope), _p(c_cache), c_cache.stride(0), _p(kr_cache),
+                              kr_cache.stride(0), pool_pages, _p(page_table), pages_per_seq, _p(seq_of_row),
+                              _p(idx), rows, H, k, d_c, d_R, float(scale), _p(out), _p(lse), _p(workspace),
+                              wbytes, _stream())
+    _check(name, st)
     return out
 
 
@@ -295,12 +304,18 @@ def mla_absorb_query(q_c, U_K, q_lat=None):
 
 
 def mla_up_project(o_lat, U_V, out=None):
-    """out[r,h,:] = U_V[h] o_lat[r,h,:]: o_lat [rows,H,d_c] fp32, U_V [H,d_v,d_c] bf16 -> [rows,H,d_v] fp32."""
+    """out[r,h,:] = U_V[h] o_lat[r,h,:]: o_lat [rows,H,d_c] fp32 or bf16, U_V [H,d_v,d_c] bf16 -> [rows,H,d_v] fp32."""
     rows, H, d_c = o_lat.shape
     d_v = U_V.shape[1]
     if out is None:
         out = torch.empty(rows, H, d_v, dtype=torch.float32, device=o_lat.device)
-    _check("sa_mla_up_project", lib().sa_mla_up_project(_p(o_lat), _p(U_V), rows, H, d_c, d_v, _p(out), _stream()))
+    if o_lat.dtype == torch.bfloat16:
+        name = "sa_mla_up_project_bf16"
+    elif o_lat.dtype == torch.float32:
+        name = "sa_mla_up_project"
+    else:
+        raise TypeError(f"o_lat must be float32 or bfloat16, not {o_lat.dtype}")
+    _check(name, getattr(lib(), name)(_p(o_lat), _p(U_V), rows, H, d_c, d_v, _p(out), _stream()))
     return out
 
 

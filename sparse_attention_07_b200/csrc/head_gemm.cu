@@ -233,9 +233,9 @@ sa_status mla_absorb_query_launch(const void* q_c, const void* U_K, int rows, in
     return head_gemm_launch(U_K, g, st);
 }
 
-sa_status mla_up_project_launch(const float* o_lat, const void* U_V, int rows, int H, int d_c, int d_v, float* out,
-                                int* err, cudaStream_t st) {
-    GemmArgs g{o_lat, 1, rows, H, d_v, d_c, 0, out, 1, err};
+sa_status mla_up_project_launch(const void* o_lat, bool o_lat_fp32, const void* U_V, int rows, int H, int d_c,
+                                int d_v, float* out, int* err, cudaStream_t st) {
+    GemmArgs g{o_lat, o_lat_fp32 ? 1 : 0, rows, H, d_v, d_c, 0, out, 1, err};
     return head_gemm_launch(U_V, g, st);
 }
 

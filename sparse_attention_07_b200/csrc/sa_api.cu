@@ -249,7 +249,7 @@ size_t sa_sparse_mla_workspace_size(int rows, int H, int k, int d_c) {
 static sa_status mla_common(const void* q_lat, const void* q_rope, const void* c_cache, int64_t c_ld,
                             const void* kr_cache, int64_t kr_ld, int64_t pool_pages, const int32_t* page_table,
                             int pages_per_seq, const int32_t* seq_of_row, const int32_t* idx, int rows, int H, int k,
-                            int d_c, int d_R, float scale, float* out, float* lse, MlaArgs* a) {
+                            int d_c, int d_R, float scale, void* out, bool out_bf16, float* lse, MlaArgs* a) {
     if (rows < 0 || H < 1 || k < 1 || pages_per_seq < 1 || pool_pages < 1 || !std::isfinite(scale)) return SA_EINVAL;
     if (!q_lat || !q_rope || !c_cache || !kr_cache || !out) return SA_EINVAL;
     if (d_c != 512 || d_R != 64 || H > 128) return SA_EUNSUPPORTED;
@@ -276,22 +276,23 @@ static sa_status mla_common(const void* q_lat, const void* q_rope, const void* c
     a->d_c = d_c;
     a->d_R = d_R;
     a->scale = scale;
-    a->out = out;
+    a->out = out_bf16 ? nullptr : static_cast<float*>(out);
+    a->out_bf16 = out_bf16 ? out : nullptr;
     a->lse = lse;
     a->err = device_error_word();
     return SA_OK;
 }
 
-sa_status sa_sparse_mla_decode(const void* q_lat, const void* q_rope, const void* c_cache, int64_t c_ld,
-                               const void* kr_cache, int64_t kr_ld, int64_t pool_pages, const int32_t* page_table,
-                               int pages_per_seq, const int32_t* seq_of_row, const int32_t* idx, int rows, int H,
-                               int k, int d_c, int d_R, float scale, float* out, float* lse, void* workspace,
-                               size_t workspace_bytes, sa_stream_t stream) {
+static sa_status mla_decode_impl(const void* q_lat, const void* q_rope, const void* c_cache, int64_t c_ld,
+                                 const void* kr_cache, int64_t kr_ld, int64_t pool_pages, const int32_t* page_table,
+                                 int pages_per_seq, const int32_t* seq_of_row, const int32_t* idx, int rows, int H,
+                                 int k, int d_c, int d_R, float scale, void* out, bool out_bf16, float* lse,
+                                 void* workspace, size_t workspace_bytes, sa_stream_t stream) {
     if (rows == 0) return SA_OK;
     if (!idx) return SA_EINVAL;
     MlaArgs a;
     sa_status s = mla_common(q_lat, q_rope, c_cache, c_ld, kr_cache, kr_ld, pool_pages, page_table, pages_per_seq,
-                             seq_of_row, idx, rows, H, k, d_c, d_R, scale, out, lse, &a);
+                             seq_of_row, idx, rows, H, k, d_c, d_R, scale, out, out_bf16, lse, &a);
     if (s != SA_OK) return s;
     const int ns = mla_decode_splits(rows, k);
     if (!workspace || !aligned(workspace, 256) || workspace_bytes < mla_workspace_bytes(rows, H, k, d_c, ns))
@@ -304,21 +305,61 @@ size_t sa_sparse_mla_prefill_workspace_size(int rows, int H, int k, int d_c) {
     return mla_workspace_bytes(rows, H, k, d_c, 1);
 }
 
-sa_status sa_sparse_mla_prefill(const void* q_lat, const void* q_rope, const void* c_cache, int64_t c_ld,
-                                const void* kr_cache, int64_t kr_ld, int64_t pool_pages, const int32_t* page_table,
-                                int pages_per_seq, const int32_t* seq_of_row, const int32_t* idx, int rows, int H,
-                                int k, int d_c, int d_R, float scale, float* out, float* lse, void* workspace,
-                                size_t workspace_bytes, sa_stream_t stream) {
+static sa_status mla_prefill_impl(const void* q_lat, const void* q_rope, const void* c_cache, int64_t c_ld,
+                                  const void* kr_cache, int64_t kr_ld, int64_t pool_pages, const int32_t* page_table,
+                                  int pages_per_seq, const int32_t* seq_of_row, const int32_t* idx, int rows, int H,
+                                  int k, int d_c, int d_R, float scale, void* out, bool out_bf16, float* lse,
+                                  void* workspace, size_t workspace_bytes, sa_stream_t stream) {
     if (rows == 0) return SA_OK;
     if (!idx) return SA_EINVAL;
     MlaArgs a;
     sa_status s = mla_common(q_lat, q_rope, c_cache, c_ld, kr_cache, kr_ld, pool_pages, page_table, pages_per_seq,
-                             seq_of_row, idx, rows, H, k, d_c, d_R, scale, out, lse, &a);
+                             seq_of_row, idx, rows, H, k, d_c, d_R, scale, out, out_bf16, lse, &a);
     if (s != SA_OK) return s;
     if (k > 64 * kMaxTilesPerCta) return SA_EUNSUPPORTED;
     if (!workspace || !aligned(workspace, 256) || workspace_bytes < mla_workspace_bytes(rows, H, k, d_c, 1))
         return SA_EINVAL;
     return sparse_mla_launch(a, 1, workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+sa_status sa_sparse_mla_decode(const void* q_lat, const void* q_rope, const void* c_cache, int64_t c_ld,
+                               const void* kr_cache, int64_t kr_ld, int64_t pool_pages, const int32_t* page_table,
+                               int pages_per_seq, const int32_t* seq_of_row, const int32_t* idx, int rows, int H,
+                               int k, int d_c, int d_R, float scale, float* out, float* lse, void* workspace,
+                               size_t workspace_bytes, sa_stream_t stream) {
+    return mla_decode_impl(q_lat, q_rope, c_cache, c_ld, kr_cache, kr_ld, pool_pages, page_table, pages_per_seq,
+                           seq_of_row, idx, rows, H, k, d_c, d_R, scale, out, false, lse, workspace,
+                           workspace_bytes, stream);
+}
+
+sa_status sa_sparse_mla_decode_bf16(const void* q_lat, const void* q_rope, const void* c_cache, int64_t c_ld,
+                                    const void* kr_cache, int64_t kr_ld, int64_t pool_pages, const int32_t* page_table,
+                                    int pages_per_seq, const int32_t* seq_of_row, const int32_t* idx, int rows, int H,
+                                    int k, int d_c, int d_R, float scale, void* out, float* lse, void* workspace,
+                                    size_t workspace_bytes, sa_stream_t stream) {
+    return mla_decode_impl(q_lat, q_rope, c_cache, c_ld, kr_cache, kr_ld, pool_pages, page_table, pages_per_seq,
+                           seq_of_row, idx, rows, H, k, d_c, d_R, scale, out, true, lse, workspace,
+                           workspace_bytes, stream);
+}
+
+sa_status sa_sparse_mla_prefill(const void* q_lat, const void* q_rope, const void* c_cache, int64_t c_ld,
+                                const void* kr_cache, int64_t kr_ld, int64_t pool_pages, const int32_t* page_table,
+                                int pages_per_seq, const int32_t* seq_of_row, const int32_t* idx, int rows, int H,
+                                int k, int d_c, int d_R, float scale, float* out, float* lse, void* workspace,
+                                size_t workspace_bytes, sa_stream_t stream) {
+    return mla_prefill_impl(q_lat, q_rope, c_cache, c_ld, kr_cache, kr_ld, pool_pages, page_table, pages_per_seq,
+                            seq_of_row, idx, rows, H, k, d_c, d_R, scale, out, false, lse, workspace,
+                            workspace_bytes, stream);
+}
+
+sa_status sa_sparse_mla_prefill_bf16(const void* q_lat, const void* q_rope, const void* c_cache, int64_t c_ld,
+                                     const void* kr_cache, int64_t kr_ld, int64_t pool_pages, const int32_t* page_table,
+                                     int pages_per_seq, const int32_t* seq_of_row, const int32_t* idx, int rows, int H,
+                                     int k, int d_c, int d_R, float scale, void* out, float* lse, void* workspace,
+                                     size_t workspace_bytes, sa_stream_t stream) {
+    return mla_prefill_impl(q_lat, q_rope, c_cache, c_ld, kr_cache, kr_ld, pool_pages, page_table, pages_per_seq,
+                            seq_of_row, idx, rows, H, k, d_c, d_R, scale, out, true, lse, workspace,
+                            workspace_bytes, stream);
 }
 
 size_t sa_dense_mla_workspace_size(int rows, int H, int L_max, int d_c) {
@@ -334,7 +375,7 @@ sa_status sa_dense_mla_decode(const void* q_lat, const void* q_rope, const void*
     if (!n_visible || !aligned(n_visible, 4)) return SA_EINVAL;
     MlaArgs a;
     sa_status s = mla_common(q_lat, q_rope, c_cache, c_ld, kr_cache, kr_ld, pool_pages, page_table, pages_per_seq,
-                             seq_of_row, nullptr, rows, H, L_max, d_c, d_R, scale, out, lse, &a);
+                             seq_of_row, nullptr, rows, H, L_max, d_c, d_R, scale, out, false, lse, &a);
     if (s != SA_OK) return s;
     a.n_visible = n_visible;
     const int ns = mla_decode_splits(rows, L_max);
@@ -389,7 +430,7 @@ sa_status sa_sparse_mla_decode_static(const void* q_lat, const void* q_rope, con
     if (!idx) return SA_EINVAL;
     MlaArgs a;
     sa_status s = mla_common(q_lat, q_rope, c_cache, c_ld, kr_cache, kr_ld, pool_pages, page_table, pages_per_seq,
-                             seq_of_row, idx, rows, H, k, d_c, d_R, scale, out, lse, &a);
+                             seq_of_row, idx, rows, H, k, d_c, d_R, scale, out, false, lse, &a);
     if (s != SA_OK) return s;
     const int ns = mla_decode_splits(rows, k);
     const size_t need = mla_workspace_bytes(rows, H, k, d_c, ns);
@@ -410,15 +451,25 @@ sa_status sa_mla_absorb_query(const void* q_c, const void* U_K, int rows, int H,
                                    reinterpret_cast<cudaStream_t>(stream));
 }
 
-sa_status sa_mla_up_project(const float* o_lat, const void* U_V, int rows, int H, int d_c, int d_v, float* out,
-                            sa_stream_t stream) {
+static sa_status up_project_impl(const void* o_lat, bool o_lat_fp32, const void* U_V, int rows, int H, int d_c,
+                                 int d_v, float* out, sa_stream_t stream) {
     if (rows < 0 || H < 1 || d_c < 1 || d_v < 1) return SA_EINVAL;
     if (rows == 0) return SA_OK;
     if (!o_lat || !U_V || !out) return SA_EINVAL;
     if (d_c % 64 != 0 || d_c > 512 || d_v % 128 != 0 || H > 65535) return SA_EUNSUPPORTED;
     if (!aligned(o_lat, 16) || !aligned(U_V, 16) || !aligned(out, 4)) return SA_EINVAL;
-    return mla_up_project_launch(o_lat, U_V, rows, H, d_c, d_v, out, device_error_word(),
+    return mla_up_project_launch(o_lat, o_lat_fp32, U_V, rows, H, d_c, d_v, out, device_error_word(),
                                  reinterpret_cast<cudaStream_t>(stream));
+}
+
+sa_status sa_mla_up_project(const float* o_lat, const void* U_V, int rows, int H, int d_c, int d_v, float* out,
+                            sa_stream_t stream) {
+    return up_project_impl(o_lat, true, U_V, rows, H, d_c, d_v, out, stream);
+}
+
+sa_status sa_mla_up_project_bf16(const void* o_lat, const void* U_V, int rows, int H, int d_c, int d_v, float* out,
+                                 sa_stream_t stream) {
+    return up_project_impl(o_lat, false, U_V, rows, H, d_c, d_v, out, stream);
 }
 
 sa_status sa_block_mean_pool(const void* K, int64_t stride_b, int64_t stride_t, int64_t stride_h, int B, int L,

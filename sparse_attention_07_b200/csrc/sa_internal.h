@@ -87,6 +87,7 @@ struct MlaArgs {
     float* out;
     float* lse;
     int* err;
+    void* out_bf16 = nullptr;  // [rows][H][d_c] bf16 output in place of `out` when set
 };
 
 // Sparse MLA: the two CTAs of a pair exchange partial scores through an
@@ -104,8 +105,8 @@ sa_status sparse_mla_launch(const MlaArgs& a, int nsplit, void* ws, size_t ws_by
 
 sa_status mla_absorb_query_launch(const void* q_c, const void* U_K, int rows, int H, int d_C, int d_c, void* q_lat,
                                   int* err, cudaStream_t st);
-sa_status mla_up_project_launch(const float* o_lat, const void* U_V, int rows, int H, int d_c, int d_v, float* out,
-                                int* err, cudaStream_t st);
+sa_status mla_up_project_launch(const void* o_lat, bool o_lat_fp32, const void* U_V, int rows, int H, int d_c,
+                                int d_v, float* out, int* err, cudaStream_t st);
 
 sa_status block_mean_pool_launch(const void* K, int64_t sb, int64_t st_, int64_t sh, int B, int L, int H, int D,
                                  int block, float* pooled, int64_t pooled_ld, cudaStream_t st);

@@ -101,6 +101,12 @@ __device__ __forceinline__ int idx_at(const MlaArgs& a, int r, int slot) {
     return slot < a.n_visible[r] ? slot : -1;
 }
 
+// Four fp32 values rounded to bf16 (nearest, ties to even), packed in order.
+__device__ __forceinline__ uint2 bf16x4_bits(float4 f) {
+    const __nv_bfloat162 lo = __floats2bfloat162_rn(f.x, f.y), hi = __floats2bfloat162_rn(f.z, f.w);
+    return make_uint2(*reinterpret_cast<const uint32_t*>(&lo), *reinterpret_cast<const uint32_t*>(&hi));
+}
+
 template <int N>
 __device__ __forceinline__ float tree_max(float (&v)[N]) {
 #pragma unroll
@@ -532,6 +538,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1) mla_ker
         if (ok && !*wc.abort) {
             tc_fence_after();
             const bool partial = ka.nsplit > 1;
+            const bool bf = !partial && a.out_bf16 != nullptr;  // final output rounded to bf16
             const bool empty = !(l > 0.f);
             const float inv = (!empty && !partial) ? 1.f / l : 1.f;
             float* srow = reinterpret_cast<float*>(sStage + h * kORowBytes);
@@ -552,11 +559,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1) mla_ker
                     f.y = empty ? 0.f : __uint_as_float(o[j + 1]) * inv;
                     f.z = empty ? 0.f : __uint_as_float(o[j + 2]) * inv;
                     f.w = empty ? 0.f : __uint_as_float(o[j + 3]) * inv;
-                    *reinterpret_cast<float4*>(srow + c + j) = f;
+                    if (bf)
+                        *reinterpret_cast<uint2*>(reinterpret_cast<uint8_t*>(srow) + 2 * (c + j)) = bf16x4_bits(f);
+                    else
+                        *reinterpret_cast<float4*>(srow + c + j) = f;
                 }
             }
             fence_proxy_async_smem();  // generic-proxy writes -> bulk-copy reads
-            if (h < a.H) {
+            if (h < a.H && bf) {
+                uint8_t* dst = static_cast<uint8_t*>(a.out_bf16) +
+                               ((static_cast<int64_t>(r) * a.H + h) * a.d_c + rank * 256) * 2;
+                bulk_copy_s2g(dst, srow, 256 * 2);
+                if (rank == 0 && a.lse)
+                    a.lse[static_cast<int64_t>(r) * a.H + h] =
+                        l > 0.f ? (m + log2f(lx)) * 0.6931471805599453f : -INFINITY;
+                bulk_wait_all();
+            } else if (h < a.H) {
                 float* dst = partial ? ka.ws_o + ((static_cast<int64_t>(r) * ka.nsplit + split) * a.H + h) * 512 + rank * 256
                                      : a.out + (static_cast<int64_t>(r) * a.H + h) * a.d_c + rank * 256;
                 bulk_copy_s2g(dst, srow, 256 * 4);
@@ -658,11 +676,19 @@ __global__ void __launch_bounds__(kCombThreads, 3) mla_combine_kernel(const MlaK
         }
     }
     const float inv = L > 0.f ? 1.f / L : 0.f;
-    float* dst = a.out + (static_cast<int64_t>(r) * a.H + h) * a.d_c + d;
+    const int64_t o0 = (static_cast<int64_t>(r) * a.H + h) * a.d_c + d;
+    if (a.out_bf16) {
+        uint2* dst = reinterpret_cast<uint2*>(static_cast<uint8_t*>(a.out_bf16) + o0 * 2);
 #pragma unroll
-    for (int p = 0; p < 4; ++p)
-        *reinterpret_cast<float4*>(dst + 128 * p) =
-            make_float4(acc[p].x * inv, acc[p].y * inv, acc[p].z * inv, acc[p].w * inv);
+        for (int p = 0; p < 4; ++p)
+            dst[32 * p] = bf16x4_bits(make_float4(acc[p].x * inv, acc[p].y * inv, acc[p].z * inv, acc[p].w * inv));
+    } else {
+        float* dst = a.out + o0;
+#pragma unroll
+        for (int p = 0; p < 4; ++p)
+            *reinterpret_cast<float4*>(dst + 128 * p) =
+                make_float4(acc[p].x * inv, acc[p].y * inv, acc[p].z * inv, acc[p].w * inv);
+    }
     if ((threadIdx.x & 31) == 0 && a.lse)
         a.lse[static_cast<int64_t>(r) * a.H + h] = L > 0.f ? (M + log2f(LX)) * 0.6931471805599453f : -INFINITY;
 }

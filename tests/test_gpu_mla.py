@@ -172,3 +172,30 @@ def test_sparse_mla_bad_position_is_reported():
     out, _ = _run(sa.sparse_mla_decode, cfg, inp, idx)
     assert sa.check_device_error() == 0
     assert_attention_close(out, ref_out, "after the reports")
+
+
+@pytest.mark.parametrize("fn_name,rows,H,k,L", [
+    ("decode", 3, 128, 2048, 5000),   # keys split over several pairs: the combine writes the output
+    ("decode", 80, 128, 256, 700),    # one pair per row: the attention kernel writes it
+    ("decode", 5, 77, 33, 40),
+    ("prefill", 6, 128, 1000, 3000),
+])
+def test_sparse_mla_bf16_output(fn_name, rows, H, k, L):
+    """The bf16-output calls: every element is the fp32 call's output rounded
+    to the nearest bf16 (bit for bit), lse as the fp32 call's, and the result
+    within the attention tolerance of the oracle."""
+    cfg, inp, idx = _case(rows, H, k, L, seed=300 + rows, empty_rows=(1,))
+    fn = sa.sparse_mla_decode if fn_name == "decode" else sa.sparse_mla_prefill
+    lse32 = torch.empty(cfg.rows, cfg.H, dtype=torch.float32, device=DEV)
+    lse16 = torch.empty_like(lse32)
+    o32 = fn(inp["q_lat"], inp["q_rope"], inp["c_cache"], inp["kr_cache"], idx, cfg.scale, cfg.pages_per_seq,
+             page_table=inp["page_table"], lse=lse32)
+    o16 = torch.empty(cfg.rows, cfg.H, cfg.d_c, dtype=torch.bfloat16, device=DEV)
+    fn(inp["q_lat"], inp["q_rope"], inp["c_cache"], inp["kr_cache"], idx, cfg.scale, cfg.pages_per_seq,
+       page_table=inp["page_table"], out=o16, lse=lse16)
+    torch.cuda.synchronize()
+    assert torch.equal(o16, o32.to(torch.bfloat16))
+    assert torch.equal(lse16, lse32)
+    out, lse = _oracle(cfg, inp, idx)
+    assert_attention_close(o16.float().cpu().numpy(), out)
+    assert sa.check_device_error() == 0

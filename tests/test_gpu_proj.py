@@ -56,6 +56,9 @@ def test_up_project_vs_oracle(rows, H):
     # and against the unrounded latent output: within the bf16 input rounding
     ref32 = oracle.up_project(_f64(U_V), _f64(o_lat))
     assert np.abs(got - ref32).max() <= 2e-3
+    # a bf16 latent output (the _bf16 attention calls) gives the same product bit for bit
+    got_b = sa.mla_up_project(o_lat.to(torch.bfloat16), U_V)
+    assert np.array_equal(_f64(got_b), got)
     assert sa.check_device_error() == 0
 
 
