@@ -66,13 +66,13 @@ def test_csa_decode_bytes():
 
 def test_step_working_set_and_e2e_flush_rule():
     """Distinct bytes a step reads, which decides whether the end-to-end loop
-    flushes L2 between steps (under twice the 126 MB L2: flush)."""
+    flushes L2 between steps (working set under the 126 MB L2: flush)."""
     import bench
     long_b = bench.step_working_set(W.LONG, None)
     assert long_b == 32 * (32768 * 128 + 2048 * 1152) == 209715200
-    assert long_b < 2 * bench.L2_BYTES
+    assert long_b > bench.L2_BYTES  # streams through L2: no flush
     ragged_b = bench.step_working_set(W.RAGGED, None)
-    assert ragged_b == sum(bench.decode_bytes(W.RAGGED)) and ragged_b > 2 * bench.L2_BYTES
+    assert ragged_b == sum(bench.decode_bytes(W.RAGGED)) and ragged_b > bench.L2_BYTES
     prefill_b = bench.step_working_set(W.PREFILL, None)
-    assert prefill_b == 65536 * (128 + 1152)  # the history once, however many query rows read it
-    assert bench.step_working_set(W.NSA, None) == bench.nsa_bytes(W.NSA) < 2 * bench.L2_BYTES
+    assert prefill_b == 65536 * (128 + 1152) < bench.L2_BYTES  # the history once, however many rows read it
+    assert bench.step_working_set(W.NSA, None) == bench.nsa_bytes(W.NSA) < bench.L2_BYTES
