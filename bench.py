@@ -510,6 +510,25 @@ def time_projections(step, K: int, flush, hbm: float):
 E2E_SLOTS = 3  # steps in flight in the end-to-end pipeline
 
 
+def pack_layout(tensors):
+    """(offset, bytes) of each tensor in one packed byte buffer (pieces start
+    on 16-byte boundaries), and the buffer's size."""
+    offs, total = [], 0
+    for t in tensors:
+        nb = t.numel() * t.element_size()
+        offs.append((total, nb))
+        total += (nb + 15) // 16 * 16
+    return offs, total
+
+
+def pack_host(tensors, offs, total):
+    """The tensors' bytes at their offsets in one host uint8 buffer."""
+    buf = torch.zeros(total, dtype=torch.uint8)
+    for t, (o, nb) in zip(tensors, offs):
+        buf[o:o + nb].copy_(t.detach().contiguous().view(-1).view(torch.uint8).cpu())
+    return buf
+
+
 def e2e_steps(step, K: int, flush, flush_each: bool):
     """The step through the public API as a serving loop runs it: every step's
     query inputs are copied in from pinned host memory (packed in one buffer,
@@ -534,17 +553,11 @@ def e2e_steps(step, K: int, flush, flush_each: bool):
     result = step.out
     # two slots when a step's output is large (the prefill chunk's is 1 GB)
     S = E2E_SLOTS if result.numel() * result.element_size() <= (256 << 20) else 2
-    # the step's inputs packed in one pinned buffer (16-byte aligned pieces):
-    # one host-to-device copy per step, split into the step's tensors on the device
-    offs, total = {}, 0
-    for n in names:
-        nb = inp[n].numel() * inp[n].element_size()
-        offs[n] = (total, nb)
-        total += (nb + 15) // 16 * 16
-    host_in = torch.empty(total, dtype=torch.uint8).pin_memory()
-    for n in names:
-        o, nb = offs[n]
-        host_in[o:o + nb].copy_(inp[n].contiguous().view(-1).view(torch.uint8).cpu())
+    # the step's inputs packed in one pinned buffer: one host-to-device copy
+    # per step, split into the step's tensors on the device
+    offs, total = pack_layout([inp[n] for n in names])
+    offs = dict(zip(names, offs))
+    host_in = pack_host([inp[n] for n in names], offs.values(), total).pin_memory()
     host_out = [torch.empty(result.shape, dtype=result.dtype).pin_memory() for _ in range(S)]
     dev_in = [torch.empty(total, dtype=torch.uint8, device=result.device) for _ in range(S)]
     dev_out = [torch.empty_like(result) for _ in range(S)]

@@ -76,3 +76,25 @@ def test_step_working_set_and_e2e_flush_rule():
     prefill_b = bench.step_working_set(W.PREFILL, None)
     assert prefill_b == 65536 * (128 + 1152) < bench.L2_BYTES  # the history once, however many rows read it
     assert bench.step_working_set(W.NSA, None) == bench.nsa_bytes(W.NSA) < bench.L2_BYTES
+
+
+def test_e2e_input_packing():
+    """The end-to-end loop's packed input buffer: every piece starts on a
+    16-byte boundary, pieces do not overlap, and each tensor's bytes come back
+    unchanged from its slice (fp32, e4m3 and bf16 pieces of odd sizes)."""
+    import torch
+    import bench
+    g = torch.Generator().manual_seed(5)
+    ts = [torch.randn(3, 5, generator=g),
+          torch.randint(-8, 9, (7,), generator=g).to(torch.float32).to(torch.float8_e4m3fn),
+          torch.randn(2, 3, generator=g).to(torch.bfloat16),
+          torch.randn(33, generator=g)]
+    offs, total = bench.pack_layout(ts)
+    assert all(o % 16 == 0 for o, _ in offs)
+    ends = [o + nb for o, nb in offs]
+    assert all(ends[i] <= offs[i + 1][0] for i in range(len(ts) - 1)) and ends[-1] <= total
+    buf = bench.pack_host(ts, offs, total)
+    for t, (o, nb) in zip(ts, offs):
+        back = torch.empty_like(t)
+        back.view(-1).view(torch.uint8).copy_(buf[o:o + nb])
+        assert torch.equal(back.view(-1).view(torch.uint8), t.view(-1).view(torch.uint8))
