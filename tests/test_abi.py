@@ -89,12 +89,10 @@ def _mla(L, fn, **kw):
     a.update(kw)
     args = [a["ql"], a["qr"], a["c"], a["cld"], a["kr"], a["krld"], a["pool"], a["pt"], a["pps"], a["sor"],
             a["idx"], a["rows"], a["H"], a["k"], a["dc"], a["dR"], a["scale"], a["out"], a["lse"]]
-    if fn == "decode":
-        return L.sa_sparse_mla_decode(*args, None, 0, None)
-    return L.sa_sparse_mla_prefill(*args, None, 0, None)
+    return getattr(L, f"sa_sparse_mla_{fn}")(*args, None, 0, None)
 
 
-@pytest.mark.parametrize("fn", ["decode", "prefill"])
+@pytest.mark.parametrize("fn", ["decode", "prefill", "decode_bf16", "prefill_bf16"])
 def test_sparse_mla_validation(L, fn):
     assert _mla(L, fn, rows=0) == sa.SA_OK
     assert _mla(L, fn, k=0) == sa.SA_EINVAL
@@ -212,3 +210,52 @@ def test_static_scratch_size_matches_the_header():
     assert m, "definition not found"
     expr = m.group(1).replace("(size_t)", "")
     assert eval(expr, {}) == sa.STATIC_SCRATCH_BYTES
+
+
+def test_candidate_path_validation(L):
+    """sa_index_candidates / sa_topk_from_candidates: bad counts, missing or
+    misaligned buffers, a candidate row shorter than the page table's reach,
+    and shapes off the tensor-core indexer are refused on the host."""
+    f = L.sa_index_candidates
+    good = dict(q=FAKE, w=FAKE, k=FAKE, pool=4, dt=sa.SA_E4M3, pt=None, pps=4, nv=FAKE, rows=2, H_I=64, d_I=128,
+                topk=64, ld=256, cand=FAKE, cnt=FAKE, hist=FAKE)
+
+    def call(**kw):
+        a = {**good, **kw}
+        return f(a["q"], a["w"], a["k"], a["pool"], a["dt"], a["pt"], a["pps"], a["nv"], a["rows"], a["H_I"],
+                 a["d_I"], a["topk"], a["ld"], a["cand"], a["cnt"], a["hist"], None)
+
+    assert call(rows=0) == sa.SA_OK
+    assert call(rows=-1) == sa.SA_EINVAL
+    assert call(topk=0) == sa.SA_EINVAL
+    assert call(ld=255) == sa.SA_EINVAL                 # shorter than pages_per_seq * 64
+    assert call(cand=None) == sa.SA_EINVAL
+    assert call(cnt=None) == sa.SA_EINVAL
+    assert call(hist=None) == sa.SA_EINVAL
+    assert call(hist=MISALIGNED) == sa.SA_EINVAL        # the bound is read in 16-byte pieces
+    assert call(q=MISALIGNED) == sa.SA_EINVAL
+    assert call(dt=sa.SA_F32) == sa.SA_EUNSUPPORTED     # the tensor-core indexer only
+    assert call(d_I=64) == sa.SA_EUNSUPPORTED
+    assert call(rows=4097) == sa.SA_EUNSUPPORTED
+    assert call(pps=4097, ld=4097 * 64) == sa.SA_EUNSUPPORTED  # rows longer than the Top-K's bitmaps
+
+    g = L.sa_topk_from_candidates
+    assert g(FAKE, 256, FAKE, FAKE, 0, 8, FAKE, FAKE, None) == sa.SA_OK
+    assert g(FAKE, 256, FAKE, FAKE, -1, 8, FAKE, FAKE, None) == sa.SA_EINVAL
+    assert g(FAKE, 256, FAKE, FAKE, 2, 0, FAKE, FAKE, None) == sa.SA_EINVAL
+    assert g(FAKE, 0, FAKE, FAKE, 2, 8, FAKE, FAKE, None) == sa.SA_EINVAL
+    assert g(None, 256, FAKE, FAKE, 2, 8, FAKE, FAKE, None) == sa.SA_EINVAL
+    assert g(FAKE, 256, FAKE, FAKE, 2, 8, None, FAKE, None) == sa.SA_EINVAL
+    assert g(ctypes.c_void_p(0x1004), 256, FAKE, FAKE, 2, 8, FAKE, FAKE, None) == sa.SA_EINVAL
+    assert g(FAKE, 262144 + 64, FAKE, FAKE, 2, 8, FAKE, FAKE, None) == sa.SA_EUNSUPPORTED
+
+
+@pytest.mark.parametrize("name", ["sa_mla_up_project", "sa_mla_up_project_bf16"])
+def test_up_project_validation(L, name):
+    f = getattr(L, name)
+    assert f(FAKE, FAKE, 0, 8, 512, 128, FAKE, None) == sa.SA_OK
+    assert f(FAKE, FAKE, -1, 8, 512, 128, FAKE, None) == sa.SA_EINVAL
+    assert f(None, FAKE, 2, 8, 512, 128, FAKE, None) == sa.SA_EINVAL
+    assert f(MISALIGNED, FAKE, 2, 8, 512, 128, FAKE, None) == sa.SA_EINVAL
+    assert f(FAKE, FAKE, 2, 8, 500, 128, FAKE, None) == sa.SA_EUNSUPPORTED   # d_c not a multiple of 64
+    assert f(FAKE, FAKE, 2, 8, 512, 100, FAKE, None) == sa.SA_EUNSUPPORTED   # d_v not a multiple of 128
